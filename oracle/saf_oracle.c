@@ -1,0 +1,282 @@
+/*
+ * fp64 CPU oracle for the mixed-head causal attention layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this file's library.  The GPU product
+ * path never calls it and shares no code, header or table with it.
+ *
+ * Everything here is the plain definition, written as straight loops over
+ * one (batch, head) slice at a time, in double precision:
+ *
+ *  - Ordinary heads: causal softmax attention,
+ *      A = softmax_causal(Q K^T / sqrt(d_h)),  Z = A V
+ *    ("When Can Attention Heads Be Statically Defined?" reading notes,
+ *    section 一, the equation for A and Z).  The row log-sum-exp of the
+ *    scaled scores is returned as lse.
+ *  - Replaced heads: the compact fixed pattern of Eq. (3) of the same page
+ *    (section 二.3):  P(i,j) = exp(alpha(j) + rho(i-j)) / Z(i) for j <= i,
+ *    zero for j > i, with Z(i) = sum_{k<=i} exp(alpha(k) + rho(i-k)).
+ *    Indices are 0-based here: j, k in [0, i], distance i-j in [0, T-1].
+ *    lse returns log Z(i).
+ *  - Backward (section 二.4 of the same page): replaced heads only get
+ *    dV = P^T dO (their pattern is a frozen buffer with no Q/K path, so dQ
+ *    and dK are zero); ordinary heads get the textbook softmax-attention
+ *    gradients dV = P^T dO, dP = dO V^T, dS = P o (dP - rowsum(P o dP)),
+ *    dQ = s dS K, dK = s dS^T Q with s = 1/sqrt(d_h).
+ *
+ * Max-shifts (subtracting the row maximum before exp) are the only numerical
+ * device used; they leave every result unchanged mathematically.  A row
+ * whose every term is -inf (possible only with -inf alpha/rho) yields an all
+ * zero output row and lse = -inf.
+ *
+ * Worker threads take whole slices from a shared counter; each slice is
+ * computed start to finish by one thread with no blocking or reordering.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Eq. (3): log Z(i) = log sum_{k<=i} exp(a[k] + r[i-k]), for one head. */
+void oracle_lognorm(int T, const double *a, const double *r, double *logz)
+{
+    for (int i = 0; i < T; ++i) {
+        double L = -INFINITY;
+        for (int k = 0; k <= i; ++k) {
+            double e = a[k] + r[i - k];
+            if (e > L) L = e;
+        }
+        if (L == -INFINITY) {
+            logz[i] = -INFINITY;
+            continue;
+        }
+        double s = 0.0;
+        for (int k = 0; k <= i; ++k) s += exp(a[k] + r[i - k] - L);
+        logz[i] = L + log(s);
+    }
+}
+
+/* ---------------------------------------------------------------- forward */
+
+static void fwd_replaced(int T, int d, const double *a, const double *r,
+                         const double *v, double *o, double *lse, double *logz)
+{
+    oracle_lognorm(T, a, r, logz);
+    for (int i = 0; i < T; ++i) {
+        double *oi = o + (size_t)i * d;
+        for (int c = 0; c < d; ++c) oi[c] = 0.0;
+        lse[i] = logz[i];
+        if (logz[i] == -INFINITY) continue;
+        for (int j = 0; j <= i; ++j) {
+            double p = exp(a[j] + r[i - j] - logz[i]);
+            const double *vj = v + (size_t)j * d;
+            for (int c = 0; c < d; ++c) oi[c] += p * vj[c];
+        }
+    }
+}
+
+static void fwd_ordinary(int T, int d, const double *q, const double *k,
+                         const double *v, double *o, double *lse, double *srow)
+{
+    const double scale = 1.0 / sqrt((double)d);
+    for (int i = 0; i < T; ++i) {
+        const double *qi = q + (size_t)i * d;
+        double m = -INFINITY;
+        for (int j = 0; j <= i; ++j) {
+            const double *kj = k + (size_t)j * d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];
+            srow[j] = scale * dot;
+            if (srow[j] > m) m = srow[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j <= i; ++j) l += exp(srow[j] - m);
+        double *oi = o + (size_t)i * d;
+        for (int c = 0; c < d; ++c) oi[c] = 0.0;
+        for (int j = 0; j <= i; ++j) {
+            double p = exp(srow[j] - m) / l;
+            const double *vj = v + (size_t)j * d;
+            for (int c = 0; c < d; ++c) oi[c] += p * vj[c];
+        }
+        lse[i] = m + log(l);
+    }
+}
+
+/* --------------------------------------------------------------- backward */
+
+static void bwd_replaced(int T, int d, const double *a, const double *r,
+                         const double *dout, double *dq, double *dk, double *dv,
+                         double *logz)
+{
+    oracle_lognorm(T, a, r, logz);
+    memset(dq, 0, sizeof(double) * (size_t)T * d);
+    memset(dk, 0, sizeof(double) * (size_t)T * d);
+    memset(dv, 0, sizeof(double) * (size_t)T * d);
+    for (int i = 0; i < T; ++i) {
+        if (logz[i] == -INFINITY) continue;
+        const double *doi = dout + (size_t)i * d;
+        for (int j = 0; j <= i; ++j) {
+            double p = exp(a[j] + r[i - j] - logz[i]);
+            double *dvj = dv + (size_t)j * d;
+            for (int c = 0; c < d; ++c) dvj[c] += p * doi[c];
+        }
+    }
+}
+
+static void bwd_ordinary(int T, int d, const double *q, const double *k,
+                         const double *v, const double *dout, double *dq,
+                         double *dk, double *dv, double *prow, double *dprow)
+{
+    const double scale = 1.0 / sqrt((double)d);
+    memset(dq, 0, sizeof(double) * (size_t)T * d);
+    memset(dk, 0, sizeof(double) * (size_t)T * d);
+    memset(dv, 0, sizeof(double) * (size_t)T * d);
+    for (int i = 0; i < T; ++i) {
+        const double *qi = q + (size_t)i * d;
+        const double *doi = dout + (size_t)i * d;
+        /* row i of P = softmax over j <= i of the scaled scores */
+        double m = -INFINITY;
+        for (int j = 0; j <= i; ++j) {
+            const double *kj = k + (size_t)j * d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];
+            prow[j] = scale * dot;
+            if (prow[j] > m) m = prow[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j <= i; ++j) {
+            prow[j] = exp(prow[j] - m);
+            l += prow[j];
+        }
+        for (int j = 0; j <= i; ++j) prow[j] /= l;
+        /* dP = dO V^T (row i), and the row term sum_j P dP */
+        double D = 0.0;
+        for (int j = 0; j <= i; ++j) {
+            const double *vj = v + (size_t)j * d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += doi[c] * vj[c];
+            dprow[j] = dot;
+            D += prow[j] * dot;
+        }
+        double *dqi = dq + (size_t)i * d;
+        for (int j = 0; j <= i; ++j) {
+            double ds = prow[j] * (dprow[j] - D);
+            const double *kj = k + (size_t)j * d;
+            double *dkj = dk + (size_t)j * d;
+            double *dvj = dv + (size_t)j * d;
+            for (int c = 0; c < d; ++c) {
+                dqi[c] += scale * ds * kj[c];
+                dkj[c] += scale * ds * qi[c];
+                dvj[c] += prow[j] * doi[c];
+            }
+        }
+    }
+}
+
+/* ----------------------------------------------------- slice thread pool */
+
+typedef struct {
+    int n, T, d, is_bwd;
+    const uint8_t *replaced;
+    const double *q, *k, *v, *dout, *a, *r;
+    double *o, *lse, *dq, *dk, *dv;
+    int next;
+    int failed;
+    pthread_mutex_t mu;
+} job_t;
+
+static void *worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    const size_t TD = (size_t)J->T * J->d;
+    double *buf1 = (double *)malloc(sizeof(double) * (size_t)(J->T > 0 ? J->T : 1));
+    double *buf2 = (double *)malloc(sizeof(double) * (size_t)(J->T > 0 ? J->T : 1));
+    if (!buf1 || !buf2) {
+        pthread_mutex_lock(&J->mu);
+        J->failed = 1;
+        pthread_mutex_unlock(&J->mu);
+        free(buf1);
+        free(buf2);
+        return NULL;
+    }
+    for (;;) {
+        pthread_mutex_lock(&J->mu);
+        int s = J->next++;
+        pthread_mutex_unlock(&J->mu);
+        if (s >= J->n) break;
+        const double *a = J->a + (size_t)s * J->T;
+        const double *r = J->r + (size_t)s * J->T;
+        if (!J->is_bwd) {
+            if (J->replaced[s])
+                fwd_replaced(J->T, J->d, a, r, J->v + s * TD, J->o + s * TD,
+                             J->lse + (size_t)s * J->T, buf1);
+            else
+                fwd_ordinary(J->T, J->d, J->q + s * TD, J->k + s * TD, J->v + s * TD,
+                             J->o + s * TD, J->lse + (size_t)s * J->T, buf1);
+        } else {
+            if (J->replaced[s])
+                bwd_replaced(J->T, J->d, a, r, J->dout + s * TD, J->dq + s * TD,
+                             J->dk + s * TD, J->dv + s * TD, buf1);
+            else
+                bwd_ordinary(J->T, J->d, J->q + s * TD, J->k + s * TD, J->v + s * TD,
+                             J->dout + s * TD, J->dq + s * TD, J->dk + s * TD,
+                             J->dv + s * TD, buf1, buf2);
+        }
+    }
+    free(buf1);
+    free(buf2);
+    return NULL;
+}
+
+static int run(job_t *J, int n_threads)
+{
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > J->n) n_threads = J->n > 0 ? J->n : 1;
+    J->next = 0;
+    J->failed = 0;
+    pthread_mutex_init(&J->mu, NULL);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    if (!th) return -1;
+    int started = 0;
+    for (int t = 0; t < n_threads; ++t) {
+        if (pthread_create(&th[t], NULL, worker, J) != 0) break;
+        ++started;
+    }
+    if (started == 0) worker(J);
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->mu);
+    return J->failed ? -1 : 0;
+}
+
+/*
+ * n independent slices.  replaced[n]; q,k,v [n,T,d]; a,r [n,T] (the pattern
+ * row of each slice's head, read only for replaced slices); o [n,T,d];
+ * lse [n,T].  Returns 0, or -1 on allocation failure.
+ */
+int oracle_fwd_slices(int n, int T, int d, const uint8_t *replaced,
+                      const double *q, const double *k, const double *v,
+                      const double *a, const double *r, double *o, double *lse,
+                      int n_threads)
+{
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    J.n = n; J.T = T; J.d = d; J.is_bwd = 0; J.replaced = replaced;
+    J.q = q; J.k = k; J.v = v; J.a = a; J.r = r; J.o = o; J.lse = lse;
+    return run(&J, n_threads);
+}
+
+/* Same slicing; dout [n,T,d] in, dq/dk/dv [n,T,d] out. */
+int oracle_bwd_slices(int n, int T, int d, const uint8_t *replaced,
+                      const double *q, const double *k, const double *v,
+                      const double *dout, const double *a, const double *r,
+                      double *dq, double *dk, double *dv, int n_threads)
+{
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    J.n = n; J.T = T; J.d = d; J.is_bwd = 1; J.replaced = replaced;
+    J.q = q; J.k = k; J.v = v; J.dout = dout; J.a = a; J.r = r;
+    J.dq = dq; J.dk = dk; J.dv = dv;
+    return run(&J, n_threads);
+}

@@ -1,0 +1,109 @@
+"""The oracle against what the pages and the mathematics fix (no GPU).
+
+Each pin is a check in ``oracle_pins``; the mutation test below plants
+plausible mistakes in a copy of the oracle's C source (on the CPU) and
+requires that some pin rejects every one of them.
+"""
+import json
+import os
+import shutil
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_pins as pins
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.default()
+
+
+@pytest.mark.parametrize("check", pins.ALL_CHECKS, ids=lambda c: c.__name__)
+def test_pin(orc, check):
+    check(orc)
+
+
+# (description, exact snippet in saf_oracle.c, replacement, occurrence index)
+MUTANTS = [
+    ("replaced: diagonal dropped",
+     "for (int j = 0; j <= i; ++j) {\n            double p = exp(a[j] + r[i - j] - logz[i]);\n            const double *vj",
+     "for (int j = 0; j < i; ++j) {\n            double p = exp(a[j] + r[i - j] - logz[i]);\n            const double *vj", 0),
+    ("replaced: a and r roles swapped",
+     "double p = exp(a[j] + r[i - j] - logz[i]);\n            const double *vj",
+     "double p = exp(a[i - j] + r[j] - logz[i]);\n            const double *vj", 0),
+    ("lognorm: distance index wrong",
+     "s += exp(a[k] + r[i - k] - L);", "s += exp(a[k] + r[k] - L);", 0),
+    ("lognorm: max shift not added back",
+     "logz[i] = L + log(s);", "logz[i] = log(s);", 0),
+    ("ordinary fwd: scale dropped",
+     "srow[j] = scale * dot;", "srow[j] = dot;", 0),
+    ("ordinary fwd: lse misses the max",
+     "lse[i] = m + log(l);", "lse[i] = log(l);", 0),
+    ("ordinary fwd: causal bound off by one",
+     "for (int j = 0; j <= i; ++j) {\n            const double *kj = k + (size_t)j * d;\n            double dot = 0.0;\n            for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];\n            srow[j]",
+     "for (int j = 0; j <= i && j < T - 1; ++j) {\n            const double *kj = k + (size_t)j * d;\n            double dot = 0.0;\n            for (int c = 0; c < d; ++c) dot += qi[c] * kj[c];\n            srow[j]", 0),
+    ("ordinary bwd: D term dropped",
+     "double ds = prow[j] * (dprow[j] - D);", "double ds = prow[j] * dprow[j];", 0),
+    ("ordinary bwd: dK uses K instead of Q",
+     "dkj[c] += scale * ds * qi[c];", "dkj[c] += scale * ds * kj[c];", 0),
+    ("ordinary bwd: dQ sign flipped",
+     "dqi[c] += scale * ds * kj[c];", "dqi[c] -= scale * ds * kj[c];", 0),
+    ("ordinary bwd: dV uses Q instead of dO",
+     "dvj[c] += prow[j] * doi[c];", "dvj[c] += prow[j] * qi[c];", 0),
+    ("ordinary bwd: scale dropped in dQ",
+     "dqi[c] += scale * ds * kj[c];", "dqi[c] += ds * kj[c];", 0),
+    ("replaced bwd: normaliser of the wrong row",
+     "double p = exp(a[j] + r[i - j] - logz[i]);\n            double *dvj",
+     "double p = exp(a[j] + r[i - j] - logz[j]);\n            double *dvj", 0),
+    ("replaced bwd: dQ not cleared",
+     "memset(dq, 0, sizeof(double) * (size_t)T * d);\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz",
+     "for (int c = 0; c < T * d; ++c) dq[c] = 1e-3 * c;\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz", 0),
+]
+
+
+def _replace_nth(text, old, new, n):
+    start = -1
+    for _ in range(n + 1):
+        start = text.find(old, start + 1)
+        assert start >= 0, f"snippet not found: {old!r}"
+    return text[:start] + new + text[start + len(old):]
+
+
+@pytest.mark.parametrize("desc,old,new,nth", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(desc, old, new, nth):
+    src = open(oracle.SOURCE).read()
+    mutated = _replace_nth(src, old, new, nth)
+    assert mutated != src
+    tmp = tempfile.mkdtemp(prefix="oracle_mutant_")
+    try:
+        csrc = os.path.join(tmp, "m.c")
+        with open(csrc, "w") as f:
+            f.write(mutated)
+        mut = oracle.Oracle(oracle.compile_library(csrc, os.path.join(tmp, "m.so")))
+        caught = []
+        for check in pins.ALL_CHECKS:
+            try:
+                check(mut)
+            except AssertionError:
+                caught.append(check.__name__)
+        assert caught, f"no pin rejects the planted mistake: {desc}"
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+
+
+def test_golden_regression(orc):
+    """Frozen oracle outputs on a tiny mixed case (tests/golden/make_golden.py)."""
+    path = os.path.join(HERE, "golden", "tiny_mixed_layer.json")
+    with open(path) as f:
+        g = json.load(f)
+    arr = {k: np.asarray(v, dtype=np.float64) for k, v in g["inputs"].items()}
+    o, lse = orc.fwd(arr["q"], arr["k"], arr["v"], arr["alpha"], arr["rho"], arr["mask"].astype(np.uint8))
+    dq, dk, dv = orc.bwd(arr["q"], arr["k"], arr["v"], arr["do"], arr["alpha"], arr["rho"],
+                         arr["mask"].astype(np.uint8))
+    for name, got in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+        np.testing.assert_allclose(got, np.asarray(g["outputs"][name]), rtol=1e-12, atol=1e-13, err_msg=name)
