@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the mixed-head causal attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step is the whole hot path on one batch: the forward call (replaced-head
+log-normalisers + fused forward) and the backward call (log-normalisers,
+row terms, fused backward), all through the C ABI, inputs resident in HBM.
+Default workload: the 124M-shape layer B=8, H=12 (3 replaced), T=4096,
+d_h=64, forward + backward.
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank processes
+its own batch shard of the same shape (weak scaling, no collective on the
+data path); the time is the max over ranks.  `--impl reference` times the
+fp64 CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from mixed_head_causal_b200 import inputs as I  # noqa: E402
+
+DEFAULT_WORKLOAD = "124m_b8_t4096_r25"
+METRIC = "mixed-head causal attn fwd+bwd tokens/s & TFLOP/s on 1 B200; % of bf16 TC peak"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--grad-dtype", default="bf16", choices=["bf16", "fp32"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(loaded), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in sorted(paths):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(w, seed=0):
+    """A bounded sample of (b, h) slices with the workload's head-kind mix."""
+    mask = I.replaced_mask(w, seed).numpy()
+    rep = [h for h in range(w.H) if mask[h]]
+    ordn = [h for h in range(w.H) if not mask[h]]
+    # keep the ordinary:replaced ratio of the layer (e.g. 3:1 for 9:3)
+    from math import gcd
+    g = gcd(len(ordn), len(rep)) if rep and ordn else 1
+    n_o, n_r = (len(ordn) // g, len(rep) // g) if rep and ordn else (min(4, len(ordn)), min(4, len(rep)))
+    slices = [(0, ordn[i % len(ordn)]) for i in range(n_o)] + [(0, rep[i % len(rep)]) for i in range(n_r)]
+    return slices
+
+
+def run_oracle_sample(w, slices, seed=0, threads=None):
+    import numpy as np
+    import oracle
+    a, r = I.make_pattern(w, seed)
+    mask = I.replaced_mask(w, seed).numpy()
+    q = torch.stack([I.make_slice(w, seed, "q", b, h) for b, h in slices])
+    k = torch.stack([I.make_slice(w, seed, "k", b, h) for b, h in slices])
+    v = torch.stack([I.make_slice(w, seed, "v", b, h) for b, h in slices])
+    ar = np.stack([a[h].double().numpy() for _, h in slices])
+    rr = np.stack([r[h].double().numpy() for _, h in slices])
+    rep = [int(mask[h]) for _, h in slices]
+    threads = threads or oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.fwd_slices(q, k, v, ar, rr, rep, threads)
+    if w.backward:
+        do = torch.stack([I.make_slice(w, seed, "do", b, h) for b, h in slices])
+        oracle.bwd_slices(q, k, v, do, ar, rr, rep, threads)
+    dt = time.perf_counter() - t0
+    frac = len(slices) / float(w.B * w.H)
+    return dt, frac, min(threads, len(slices))
+
+
+def cpu_baseline(w):
+    slices = oracle_sample(w)
+    dt, frac, cores = run_oracle_sample(w, slices)
+    return {"value": w.tokens * frac / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(slices)} of {w.B * w.H} (batch, head) slices of {w.name} (same head-kind mix), "
+                      f"fwd{'+bwd' if w.backward else ''}, {dt:.1f} s, scaled by slice count"}
+
+
+def reference_arm(args, world, rank):
+    w = I.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    slices = oracle_sample(w)
+    for _ in range(args.warmup):
+        run_oracle_sample(w, slices)
+    times = []
+    for _ in range(args.steps):
+        dt, frac, cores = run_oracle_sample(w, slices)
+        times.append(dt)
+    total = sum(times)
+    value = w.tokens * frac * args.steps / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_h": w.d,
+                       "n_replaced": len(I.replaced_heads(w))},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{len(slices)} of {w.B * w.H} (batch, head) slices per step, "
+                                       "scaled by slice count"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def algorithmic_flops_per_launch(kernel: str, w, n_r: int) -> float:
+    """Algorithmic flops of one launch of `kernel` on workload w (causal
+    T^2/2 convention; one unit = d_h * T^2 flops per (batch, head) = one
+    T x T x d_h causal contraction)."""
+    n_o = w.H - n_r
+    unit = float(w.d) * w.T * w.T * w.B
+    table = {
+        "fwd_mma": unit * (2 * n_o + n_r),     # QK^T + PV (ordinary), PV (replaced)
+        "fwd_tc": unit * (2 * n_o + n_r),
+        "dkdv_mma": unit * (4 * n_o + n_r),    # S recompute, dV, dP, dK (ordinary); dV (replaced)
+        "dq_mma": unit * n_o,                  # dQ (its S/dP recompute is not algorithmic)
+        "bwd_tc": unit * (5 * n_o + n_r),
+    }
+    return table.get(kernel, 0.0)
+
+
+def our_arm(args, world, rank, local):
+    from mixed_head_causal_b200 import saf
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the product path has no CPU fallback)")
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS[args.workload]
+    gd = torch.bfloat16 if args.grad_dtype == "bf16" else torch.float32
+    seed = rank  # each rank's shard of the global batch
+    host = I.make_inputs(w, seed, pin=True, threads=min(16, os.cpu_count() or 1))
+    mask = host["mask"]
+    n_r = int(mask.sum())
+    x = {k: (v.to(dev, non_blocking=True) if k != "mask" else v) for k, v in host.items()}
+    B, H, T, d = w.B, w.H, w.T, w.d
+    o = torch.empty(B, H, T, d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, T, dtype=torch.float32, device=dev)
+    dq = torch.empty(B, H, T, d, dtype=gd, device=dev)
+    dk = torch.empty_like(dq)
+    dv = torch.empty_like(dq)
+    ws_f = saf.new_workspace(B, H, T, dev, backward=False)
+    ws_b = saf.new_workspace(B, H, T, dev, backward=True) if w.backward else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, out=o, lse=lse, workspace=ws_f)
+        if w.backward:
+            saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask,
+                               grad_dtype=gd, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+
+    torch.cuda.synchronize()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- headline: device time of K steps, inputs resident (all > L2 in total)
+    launches0 = saf.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    launches = saf.launch_count() - launches0
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    ms_step = ms_total / args.steps
+    tokens = w.tokens * world
+    value = tokens / (ms_step * 1e-3)
+    fl = I.flops(w)
+    tflops = fl["total"] * world / (ms_step * 1e-3) / 1e12
+
+    # ---- per-kernel timing (separate pass, same steps, events around each launch)
+    prof_steps = min(args.steps, 20)
+    per_launch = 6 if w.backward else 2
+    saf.profile_enable(prof_steps * (per_launch + 4))
+    for _ in range(prof_steps):
+        step()
+    torch.cuda.synchronize()
+    recs = saf.profile_read()
+    saf.profile_enable(0)
+    per_kernel = {}
+    for name, ms in recs:
+        e = per_kernel.setdefault(name, [0, 0.0])
+        e[0] += 1
+        e[1] += ms
+    total_ms = sum(v[1] for v in per_kernel.values()) or 1.0
+    kernels = {k: {"launches": v[0], "avg_ms": v[1] / v[0], "share": v[1] / total_ms} for k, v in per_kernel.items()}
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    pk = peaks()
+    dom_flops = algorithmic_flops_per_launch(dom, w, n_r)
+    achieved = dom_flops / (kernels[dom]["avg_ms"] * 1e-3) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tj = json.load(f)
+        csrc = os.path.join(ROOT, "mixed_head_causal_b200", "csrc")
+        cur = source_hash([os.path.join(csrc, f) for f in os.listdir(csrc)])
+        ent = tj.get(dom)
+        if ent and ent.get("source_hash") == cur and ent.get("workload") == w.name:
+            traffic = ent.get("bytes_per_launch")
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "traffic": traffic, "kernel": dom,
+                "peak_src": f"{pk['src']} (burst bf16 dense)"}
+
+    # ---- end to end: pinned host -> device, both calls, device -> host of the outputs
+    e2e = None
+    if not args.no_e2e:
+        outs_host = {"o": torch.empty(B, H, T, d, dtype=torch.bfloat16, pin_memory=True)}
+        if w.backward:
+            for k_ in ("dq", "dk", "dv"):
+                outs_host[k_] = torch.empty(B, H, T, d, dtype=gd, pin_memory=True)
+        in_keys = ["q", "k", "v"] + (["do"] if w.backward else [])
+        h2d = sum(host[k_].numel() * host[k_].element_size() for k_ in in_keys)
+        h2d += sum(host[k_].numel() * 4 for k_ in ("alpha", "rho"))
+        d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+        dev_out = {"o": o, "dq": dq, "dk": dk, "dv": dv}
+        e2e_steps = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            for k_ in in_keys + ["alpha", "rho"]:
+                x[k_].copy_(host[k_], non_blocking=True)
+            step()
+            for k_, t in outs_host.items():
+                t.copy_(dev_out[k_], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+        e2e = {"value": tokens / (e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "tflops": tflops, "tflops_frac_of_peak": tflops / pk["bf16_tflops"],
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_h": w.d, "n_replaced": n_r,
+                       "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+                       "passes": "fwd+bwd" if w.backward else "fwd", "grad_dtype": args.grad_dtype,
+                       "l2": "inputs larger than L2 (no flush)",
+                       "flops_per_step": fl["total"] * world},
+            "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
+            "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            reference_arm(args, world, rank)
+        else:
+            our_arm(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

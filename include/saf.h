@@ -1,0 +1,174 @@
+/*
+ * saf.h — C ABI of the B200 (sm_100a) mixed-head causal attention library
+ * (libsaf.so).
+ *
+ * The layer is the one described in "When Can Attention Heads Be Statically
+ * Defined?" (Selective Attention Freezing).  In one layer:
+ *   - an ORDINARY head computes causal softmax attention
+ *       A = softmax_causal(Q K^T / sqrt(d_h)),  O = A V
+ *     (reading notes, section 一, the first displayed equation);
+ *   - a REPLACED head mixes the current V with a frozen causal pattern rebuilt
+ *     from two length-T vectors, the absolute-position preference a and the
+ *     relative-distance preference r:
+ *       P(i,j) = exp(a[j] + r[i-j]) / Z(i)  for j <= i, 0 for j > i,
+ *       Z(i)   = sum_{k<=i} exp(a[k] + r[i-k]),        O = P V
+ *     (Eq. (3), section 二.3; indices are 0-based here, so the distance i-j
+ *     runs over 0..T-1 and both vectors have length T);
+ *   - the backward gives dQ, dK, dV for ordinary heads, and only dV = P^T dO
+ *     for replaced heads (section 二.4: the pattern is a frozen buffer; the
+ *     head's query/key path is gone, so dQ = dK = 0 there).
+ *
+ * Conventions shared by every entry point
+ *   Layout     Q, K, V, O, dO, dQ, dK, dV: contiguous row-major [B, H, T, d_h]
+ *              (d_h fastest), bf16 (IEEE bfloat16 bit patterns) unless stated.
+ *              lse: [B, H, T] fp32.  a, r, logz: [H, T] fp32; rows of ordinary
+ *              heads are never read (they may hold anything, NaN included).
+ *              d_h must be 64 (SAF_ERR_UNSUPPORTED otherwise).  Any T >= 1.
+ *   Memory     Every tensor pointer is a DEVICE pointer on the current CUDA
+ *              device, 16-byte aligned.  replaced_mask is a HOST array of H
+ *              bytes (nonzero = replaced head), read only during the call.
+ *              The caller owns all buffers, including the workspace; the
+ *              library allocates no device memory in these calls.
+ *   Streams    `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *              default stream).  Calls enqueue work and return; results are
+ *              ready when the stream reaches that point.
+ *   Errors     Argument errors are detected on the host before anything is
+ *              enqueued and return SAF_ERR_INVALID_ARG / SAF_ERR_UNSUPPORTED /
+ *              SAF_ERR_WORKSPACE.  A failed launch returns SAF_ERR_CUDA.
+ *              Device-side waits are bounded; one that gives up records an
+ *              error word in the workspace, which saf_device_status reports
+ *              as SAF_ERR_TIMEOUT.
+ *   Outputs    Always overwritten, never accumulated into.  Inputs and outputs
+ *              must not alias.  Calls that share a workspace must not overlap
+ *              on the GPU.
+ *   Empty      B == 0, H == 0 or T == 0 is valid and enqueues nothing.
+ */
+#ifndef SAF_H_
+#define SAF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAF_API __attribute__((visibility("default")))
+#else
+#define SAF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum saf_status {
+    SAF_OK = 0,
+    SAF_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, overflow */
+    SAF_ERR_UNSUPPORTED = 2, /* d_h != 64, or grad_dtype not 0/1           */
+    SAF_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
+    SAF_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed        */
+    SAF_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up          */
+} saf_status;
+
+/* Human-readable name of a status code (static string; never NULL). */
+SAF_API const char *saf_status_string(int status);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+SAF_API int saf_version(void);
+
+/*
+ * Bytes of device workspace that saf_mixed_attn_fwd (is_bwd = 0) or
+ * saf_mixed_attn_bwd (is_bwd = 1) needs for this shape, whatever the mask.
+ * 0 for an empty problem.  Returns (size_t)-1 for an invalid shape.
+ */
+SAF_API size_t saf_workspace_size(int B, int H, int T, int d_h, int is_bwd);
+
+/*
+ * Row log-normalisers of the replaced heads' patterns (Eq. (3)):
+ *   logz[h, i] = log sum_{k<=i} exp(a[h,k] + r[h,i-k])     (natural log)
+ * for every h with replaced_mask[h] != 0; other rows of logz are untouched.
+ * a, r: [H, T] fp32 device; logz: [H, T] fp32 device output.
+ * The values depend only on a and r, never on the batch, so a caller may
+ * compute them once and pass them to the forward and backward calls.
+ */
+SAF_API saf_status saf_replaced_lognorm(const float *a, const float *r,
+                                const uint8_t *replaced_mask, int H, int T,
+                                float *logz, void *stream);
+
+/*
+ * Forward pass (causal prefill) of one mixed-head layer.
+ *   q, k, v  [B,H,T,d_h] bf16 in.  q and k rows of replaced heads are not read.
+ *   o        [B,H,T,d_h] bf16 out.
+ *   lse      [B,H,T] fp32 out: ordinary heads, log sum_{j<=i} exp(q_i.k_j/sqrt(d_h));
+ *            replaced heads, log Z(i).  The backward needs it.
+ *   a, r     [H,T] fp32 pattern vectors (read for replaced heads only).
+ *   logz     [H,T] fp32 from saf_replaced_lognorm, or NULL to compute it
+ *            inside the call (into the workspace).
+ *   workspace, workspace_bytes: device scratch of at least
+ *            saf_workspace_size(B,H,T,d_h,0) bytes, 256-byte aligned.
+ */
+SAF_API saf_status saf_mixed_attn_fwd(const void *q, const void *k, const void *v,
+                              void *o, float *lse,
+                              const float *a, const float *r, const float *logz,
+                              const uint8_t *replaced_mask,
+                              int B, int H, int T, int d_h,
+                              void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
+ * Backward pass of one mixed-head layer.
+ *   q, k, v, o, dout  [B,H,T,d_h] bf16 in (o and lse as written by the forward).
+ *   lse      [B,H,T] fp32 in.
+ *   a, r, logz as in the forward (logz may be NULL).
+ *   dq, dk, dv  [B,H,T,d_h] out, bf16 (grad_dtype = 0) or fp32 (grad_dtype = 1).
+ *            Replaced heads: dq and dk are written as zeros, dv = P^T dout.
+ *   workspace: at least saf_workspace_size(B,H,T,d_h,1) bytes, 256-byte aligned.
+ * No gradient flows to a, r or logz (they are frozen buffers).
+ */
+SAF_API saf_status saf_mixed_attn_bwd(const void *q, const void *k, const void *v,
+                              const void *o, const void *dout, const float *lse,
+                              const float *a, const float *r, const float *logz,
+                              const uint8_t *replaced_mask,
+                              int B, int H, int T, int d_h,
+                              void *dq, void *dk, void *dv, int grad_dtype,
+                              void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
+ * Reads (synchronously: waits for `stream`) and clears the device error word
+ * that the kernels keep in the first 256 bytes of `workspace`.  Those bytes
+ * must be zero before the workspace is first used (e.g. one cudaMemset); the
+ * kernels only ever set the word, and this call clears it again.
+ * Returns SAF_OK, SAF_ERR_TIMEOUT if a bounded device wait gave up since the
+ * last check, SAF_ERR_WORKSPACE for a missing/short workspace, or SAF_ERR_CUDA.
+ */
+SAF_API saf_status saf_device_status(void *workspace, size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Launch accounting and per-kernel timing (for benchmarks and tracing).
+ * ------------------------------------------------------------------------ */
+
+/* Kernels enqueued by this library since it was loaded (all threads). */
+SAF_API uint64_t saf_launch_count(void);
+
+/*
+ * Starts (max_launches > 0) or stops (0) per-kernel timing.  While on, every
+ * kernel the library enqueues, up to max_launches, is bracketed by two CUDA
+ * events recorded on its stream (host-side event objects created here; no
+ * device memory).  Restarting discards earlier records.
+ */
+SAF_API saf_status saf_profile_enable(int max_launches);
+
+/*
+ * Copies up to n timing records (kernel id and milliseconds between the
+ * bracketing events) of the current profiling session; waits for those
+ * events.  Returns the number of records available, or -1 on a CUDA error.
+ */
+SAF_API int saf_profile_read(int *kernel_ids, float *ms, int n);
+
+/* Name of a kernel id from saf_profile_read ("?" if unknown). */
+SAF_API const char *saf_kernel_name(int kernel_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAF_H_ */

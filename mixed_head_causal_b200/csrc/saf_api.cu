@@ -1,0 +1,175 @@
+// C ABI of libsaf.so (declared in include/saf.h): argument validation,
+// workspace carving and kernel sequencing.  No device memory is allocated
+// here; every buffer belongs to the caller.
+#include <limits.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "saf_common.cuh"
+
+using namespace saf;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// Shape checks shared by every entry point.  Sizes must be non-negative and
+// every tensor's element count must fit the kernels' 64-bit indexing with
+// the per-slice offsets they compute in 32-bit (T * d_h < 2^31).
+saf_status check_shape(int B, int H, int T, int d_h) {
+    if (B < 0 || H < 0 || T < 0) return SAF_ERR_INVALID_ARG;
+    if (d_h != kHeadDim) return SAF_ERR_UNSUPPORTED;
+    if (H > kMaxHeads) return SAF_ERR_UNSUPPORTED;
+    if ((int64_t)T * kHeadDim > (int64_t)INT_MAX) return SAF_ERR_INVALID_ARG;
+    if ((int64_t)B * H > 65535LL * 1024) return SAF_ERR_INVALID_ARG;
+    const int64_t bht = (int64_t)B * H * T;
+    if (bht > (INT64_MAX / 4) / kHeadDim) return SAF_ERR_INVALID_ARG;
+    return SAF_OK;
+}
+
+saf_status build_headlist(const uint8_t* mask, int H, HeadList* hl) {
+    if (H > 0 && mask == nullptr) return SAF_ERR_INVALID_ARG;
+    memset(hl, 0, sizeof(*hl));
+    for (int h = 0; h < H; ++h) {
+        if (mask[h]) {
+            hl->replaced[h] = 1;
+            hl->heads[hl->n++] = (int16_t)h;
+        }
+    }
+    return SAF_OK;
+}
+
+inline saf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAF_OK : SAF_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* saf_status_string(int status) {
+    switch (status) {
+        case SAF_OK: return "SAF_OK";
+        case SAF_ERR_INVALID_ARG: return "SAF_ERR_INVALID_ARG";
+        case SAF_ERR_UNSUPPORTED: return "SAF_ERR_UNSUPPORTED";
+        case SAF_ERR_WORKSPACE: return "SAF_ERR_WORKSPACE";
+        case SAF_ERR_CUDA: return "SAF_ERR_CUDA";
+        case SAF_ERR_TIMEOUT: return "SAF_ERR_TIMEOUT";
+        default: return "SAF_ERR_UNKNOWN";
+    }
+}
+
+int saf_version(void) { return kVersion; }
+
+size_t saf_workspace_size(int B, int H, int T, int d_h, int is_bwd) {
+    if (check_shape(B, H, T, d_h) != SAF_OK) return (size_t)-1;
+    if ((int64_t)B * H * T == 0) return 0;
+    return ws_layout(B, H, T, is_bwd ? 1 : 0).total;
+}
+
+saf_status saf_replaced_lognorm(const float* a, const float* r, const uint8_t* replaced_mask,
+                                int H, int T, float* logz, void* stream) {
+    saf_status st = check_shape(1, H, T, kHeadDim);
+    if (st != SAF_OK) return st;
+    if ((int64_t)H * T == 0) return SAF_OK;
+    HeadList hl;
+    st = build_headlist(replaced_mask, H, &hl);
+    if (st != SAF_OK) return st;
+    if (hl.n == 0) return SAF_OK;
+    if (!a || !r || !logz) return SAF_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(r) || !aligned16(logz)) return SAF_ERR_INVALID_ARG;
+    return cuda_status(launch_lognorm(a, r, hl, T, logz, (cudaStream_t)stream));
+}
+
+saf_status saf_mixed_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const float* a, const float* r, const float* logz,
+                              const uint8_t* replaced_mask, int B, int H, int T, int d_h,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    saf_status st = check_shape(B, H, T, d_h);
+    if (st != SAF_OK) return st;
+    if ((int64_t)B * H * T == 0) return SAF_OK;
+    HeadList hl;
+    st = build_headlist(replaced_mask, H, &hl);
+    if (st != SAF_OK) return st;
+    if (!q || !k || !v || !o || !lse) return SAF_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return SAF_ERR_INVALID_ARG;
+    if (hl.n > 0) {
+        if (!a || !r) return SAF_ERR_INVALID_ARG;
+        if (!aligned16(a) || !aligned16(r) || (logz && !aligned16(logz))) return SAF_ERR_INVALID_ARG;
+    }
+    const WsLayout L = ws_layout(B, H, T, 0);
+    if (!workspace || workspace_bytes < L.total) return SAF_ERR_WORKSPACE;
+    if (!aligned256(workspace)) return SAF_ERR_INVALID_ARG;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    const float* lz = logz;
+    if (hl.n > 0 && lz == nullptr) {
+        float* lzw = reinterpret_cast<float*>(ws + L.logz);
+        cudaError_t e = launch_lognorm(a, r, hl, T, lzw, s);
+        if (e != cudaSuccess) return SAF_ERR_CUDA;
+        lz = lzw;
+    }
+    return cuda_status(launch_fwd_mma(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                      static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse,
+                                      a, r, lz, hl, B, H, T, s));
+}
+
+saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, const float* a, const float* r,
+                              const float* logz, const uint8_t* replaced_mask, int B, int H, int T,
+                              int d_h, void* dq, void* dk, void* dv, int grad_dtype,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    saf_status st = check_shape(B, H, T, d_h);
+    if (st != SAF_OK) return st;
+    if (grad_dtype != 0 && grad_dtype != 1) return SAF_ERR_UNSUPPORTED;
+    if ((int64_t)B * H * T == 0) return SAF_OK;
+    HeadList hl;
+    st = build_headlist(replaced_mask, H, &hl);
+    if (st != SAF_OK) return st;
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return SAF_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return SAF_ERR_INVALID_ARG;
+    if (hl.n > 0) {
+        if (!a || !r) return SAF_ERR_INVALID_ARG;
+        if (!aligned16(a) || !aligned16(r) || (logz && !aligned16(logz))) return SAF_ERR_INVALID_ARG;
+    }
+    const WsLayout L = ws_layout(B, H, T, 1);
+    if (!workspace || workspace_bytes < L.total) return SAF_ERR_WORKSPACE;
+    if (!aligned256(workspace)) return SAF_ERR_INVALID_ARG;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    const float* lz = logz;
+    if (hl.n > 0 && lz == nullptr) {
+        float* lzw = reinterpret_cast<float*>(ws + L.logz);
+        if (launch_lognorm(a, r, hl, T, lzw, s) != cudaSuccess) return SAF_ERR_CUDA;
+        lz = lzw;
+    }
+    float* dvec = reinterpret_cast<float*>(ws + L.dvec);
+    if (launch_bwd_dot(static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dvec,
+                       hl, B, H, T, s) != cudaSuccess)
+        return SAF_ERR_CUDA;
+    return cuda_status(launch_bwd_mma(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                      static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(dout),
+                                      lse, dvec, a, r, lz, hl, B, H, T, dq, dk, dv, grad_dtype, s));
+}
+
+saf_status saf_device_status(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < sizeof(WsHeader)) return SAF_ERR_WORKSPACE;
+    WsHeader hdr;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, s) != cudaSuccess) return SAF_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SAF_ERR_CUDA;
+    if (hdr.error != 0) {
+        if (cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned int), s) != cudaSuccess) return SAF_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return SAF_ERR_CUDA;
+        return SAF_ERR_TIMEOUT;
+    }
+    return SAF_OK;
+}
+
+}  // extern "C"

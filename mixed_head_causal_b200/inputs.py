@@ -106,13 +106,26 @@ def make_slice(w: Workload, seed: int, tensor: str, b: int, h: int) -> torch.Ten
     return x.to(torch.bfloat16)
 
 
-def make_tensor(w: Workload, seed: int, tensor: str, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Full [B, H, T, d] bf16 tensor, built slice by slice (CPU)."""
+def make_tensor(w: Workload, seed: int, tensor: str, out: Optional[torch.Tensor] = None,
+                threads: int = 0) -> torch.Tensor:
+    """Full [B, H, T, d] bf16 tensor, built slice by slice (CPU).  `threads`
+    > 1 fills slices concurrently (same values: every slice has its own
+    generator)."""
     if out is None:
         out = torch.empty(w.B, w.H, w.T, w.d, dtype=torch.bfloat16)
-    for b in range(w.B):
-        for h in range(w.H):
-            out[b, h].copy_(make_slice(w, seed, tensor, b, h))
+    jobs = [(b, h) for b in range(w.B) for h in range(w.H)]
+
+    def fill(bh):
+        b, h = bh
+        out[b, h].copy_(make_slice(w, seed, tensor, b, h))
+
+    if threads and threads > 1 and len(jobs) > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(fill, jobs))
+    else:
+        for bh in jobs:
+            fill(bh)
     return out
 
 
@@ -132,14 +145,14 @@ def make_pattern(w: Workload, seed: int = 0) -> Tuple[torch.Tensor, torch.Tensor
 
 
 def make_inputs(w: Workload, seed: int = 0, tensors: Iterable[str] = ("q", "k", "v", "do"),
-                pin: bool = False) -> Dict[str, torch.Tensor]:
+                pin: bool = False, threads: int = 0) -> Dict[str, torch.Tensor]:
     """All inputs of one workload as CPU tensors (optionally pinned)."""
     out: Dict[str, torch.Tensor] = {}
     for t in tensors:
         if t == "do" and not w.backward:
             continue
         buf = torch.empty(w.B, w.H, w.T, w.d, dtype=torch.bfloat16, pin_memory=pin)
-        out[t] = make_tensor(w, seed, t, out=buf)
+        out[t] = make_tensor(w, seed, t, out=buf, threads=threads)
     out["alpha"], out["rho"] = make_pattern(w, seed)
     out["mask"] = replaced_mask(w, seed)
     return out

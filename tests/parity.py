@@ -1,0 +1,102 @@
+"""Shared helpers of the GPU-vs-oracle parity tests.
+
+The bar (stated once, used by every parity test):
+  * mean |gpu - oracle| <= 2e-2 / 10 = 2e-3 over every element of a tensor;
+  * element-wise |gpu - oracle| <= 2e-2 for fp32-stored results, and
+    <= 2e-2 + 2^-8 |oracle| for bf16-stored results (2^-8 |x| bounds the
+    rounding of x to bfloat16's 8-bit significand, a floor no kernel can go
+    under once the result is stored in bf16);
+  * bit-exact zeros where the method fixes them (dQ, dK of replaced heads);
+  * lse within 2e-3 (natural-log units).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from mixed_head_causal_b200 import inputs as I
+from mixed_head_causal_b200 import saf
+
+TOL_MAX = 2e-2
+TOL_MEAN = 2e-3
+TOL_LSE = 2e-3
+BF16_REL = 2.0 ** -8
+
+
+def to_gpu(x):
+    return {k: (v.cuda() if torch.is_tensor(v) and k != "mask" else v) for k, v in x.items()}
+
+
+def run_layer(w, x, grad_dtype=torch.float32, backward=True):
+    """Runs the C-ABI forward (and backward) on device copies of x; returns CPU tensors."""
+    g = to_gpu(x)
+    o, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"])
+    out = {"o": o, "lse": lse}
+    if backward:
+        dq, dk, dv = saf.mixed_attn_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, g["alpha"], g["rho"],
+                                        x["mask"], grad_dtype=grad_dtype)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    return {k: v.cpu() for k, v in out.items()}
+
+
+def compare(name, got: torch.Tensor, ref: np.ndarray, stored_bf16: bool):
+    g = got.double().numpy()
+    err = np.abs(g - ref)
+    bound = TOL_MAX + (BF16_REL * np.abs(ref) if stored_bf16 else 0.0)
+    stats = {"max": float(err.max()) if err.size else 0.0, "mean": float(err.mean()) if err.size else 0.0,
+             "worst_over_bound": float((err / bound).max()) if err.size else 0.0}
+    assert np.isfinite(g).all(), f"{name}: non-finite values"
+    assert stats["mean"] <= TOL_MEAN, f"{name}: mean |err| {stats['mean']:.3e} > {TOL_MEAN}"
+    assert np.all(err <= bound), f"{name}: max |err| {stats['max']:.3e} over the bound ({stats})"
+    return stats
+
+
+def check_slices(w, x, got, slices, seed=0, grad_dtype=torch.float32):
+    """Compares the listed (b, h) slices of the GPU result with the oracle."""
+    mask = x["mask"].numpy()
+    a = x["alpha"].double().numpy()
+    r = x["rho"].double().numpy()
+    n = len(slices)
+
+    def stack(name):
+        if name in x:
+            return torch.stack([x[name][b, h] for b, h in slices])
+        return torch.stack([I.make_slice(w, seed, name, b, h) for b, h in slices])
+
+    q, k, v = stack("q"), stack("k"), stack("v")
+    rep = [int(mask[h]) for _, h in slices]
+    arows = np.stack([a[h] for _, h in slices])
+    rrows = np.stack([r[h] for _, h in slices])
+    o_ref, lse_ref = oracle.fwd_slices(q, k, v, arows, rrows, rep)
+    stats = {}
+    sel = lambda t: torch.stack([t[b, h] for b, h in slices])  # noqa: E731
+    stats["o"] = compare("O", sel(got["o"]), o_ref, stored_bf16=True)
+    lse_err = np.abs(sel(got["lse"]).double().numpy() - lse_ref)
+    assert lse_err.max() <= TOL_LSE, f"lse max err {lse_err.max():.3e}"
+    stats["lse"] = {"max": float(lse_err.max())}
+    if "dq" in got:
+        do = stack("do")
+        dq_ref, dk_ref, dv_ref = oracle.bwd_slices(q, k, v, do, arows, rrows, rep)
+        bf = grad_dtype == torch.bfloat16
+        stats["dq"] = compare("dQ", sel(got["dq"]), dq_ref, bf)
+        stats["dk"] = compare("dK", sel(got["dk"]), dk_ref, bf)
+        stats["dv"] = compare("dV", sel(got["dv"]), dv_ref, bf)
+        for i, (b, h) in enumerate(slices):
+            if rep[i]:
+                assert torch.count_nonzero(got["dq"][b, h]) == 0, "dQ of a replaced head must be 0"
+                assert torch.count_nonzero(got["dk"][b, h]) == 0, "dK of a replaced head must be 0"
+    return stats
+
+
+def sample_slices(w, mask, per_kind=2, seed=1234):
+    """A few (b, h) slices of each head kind, spread over the batch."""
+    rng = np.random.default_rng(seed)
+    rep = [h for h in range(w.H) if mask[h]]
+    ordn = [h for h in range(w.H) if not mask[h]]
+    out = []
+    for pool in (ordn, rep):
+        for _ in range(min(per_kind, len(pool) * w.B)):
+            out.append((int(rng.integers(w.B)), int(pool[rng.integers(len(pool))])))
+    return sorted(set(out))

@@ -1,0 +1,154 @@
+"""GPU path (through the C ABI) against the fp64 oracle, element by element.
+
+Tolerances are stated in tests/parity.py.  Small shapes are compared in
+full (several tiles plus ragged tails, both head kinds, degenerate patterns);
+the full-size workloads are compared on sampled (batch, head) slices that the
+oracle recomputes one by one, plus properties checked on every slice.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixed_head_causal_b200 import inputs as I
+from mixed_head_causal_b200 import saf
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+THREADS = min(16, os.cpu_count() or 1)
+
+
+def _all_slices(w):
+    return [(b, h) for b in range(w.B) for h in range(w.H)]
+
+
+@pytest.mark.parametrize("grad_dtype", [torch.float32, torch.bfloat16], ids=["grad_fp32", "grad_bf16"])
+def test_tiny_layer_full(grad_dtype):
+    w = I.WORKLOADS["tiny_b1_h4_t256"]
+    x = I.make_inputs(w, 0)
+    got = P.run_layer(w, x, grad_dtype)
+    stats = P.check_slices(w, x, got, _all_slices(w), grad_dtype=grad_dtype)
+    print(w.name, stats)
+
+
+@pytest.mark.parametrize("T", [1, 2, 7, 63, 64, 65, 127, 128, 129, 200, 255, 257, 383])
+@pytest.mark.parametrize("kind", ["mixed", "ordinary", "replaced"])
+def test_ragged_lengths(T, kind):
+    heads = {"mixed": [0, 2], "ordinary": [], "replaced": [0, 1, 2]}[kind]
+    w = I.custom(2, 3, T, heads)
+    x = I.make_inputs(w, 3)
+    got = P.run_layer(w, x, torch.float32)
+    P.check_slices(w, x, got, _all_slices(w))
+
+
+def test_several_tiles_full():
+    w = I.custom(2, 4, 1000, [1, 2])
+    x = I.make_inputs(w, 5)
+    got = P.run_layer(w, x, torch.bfloat16)
+    P.check_slices(w, x, got, _all_slices(w), grad_dtype=torch.bfloat16)
+
+
+def _special(T, a_fn, r_fn):
+    w = I.custom(1, 2, T, [1])
+    x = I.make_inputs(w, 7)
+    x["alpha"][1] = a_fn(T)
+    x["rho"][1] = r_fn(T)
+    return w, x
+
+
+def test_uniform_pattern_is_running_mean():
+    w, x = _special(300, lambda T: torch.zeros(T), lambda T: torch.zeros(T))
+    got = P.run_layer(w, x)
+    P.check_slices(w, x, got, _all_slices(w))
+    v = x["v"][0, 1].double()
+    mean = torch.cumsum(v, 0) / torch.arange(1, 301, dtype=torch.float64)[:, None]
+    assert (got["o"][0, 1].double() - mean).abs().max() < 1e-2
+
+
+def test_identity_pattern_gives_v():
+    def r_fn(T):
+        r = torch.full((T,), float("-inf"))
+        r[0] = 0.0
+        return r
+    w, x = _special(257, lambda T: torch.randn(T), r_fn)
+    got = P.run_layer(w, x)
+    assert torch.equal(got["o"][0, 1], x["v"][0, 1])
+    assert torch.equal(got["dv"][0, 1].to(torch.bfloat16), x["do"][0, 1])
+
+
+def test_sink_pattern_gives_first_value():
+    def a_fn(T):
+        a = torch.full((T,), float("-inf"))
+        a[0] = 0.0
+        return a
+    w, x = _special(190, a_fn, lambda T: torch.randn(T))
+    got = P.run_layer(w, x)
+    assert torch.equal(got["o"][0, 1], x["v"][0, 1][:1].expand(190, 64))
+    P.check_slices(w, x, got, _all_slices(w))
+
+
+def test_extreme_pattern_ranges():
+    """Long linear decay (terms far below fp32 range) and a +-60 shift."""
+    w, x = _special(2048, lambda T: torch.randn(T) * 3 + 60.0, lambda T: -0.5 * torch.arange(T, dtype=torch.float32) - 60.0)
+    got = P.run_layer(w, x)
+    P.check_slices(w, x, got, _all_slices(w))
+
+
+def test_lognorm_entry_point_and_explicit_logz():
+    w = I.custom(2, 4, 777, [0, 3])
+    x = I.make_inputs(w, 11)
+    g = P.to_gpu(x)
+    lz = saf.replaced_lognorm(g["alpha"], g["rho"], x["mask"])
+    ref = oracle.lognorm(x["alpha"][[0, 3]], x["rho"][[0, 3]])
+    err = np.abs(lz[[0, 3]].cpu().double().numpy() - ref)
+    assert err.max() < 1e-4 * max(1.0, np.abs(ref).max())
+    o1, l1 = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"])
+    o2, l2 = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"], logz=lz)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    d1 = saf.mixed_attn_bwd(g["q"], g["k"], g["v"], o1, g["do"], l1, g["alpha"], g["rho"], x["mask"])
+    d2 = saf.mixed_attn_bwd(g["q"], g["k"], g["v"], o1, g["do"], l1, g["alpha"], g["rho"], x["mask"], logz=lz)
+    for a, b in zip(d1, d2):
+        assert torch.equal(a, b)
+
+
+def test_repeatable():
+    w = I.custom(1, 3, 700, [1])
+    x = I.make_inputs(w, 2)
+    a = P.run_layer(w, x)
+    b = P.run_layer(w, x)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def _full_size(name, grad_dtype=torch.float32, per_kind=2):
+    w = I.WORKLOADS[name]
+    x = I.make_inputs(w, 0, threads=THREADS)
+    got = P.run_layer(w, x, grad_dtype, backward=w.backward)
+    mask = x["mask"]
+    # properties on every slice
+    for key in got:
+        assert torch.isfinite(got[key].float()).all(), key
+    if w.backward:
+        rep = mask.bool()
+        assert torch.count_nonzero(got["dq"][:, rep]) == 0
+        assert torch.count_nonzero(got["dk"][:, rep]) == 0
+    slices = P.sample_slices(w, mask.numpy(), per_kind=per_kind)
+    stats = P.check_slices(w, x, got, slices, grad_dtype=grad_dtype)
+    print(name, slices, stats)
+
+
+@pytest.mark.parametrize("name", ["124m_b8_t4096_r25", "124m_b4_t8192_r50", "1b_b4_h32_t8192_r25"])
+def test_full_size_fwd_bwd_sampled(name):
+    _full_size(name, torch.float32)
+
+
+def test_full_size_bf16_grads_sampled():
+    _full_size("124m_b8_t4096_r25", torch.bfloat16)
+
+
+@pytest.mark.parametrize("name", I.PREFILL_SWEEP)
+def test_prefill_sweep_sampled(name):
+    _full_size(name, per_kind=1)
