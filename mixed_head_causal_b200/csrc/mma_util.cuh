@@ -62,6 +62,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi): a two-term bf16 split
+// whose sum carries about 16 significant bits instead of 8.
+__device__ __forceinline__ void pack_bf16_split(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    float2 hf = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<uint32_t*>(&h);
+    lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
 // A fragment (16 rows x 16 k) of a swizzled tile: rows r0.., k columns k0...
 __device__ __forceinline__ void load_a_frag(uint32_t* a, uint32_t sbase, int r0, int k0, int lane) {
     const int row = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;

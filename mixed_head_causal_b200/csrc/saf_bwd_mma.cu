@@ -197,20 +197,34 @@ __global__ void __launch_bounds__(NT) dkdv_kernel(const BwdParams p) {
                     }
                 }
             }
-            // dV += P^T dO   (k = queries, n = head dim)
-            uint32_t pf[4][4];
+            // dV += P^T dO   (k = queries, n = head dim).  Replaced heads use
+            // a hi + lo bf16 split of P^T: a column of a fixed pattern (a
+            // sink, say) can hold large weights over many rows, and bf16
+            // rounding of each would add up in dV.
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                pf[kk][0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-                pf[kk][1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-                pf[kk][2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-                pf[kk][3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                uint32_t pf[4], pl[4];
+                if (!rep) {
+                    pf[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+                    pf[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+                    pf[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+                    pf[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                } else {
+                    pack_bf16_split(s[2 * kk][0], s[2 * kk][1], pf[0], pl[0]);
+                    pack_bf16_split(s[2 * kk][2], s[2 * kk][3], pf[1], pl[1]);
+                    pack_bf16_split(s[2 * kk + 1][0], s[2 * kk + 1][1], pf[2], pl[2]);
+                    pack_bf16_split(s[2 * kk + 1][2], s[2 * kk + 1][3], pf[3], pl[3]);
+                }
 #pragma unroll
                 for (int np = 0; np < 4; ++np) {
                     uint32_t b[4];
                     load_b_frag_kn(b, sOb, np * 16, kk * 16, lane);
-                    mma_bf16(dvacc[2 * np], pf[kk], b[0], b[1]);
-                    mma_bf16(dvacc[2 * np + 1], pf[kk], b[2], b[3]);
+                    mma_bf16(dvacc[2 * np], pf, b[0], b[1]);
+                    mma_bf16(dvacc[2 * np + 1], pf, b[2], b[3]);
+                    if (rep) {
+                        mma_bf16(dvacc[2 * np], pl, b[0], b[1]);
+                        mma_bf16(dvacc[2 * np + 1], pl, b[2], b[3]);
+                    }
                 }
             }
             if (!rep) {

@@ -178,20 +178,33 @@ __global__ void __launch_bounds__(NT) fwd_mma_kernel(const FwdParams p) {
                     }
                 }
             }
-            // O += P V
+            // O += P V.  A replaced head's P enters as a hi + lo bf16 pair:
+            // its weights are not renormalised by an online softmax, so their
+            // rounding would otherwise reach the output at full size.
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                uint32_t af[4];
-                af[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-                af[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-                af[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-                af[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                uint32_t af[4], al[4];
+                if (!rep) {
+                    af[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+                    af[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+                    af[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+                    af[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+                } else {
+                    pack_bf16_split(s[2 * kk][0], s[2 * kk][1], af[0], al[0]);
+                    pack_bf16_split(s[2 * kk][2], s[2 * kk][3], af[1], al[1]);
+                    pack_bf16_split(s[2 * kk + 1][0], s[2 * kk + 1][1], af[2], al[2]);
+                    pack_bf16_split(s[2 * kk + 1][2], s[2 * kk + 1][3], af[3], al[3]);
+                }
 #pragma unroll
                 for (int np = 0; np < 4; ++np) {
                     uint32_t b[4];
                     load_b_frag_kn(b, sVb, np * 16, kk * 16, lane);
                     mma_bf16(oacc[2 * np], af, b[0], b[1]);
                     mma_bf16(oacc[2 * np + 1], af, b[2], b[3]);
+                    if (rep) {
+                        mma_bf16(oacc[2 * np], al, b[0], b[1]);
+                        mma_bf16(oacc[2 * np + 1], al, b[2], b[3]);
+                    }
                 }
             }
         }
