@@ -133,6 +133,33 @@ SAF_API saf_status saf_mixed_attn_bwd(const void *q, const void *k, const void *
                               void *stream);
 
 /*
+ * Allocation-free backward, for callers that cannot pass a workspace: code
+ * that may not call cudaMalloc (custom allocators' own callbacks, frameworks
+ * that own all device memory), or that has no allocator to draw one from.
+ * (The paper has no counterpart: this is an integration aid.)
+ *
+ * Same arguments and results as saf_mixed_attn_bwd minus the workspace.  Its
+ * scratch (the per-row terms rowsum(dO o O), and the replaced heads' log Z
+ * when logz is NULL) lives in one 8 MiB array of device memory inside the
+ * library, one per GPU, held from load until process exit.  Limit:
+ *     round_up(B*H*T, 64) + (logz == NULL && any head replaced ? H*T : 0)
+ *         <= 2,097,152 fp32 values,
+ * otherwise SAF_ERR_WORKSPACE is returned and nothing is enqueued.
+ * The first call on a device looks up that array's device address (once per
+ * device, with the device current); make that first call before any stream
+ * capture.  Every call shares the array: calls that overlap on the GPU race
+ * and give wrong results.  Nothing in it needs clearing between calls.  It
+ * allocates no device memory.
+ */
+SAF_API saf_status saf_mixed_attn_bwd_noalloc(const void *q, const void *k, const void *v,
+                                              const void *o, const void *dout, const float *lse,
+                                              const float *a, const float *r, const float *logz,
+                                              const uint8_t *replaced_mask,
+                                              int B, int H, int T, int d_h,
+                                              void *dq, void *dk, void *dv, int grad_dtype,
+                                              void *stream);
+
+/*
  * Reads (synchronously: waits for `stream`) and clears the device error word
  * that the kernels keep in the first 256 bytes of `workspace`.  Those bytes
  * must be zero before the workspace is first used (e.g. one cudaMemset); the

@@ -30,6 +30,8 @@ SIGNATURES = {
     "saf_mixed_attn_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                             _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "saf_device_status": ([_vp, _sz, _vp], _i),
+    "saf_mixed_attn_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                    _vp, _vp, _vp, _i, _vp], _i),
     "saf_launch_count": ([], ctypes.c_uint64),
     "saf_profile_enable": ([_i], _i),
     "saf_profile_read": ([ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_float), _i], _i),
@@ -167,6 +169,28 @@ def mixed_attn_bwd(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtyp
                                      _ptr(dq), _ptr(dk), _ptr(dv), gd, _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
            "saf_mixed_attn_bwd")
+    return dq, dk, dv
+
+
+def mixed_attn_bwd_noalloc(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtype=torch.bfloat16,
+                           dq=None, dk=None, dv=None, stream=None):
+    """Backward without a workspace (the library's own fixed scratch, see
+    include/saf.h): for callers that cannot allocate device memory.  Output
+    tensors are still the caller's; pass them in to allocate nothing here."""
+    B, H, T, d = v.shape
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_layer_tensor(n, t, (B, H, T, d))
+    gd = 1 if grad_dtype == torch.float32 else 0
+    dq = torch.empty(B, H, T, d, dtype=grad_dtype, device=v.device) if dq is None else dq
+    dk = torch.empty(B, H, T, d, dtype=grad_dtype, device=v.device) if dk is None else dk
+    dv = torch.empty(B, H, T, d, dtype=grad_dtype, device=v.device) if dv is None else dv
+    mbuf, mh = _mask_buffer(mask)
+    if mh != H:
+        raise ValueError("mask length != H")
+    _check(load().saf_mixed_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                             _ptr(alpha), _ptr(rho), _ptr(logz), ctypes.addressof(mbuf),
+                                             B, H, T, d, _ptr(dq), _ptr(dk), _ptr(dv), gd, _stream_ptr(stream)),
+           "saf_mixed_attn_bwd_noalloc")
     return dq, dk, dv
 
 
