@@ -2,6 +2,7 @@
 // workspace carving and kernel sequencing.  No device memory is allocated
 // here; every buffer belongs to the caller.
 #include <limits.h>
+#include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -43,6 +44,13 @@ saf_status build_headlist(const uint8_t* mask, int H, HeadList* hl) {
 }
 
 inline saf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAF_OK : SAF_ERR_CUDA; }
+
+// SAF_FORCE_MMA=1 in the environment routes every head through the
+// warp-level mma.sync kernels (the per-element path), for comparisons.
+bool force_mma_path() {
+    const char* e = getenv("SAF_FORCE_MMA");
+    return e && e[0] == '1';
+}
 
 }  // namespace
 
@@ -112,9 +120,19 @@ saf_status saf_mixed_attn_fwd(const void* q, const void* k, const void* v, void*
         if (e != cudaSuccess) return SAF_ERR_CUDA;
         lz = lzw;
     }
-    return cuda_status(launch_fwd_mma(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                      static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse,
-                                      a, r, lz, hl, B, H, T, s));
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+    const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
+    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+    if (force_mma_path()) return cuda_status(launch_fwd_mma(qb, kb, vb, ob, lse, a, r, lz, hl, B, H, T, s));
+    const ReplacedWs rw = replaced_ws(ws, L, T);
+    if (hl.n > 0 && launch_prep_replaced(a, r, lz, hl, T, rw, s) != cudaSuccess) return SAF_ERR_CUDA;
+    cudaError_t e = launch_fwd_tc(qb, kb, vb, ob, lse, lz, hl, rw, B, H, T, reinterpret_cast<unsigned int*>(ws), s);
+    if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return SAF_ERR_CUDA;
+    // replaced heads whose factored form would leave fp32 range
+    if (hl.n > 0) return cuda_status(launch_fwd_mma(qb, kb, vb, ob, lse, a, r, lz, hl, B, H, T, s, rw.flag));
+    return SAF_OK;
 }
 
 saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const void* o,

@@ -28,6 +28,20 @@ struct Shape {
     int64_t row_stride_bh;  // T * d elements between consecutive (b,h) slices
 };
 
+// Device arrays of the factored replaced-head pattern (see prep_replaced in
+// saf_prep.cu), one row per replaced-head slot s (slot order = head order).
+struct ReplacedWs {
+    int Tp, Lp;          // T rounded up to 128; Tp + 256
+    uint32_t* epair;     // [slots][Lp]   bf16 pairs {E[x], E[x-1]} at x + 128
+    float* ef;           // [slots][Lp]   fp32 E[x] at x + 128
+    uint32_t* cpair;     // [slots][Tp/2] bf16 pairs {c[2m], c[2m+1]}
+    float* cf;           // [slots][Tp]   fp32 c[j]
+    float* rsc;          // [slots][Tp]   fp32 r_i
+    int* flag;           // [H] 1 = head needs the per-element exp path
+};
+
+__host__ __device__ inline int round_up128(int x) { return (x + 127) & ~127; }
+
 // ---------------------------------------------------------------- workspace
 // Offsets of the scratch regions inside the caller's workspace.  Every region
 // starts on a 256-byte boundary.
@@ -35,6 +49,7 @@ struct WsLayout {
     size_t header;   // device error word + counters (256 B)
     size_t logz;     // [H, T] fp32 (used when the caller passes logz = NULL)
     size_t dvec;     // [B, H, T] fp32 row terms rowsum(dO o O) (backward only)
+    size_t epair, ef, cpair, cf, rsc, flag;  // factored replaced-head arrays (H slots)
     size_t total;
 };
 
@@ -46,8 +61,28 @@ inline WsLayout ws_layout(int B, int H, int T, int is_bwd) {
     L.header = off; off += 256;
     L.logz = off; off = align256(off + sizeof(float) * (size_t)H * T);
     if (is_bwd) { L.dvec = off; off = align256(off + sizeof(float) * (size_t)B * H * T); }
+    const size_t Tp = (size_t)round_up128(T), Lp = Tp + 256;
+    L.epair = off; off = align256(off + 4 * (size_t)H * Lp);
+    L.ef = off; off = align256(off + 4 * (size_t)H * Lp);
+    L.cpair = off; off = align256(off + 4 * (size_t)H * (Tp / 2));
+    L.cf = off; off = align256(off + 4 * (size_t)H * Tp);
+    L.rsc = off; off = align256(off + 4 * (size_t)H * Tp);
+    L.flag = off; off = align256(off + 4 * (size_t)H);
     L.total = off;
     return L;
+}
+
+inline ReplacedWs replaced_ws(char* ws, const WsLayout& L, int T) {
+    ReplacedWs w;
+    w.Tp = round_up128(T);
+    w.Lp = w.Tp + 256;
+    w.epair = reinterpret_cast<uint32_t*>(ws + L.epair);
+    w.ef = reinterpret_cast<float*>(ws + L.ef);
+    w.cpair = reinterpret_cast<uint32_t*>(ws + L.cpair);
+    w.cf = reinterpret_cast<float*>(ws + L.cf);
+    w.rsc = reinterpret_cast<float*>(ws + L.rsc);
+    w.flag = reinterpret_cast<int*>(ws + L.flag);
+    return w;
 }
 
 // Device error word layout (first bytes of the workspace header).
@@ -71,10 +106,20 @@ void launch_end(int kid, cudaStream_t s);
 // (defined in the kernel translation units; all enqueue on `stream`)
 cudaError_t launch_lognorm(const float* a, const float* r, const HeadList& hl, int T,
                            float* logz, cudaStream_t stream);
+cudaError_t launch_prep_replaced(const float* a, const float* r, const float* logz, const HeadList& hl, int T,
+                                 const ReplacedWs& w, cudaStream_t stream);
+// Tensor-core forward of every ordinary head and every replaced head whose
+// factored form is usable (flag 0); returns cudaErrorNotSupported when the
+// tensor maps cannot be built.
+cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                          __nv_bfloat16* o, float* lse, const float* logz, const HeadList& hl,
+                          const ReplacedWs& w, int B, int H, int T, unsigned int* err, cudaStream_t stream);
+// head_only_flag != nullptr: run only replaced heads h with head_only_flag[h] != 0.
 cudaError_t launch_fwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, __nv_bfloat16* o, float* lse,
                            const float* a, const float* r, const float* logz,
-                           const HeadList& hl, int B, int H, int T, cudaStream_t stream);
+                           const HeadList& hl, int B, int H, int T, cudaStream_t stream,
+                           const int* head_only_flag = nullptr);
 cudaError_t launch_bwd_dot(const __nv_bfloat16* o, const __nv_bfloat16* dout, float* dvec,
                            const HeadList& hl, int B, int H, int T, cudaStream_t stream);
 cudaError_t launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,

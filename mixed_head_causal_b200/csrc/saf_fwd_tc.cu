@@ -1,0 +1,390 @@
+// Mixed-head causal attention forward on the 5th-generation tensor cores
+// (tcgen05, accumulators in TMEM, operands staged by TMA).
+//
+// One CTA computes one 128-row query block of one (batch, head) slice; both
+// head kinds share the grid, which is ordered longest rows first.  Warp roles:
+//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys through
+//               a 2-stage shared-memory ring (K is skipped for replaced heads)
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2..5  one query row per thread: softmax / pattern builder, epilogue
+//
+// Ordinary head, per key block j (FlashAttention-style online softmax, the
+// "FlashAttention-2 online softmax tile" of the reading notes, section 二.4):
+//   S = Q K_j^T             tcgen05 SS MMA, 128x128, fp32 in TMEM
+//   P = exp2(S*log2e/sqrt(d) - m), row max m kept lazily (the O rescale is
+//       skipped unless m grows by more than 8 in log2 units), P as bf16 into TMEM
+//   O += P V_j              tcgen05 TS MMA (A = P from TMEM), fp32 in TMEM
+// Replaced head (Eq. (3), section 二.3, in factored form): the tile
+//   W(i,j) = E[i-j] c_j     (bf16 pairs multiplied in registers, no exp)
+// is written to TMEM and O += W V_j; the epilogue scales row i by r_i, giving
+//   O_i = sum_j exp(a[j] + r[i-j] - log Z(i)) V_j.
+// Causal tile skipping: key blocks past the diagonal are never visited; the
+// diagonal block is masked (ordinary) or zero by construction (E[d<0] = 0).
+#include "saf_common.cuh"
+#include "tc_util.cuh"
+
+namespace saf {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;          // query rows per CTA
+constexpr int BN = 128;          // keys per block
+constexpr int NST = 2;           // K/V ring stages
+constexpr int NTHREADS = 192;
+constexpr uint32_t TILE_BYTES = 128 * 64 * 2;  // one 128 x 64 bf16 tile
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TS_COL = 0, TO_COL = 128, TP_COL = 192;  // S, O, P regions
+constexpr long long kWaitLimit = 1ll << 31;                 // cycles
+
+// shared memory map (offsets from a 1024-aligned base)
+constexpr uint32_t SM_Q = 0;
+constexpr uint32_t SM_K = SM_Q + TILE_BYTES;
+constexpr uint32_t SM_V = SM_K + NST * TILE_BYTES;
+constexpr uint32_t SM_BAR = SM_V + NST * TILE_BYTES;
+constexpr uint32_t SM_TOTAL = SM_BAR + 256;
+
+struct FwdTcParams {
+    __nv_bfloat16* o;
+    float* lse;
+    const float* logz;
+    ReplacedWs w;
+    unsigned int* err;
+    int16_t slot_of_head[kMaxHeads];
+    int H, T, nqb;
+    float scale_log2;
+};
+
+__device__ __forceinline__ void report(unsigned int* err, unsigned int code) {
+    atomicOr(err, 1u);
+    atomicCAS(err + 1, 0u, code);
+}
+
+__global__ void __launch_bounds__(NTHREADS, 2)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const FwdTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t bar_q = sbase + SM_BAR;
+    const uint32_t bar_kf = bar_q + 8;            // [NST]
+    const uint32_t bar_vf = bar_kf + 8 * NST;     // [NST]
+    const uint32_t bar_ke = bar_vf + 8 * NST;     // [NST] stage free
+    const uint32_t bar_s = bar_ke + 8 * NST;      // S ready
+    const uint32_t bar_p = bar_s + 8;             // P written (128 arrivals)
+    const uint32_t bar_o = bar_p + 8;             // P.V done
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 128);
+
+    const int T = p.T;
+    const int bh = blockIdx.x;
+    const int I = p.nqb - 1 - (int)blockIdx.y;
+    const int h = bh % p.H;
+    const int slot = p.slot_of_head[h];
+    const bool rep = slot >= 0;
+    if (rep && p.w.flag[h] != 0) return;  // handled by the per-element exp path
+    const int nkb = I + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bar_kf + 8 * s, 1);
+            mbar_init(bar_vf + 8 * s, 1);
+            mbar_init(bar_ke + 8 * s, 1);
+        }
+        mbar_init(bar_s, 1);
+        mbar_init(bar_p, 128);
+        mbar_init(bar_o, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            if (!rep) {
+                prefetch_tmap(&tmQ);
+                prefetch_tmap(&tmK);
+            }
+            prefetch_tmap(&tmV);
+            if (!rep) {
+                mbar_expect_tx(bar_q, TILE_BYTES);
+                tma_load_3d(sbase + SM_Q, &tmQ, bar_q, 0, I * BM, bh);
+            }
+            for (int j = 0; j < nkb; ++j) {
+                const int s = j % NST, n = j / NST;
+                if (!mbar_wait(bar_ke + 8 * s, (n & 1) ^ 1, kWaitLimit)) { report(p.err, 0x101); break; }
+                if (!rep) {
+                    mbar_expect_tx(bar_kf + 8 * s, TILE_BYTES);
+                    tma_load_3d(sbase + SM_K + s * TILE_BYTES, &tmK, bar_kf + 8 * s, 0, j * BN, bh);
+                }
+                mbar_expect_tx(bar_vf + 8 * s, TILE_BYTES);
+                tma_load_3d(sbase + SM_V + s * TILE_BYTES, &tmV, bar_vf + 8 * s, 0, j * BN, bh);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
+            const uint32_t idO = idesc_bf16(128, 64, 0, 1);   // P (TMEM) x V (MN-major)
+            const uint64_t dq = sw128_desc(sbase + SM_Q);
+            bool ok = true;
+            if (!rep && !mbar_wait(bar_q, 0, kWaitLimit)) { report(p.err, 0x201); ok = false; }
+            for (int j = 0; ok && j < nkb; ++j) {
+                const int s = j % NST, n = j / NST;
+                if (!rep) {
+                    if (!mbar_wait(bar_kf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x202); break; }
+                    tc_fence_after();
+                    const uint64_t dk = sw128_desc(sbase + SM_K + s * TILE_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
+                        mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
+                    mma_commit(bar_s);
+                }
+                if (!mbar_wait(bar_vf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x203); break; }
+                if (!mbar_wait(bar_p, j & 1, kWaitLimit)) { report(p.err, 0x204); break; }
+                tc_fence_after();
+                const uint64_t dv = sw128_desc(sbase + SM_V + s * TILE_BYTES);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
+                    mma_ts(tmem + TO_COL, tmem + TP_COL + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
+                mma_commit(bar_o);
+                mma_commit(bar_ke + 8 * s);
+            }
+        }
+    } else {
+        // ------------------------------------------------ row threads
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;  // TMEM lane = query row within the block
+        const int i = I * BM + row;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lane_off + TS_COL;
+        const uint32_t tO = tmem + lane_off + TO_COL;
+        const uint32_t tP = tmem + lane_off + TP_COL;
+        float m = kNegInf, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkb; ++j) {
+            uint32_t pw[64];
+            if (!rep) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, kWaitLimit));
+                if (!ok) { report(p.err, 0x301); break; }
+                tc_fence_after();
+                const bool diag = (j == I);
+                const int kbase = j * BN;
+                // pass 1: row max of the scaled scores
+                float mx = kNegInf;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tS + 32 * c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = kbase + 32 * c + e;
+                        float x = __uint_as_float(v[e]) * p.scale_log2;
+                        if (diag && (key > i || key >= T)) x = kNegInf;
+                        mx = fmaxf(mx, x);
+                    }
+                }
+                // the S -> P hand-off also needs the previous P.V finished
+                if (j > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, kWaitLimit));
+                    if (!ok) { report(p.err, 0x302); break; }
+                }
+                tc_fence_after();
+                float f = 1.f;
+                if (m == kNegInf) {
+                    m = mx;
+                } else if (mx > m + 8.f) {
+                    f = ex2(m - mx);
+                    l *= f;
+                    m = mx;
+                }
+                // TMEM loads/stores are warp-collective: rescale the O rows of
+                // the whole warp when any of its rows needs it (others use 1)
+                if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(tO + 32 * c, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                        tmem_st32(tO + 32 * c, v);
+                    }
+                }
+                // pass 2: P = exp2(x - m) as bf16 pairs
+                const float mref = (m == kNegInf) ? 0.f : m;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tS + 32 * c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int key = kbase + 32 * c + e;
+                        float x0 = __uint_as_float(v[e]) * p.scale_log2;
+                        float x1 = __uint_as_float(v[e + 1]) * p.scale_log2;
+                        float p0 = ex2(x0 - mref), p1 = ex2(x1 - mref);
+                        if (diag && (key > i || key >= T)) p0 = 0.f;
+                        if (diag && (key + 1 > i || key + 1 >= T)) p1 = 0.f;
+                        if (m == kNegInf) { p0 = 0.f; p1 = 0.f; }
+                        l += p0 + p1;
+                        pw[16 * c + e / 2] = pack_bf16x2(p0, p1);
+                    }
+                }
+            } else {
+                if (j > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, kWaitLimit));
+                    if (!ok) { report(p.err, 0x303); break; }
+                }
+                // W(i,j) = E[i-j] c_j, bf16 pairs
+                const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
+                const uint4* cp = reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
+#pragma unroll
+                for (int q4 = 0; q4 < 16; ++q4) {
+                    const uint4 c4 = __ldg(cp + q4);
+                    const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int mm = 4 * q4 + u;  // key pair (2mm, 2mm+1)
+                        const uint32_t e2 = __ldg(ep - 2 * mm);
+                        __nv_bfloat162 prod = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e2),
+                                                      *reinterpret_cast<const __nv_bfloat162*>(&cw[u]));
+                        pw[mm] = *reinterpret_cast<uint32_t*>(&prod);
+                    }
+                }
+            }
+            // P (or W) -> TMEM, then hand it to the MMA warp
+            {
+                uint32_t lo[32], hi[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) { lo[e] = pw[e]; hi[e] = pw[32 + e]; }
+                tmem_st32(tP, lo);
+                tmem_st32(tP + 32, hi);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_p);
+        }
+        // epilogue (TMEM reads by whole warps; rows past T are not stored)
+        if (ok) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (nkb - 1) & 1, kWaitLimit));
+            if (!ok) report(p.err, 0x304);
+        }
+        tc_fence_after();
+        if (ok) {
+            float scale = 0.f, lse_v = kNegInf;
+            if (i < T) {
+                if (!rep) {
+                    scale = l > 0.f ? 1.f / l : 0.f;
+                    lse_v = (m == kNegInf || l <= 0.f) ? kNegInf : (m + log2f(l)) * kLn2;
+                } else {
+                    scale = p.w.rsc[(size_t)slot * p.w.Tp + i];
+                    lse_v = p.logz[(size_t)h * T + i];
+                }
+            }
+            __nv_bfloat16* orow = p.o + ((size_t)bh * T + (i < T ? i : 0)) * kHeadDim;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tO + 32 * c, v);
+                tmem_wait_ld();
+                uint32_t packed[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    packed[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * scale, __uint_as_float(v[2 * e + 1]) * scale);
+                if (i < T) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                }
+            }
+            if (i < T) p.lse[(size_t)bh * T + i] = lse_v;
+        } else if (i < T) {
+            p.lse[(size_t)bh * T + i] = __int_as_float(0x7fc00000);  // NaN marks the failed rows
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+}  // namespace
+
+// [BH, T, 64] bf16 viewed as a 3-D tensor (d, t, bh); 128 x 64 boxes with the
+// 128-byte swizzle; rows past T read as zeros.
+bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {64 * 2, (cuuint64_t)T * 64 * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                          __nv_bfloat16* o, float* lse, const float* logz, const HeadList& hl,
+                          const ReplacedWs& w, int B, int H, int T, unsigned int* err, cudaStream_t stream) {
+    CUtensorMap mq, mk, mv;
+    const int BH = B * H;
+    if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, BH, T, &mk) || !make_tmap_bhtd(v, BH, T, &mv))
+        return cudaErrorNotSupported;
+    FwdTcParams p;
+    p.o = o;
+    p.lse = lse;
+    p.logz = logz;
+    p.w = w;
+    p.err = err;
+    int slot = 0;
+    for (int hh = 0; hh < kMaxHeads; ++hh) p.slot_of_head[hh] = -1;
+    for (int hh = 0; hh < H; ++hh)
+        if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
+    p.H = H;
+    p.T = T;
+    p.nqb = (T + BM - 1) / BM;
+    p.scale_log2 = kLog2e / 8.0f;
+    const int smem = SM_TOTAL + 1024;
+    cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    launch_begin(KID_FWD_TC, stream);
+    fwd_tc_kernel<<<dim3(BH, p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, p);
+    launch_end(KID_FWD_TC, stream);
+    return cudaGetLastError();
+}
+
+}  // namespace saf
