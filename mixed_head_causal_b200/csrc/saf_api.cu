@@ -167,13 +167,33 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
         if (launch_lognorm(a, r, hl, T, lzw, s) != cudaSuccess) return SAF_ERR_CUDA;
         lz = lzw;
     }
-    float* dvec = reinterpret_cast<float*>(ws + L.dvec);
-    if (launch_bwd_dot(static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dvec,
-                       hl, B, H, T, s) != cudaSuccess)
-        return SAF_ERR_CUDA;
-    return cuda_status(launch_bwd_mma(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                      static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(dout),
-                                      lse, dvec, a, r, lz, hl, B, H, T, dq, dk, dv, grad_dtype, s));
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+    const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
+    const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
+    const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
+    if (force_mma_path()) {
+        float* dvec = reinterpret_cast<float*>(ws + L.dvec);
+        if (launch_bwd_dot(ob, dob, dvec, hl, B, H, T, s) != cudaSuccess) return SAF_ERR_CUDA;
+        return cuda_status(launch_bwd_mma(qb, kb, vb, dob, lse, dvec, a, r, lz, hl, B, H, T, dq, dk, dv,
+                                          grad_dtype, s));
+    }
+    const ReplacedWs rw = replaced_ws(ws, L, T);
+    if (hl.n > 0 && launch_prep_replaced(a, r, lz, hl, T, rw, s) != cudaSuccess) return SAF_ERR_CUDA;
+    float* lse2p = reinterpret_cast<float*>(ws + L.lse2p);
+    float* dvecp = reinterpret_cast<float*>(ws + L.dvecp);
+    float* dqacc = reinterpret_cast<float*>(ws + L.dqacc);
+    if (launch_bwd_pre(ob, dob, lse, B * H, T, lse2p, dvecp, dqacc, s) != cudaSuccess) return SAF_ERR_CUDA;
+    cudaError_t e = launch_bwd_tc(qb, kb, vb, dob, lse2p, dvecp, dqacc, hl, rw, B, H, T, dk, dv, grad_dtype,
+                                  reinterpret_cast<unsigned int*>(ws), s);
+    if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return SAF_ERR_CUDA;
+    if (launch_dq_convert(dqacc, dq, (int64_t)B * H * T, grad_dtype, s) != cudaSuccess) return SAF_ERR_CUDA;
+    // replaced heads whose factored form would leave fp32 range
+    if (hl.n > 0)
+        return cuda_status(launch_bwd_mma(qb, kb, vb, dob, lse, dvecp, a, r, lz, hl, B, H, T, dq, dk, dv,
+                                          grad_dtype, s, rw.flag));
+    return SAF_OK;
 }
 
 saf_status saf_device_status(void* workspace, size_t workspace_bytes, void* stream) {

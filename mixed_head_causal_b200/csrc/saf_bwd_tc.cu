@@ -1,0 +1,585 @@
+// Mixed-head causal attention backward on the 5th-generation tensor cores.
+//
+// One CTA owns one 128-key block J of one (batch, head) slice and walks the
+// query blocks I >= J (causal tile skipping; the diagonal block is masked).
+// dK and dV accumulate in TMEM for the whole walk; each tile's dQ
+// contribution is reduced into an fp32 accumulator in global memory with a
+// TMA reduce-add.  Warp roles:
+//   warp 0      TMA producer: K, V once; Q, dO and the per-query vectors of
+//               each query block through a 2-stage ring
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2..5  one key row per thread: P^T, dS^T, dK/dV epilogue
+//   warps 6..9  one query row per thread: dQ tile TMEM -> smem -> reduce-add
+//
+// Ordinary head, per tile (rows = keys j, columns = queries i; the textbook
+// softmax-attention gradients, section 二.4 of the reading notes):
+//   S^T  = K Q^T            SS MMA            P^T = exp2(S^T s log2e - lse2_i)
+//   dP^T = V dO^T           SS MMA            dS^T = P^T o (dP^T - D_i)
+//   dV  += P^T dO           TS MMA (P^T as bf16 in TMEM, aliasing S^T)
+//   dK  += dS^T Q           TS MMA (dS^T as bf16 in TMEM, aliasing dP^T)
+//   dQ_I = dS K             SS MMA (dS^T in smem read as an MN-major A)
+// Replaced head: only dV = P^T dO (section 二.4), with P in the factored
+// form of Eq. (3): P^T(j,i) = c_j * W(j,i), W(j,i) = E[i-j] r_i in fp32,
+// fed to the tensor cores as a hi + lo bf16 pair (two TS MMAs) so that a
+// column with large weights over many rows (a sink) keeps its precision;
+// c_j is applied in the epilogue.  dK = 0 there, and dQ gets no contribution.
+#include "saf_common.cuh"
+#include "tc_util.cuh"
+
+namespace saf {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;  // queries per block
+constexpr int BN = 128;  // keys per CTA
+constexpr int NTHREADS = 320;
+constexpr uint32_t TILE = 128 * 64 * 2;  // 16 KB bf16 tile
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ0 = 384, C_DQ1 = 448;
+constexpr long long kWaitLimit = 1ll << 31;
+
+constexpr uint32_t SM_K = 0;
+constexpr uint32_t SM_V = SM_K + TILE;
+constexpr uint32_t SM_Q = SM_V + TILE;        // 2 stages
+constexpr uint32_t SM_DO = SM_Q + 2 * TILE;   // 2 stages
+constexpr uint32_t SM_DS = SM_DO + 2 * TILE;  // 32 KB: dS^T as two 64-query atoms
+constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;  // 32 KB fp32 [128][64] staging
+constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;  // 2 x 512 B: lse2 (ordinary) / r (replaced)
+constexpr uint32_t SM_VEC2 = SM_VEC1 + 1024;    // 2 x 512 B: D
+constexpr uint32_t SM_BAR = SM_VEC2 + 1024;
+constexpr uint32_t SM_TOTAL = SM_BAR + 256;
+
+struct BwdTcParams {
+    const float* lse2p;
+    const float* dvecp;
+    ReplacedWs w;
+    void* dk;
+    void* dv;
+    unsigned int* err;
+    int16_t slot_of_head[kMaxHeads];
+    int H, T, Tp, nqb, grad_fp32;
+    float scale, scale_log2;
+};
+
+__device__ __forceinline__ void report(unsigned int* err, unsigned int code) {
+    atomicOr(err, 1u);
+    atomicCAS(err + 1, 0u, code);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Stores one 64-wide row of an fp32 accumulator (already scaled) as bf16 or fp32.
+__device__ __forceinline__ void store_row(void* base, int grad_fp32, size_t row, const float* v) {
+    if (grad_fp32) {
+        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + row * kHeadDim);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    } else {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + row * kHeadDim);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]), pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                                pack_bf16x2(v[8 * e + 4], v[8 * e + 5]), pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+              const __grid_constant__ CUtensorMap tmDQ, const BwdTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_addr(smem);
+    const uint32_t bar_kv = sb + SM_BAR;
+    const uint32_t bar_qf = bar_kv + 8;    // [2]
+    const uint32_t bar_qe = bar_qf + 16;   // [2]
+    const uint32_t bar_s = bar_qe + 16;
+    const uint32_t bar_dp = bar_s + 8;
+    const uint32_t bar_p = bar_dp + 8;     // 128 arrivals
+    const uint32_t bar_ds = bar_p + 8;     // 128 arrivals
+    const uint32_t bar_dsc = bar_ds + 8;   // tile's MMAs done with P/W/dS
+    const uint32_t bar_dqf = bar_dsc + 8;  // [2]
+    const uint32_t bar_dqe = bar_dqf + 16; // [2] 128 arrivals
+    const uint32_t bar_acc = bar_dqe + 16;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 192);
+
+    const int T = p.T;
+    const int bh = blockIdx.x;
+    const int J = (int)blockIdx.y;
+    const int h = bh % p.H;
+    const int slot = p.slot_of_head[h];
+    const bool rep = slot >= 0;
+    if (rep && p.w.flag[h] != 0) return;  // handled by the per-element exp path
+    const int ntiles = p.nqb - J;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kv, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_qf + 8 * s, 1);
+            mbar_init(bar_qe + 8 * s, 1);
+            mbar_init(bar_dqf + 8 * s, 1);
+            mbar_init(bar_dqe + 8 * s, 128);
+        }
+        mbar_init(bar_s, 1);
+        mbar_init(bar_dp, 1);
+        mbar_init(bar_p, 128);
+        mbar_init(bar_ds, 128);
+        mbar_init(bar_dsc, 1);
+        mbar_init(bar_acc, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            if (!rep) {
+                prefetch_tmap(&tmQ);
+                prefetch_tmap(&tmK);
+                prefetch_tmap(&tmV);
+                mbar_expect_tx(bar_kv, 2 * TILE);
+                tma_load_3d(sb + SM_K, &tmK, bar_kv, 0, J * BN, bh);
+                tma_load_3d(sb + SM_V, &tmV, bar_kv, 0, J * BN, bh);
+            }
+            prefetch_tmap(&tmDO);
+            for (int t = 0; t < ntiles; ++t) {
+                const int I = J + t, s = t & 1, n = t >> 1;
+                if (!mbar_wait(bar_qe + 8 * s, (n & 1) ^ 1, kWaitLimit)) { report(p.err, 0x1101); break; }
+                const uint32_t bq = bar_qf + 8 * s;
+                if (!rep) {
+                    mbar_expect_tx(bq, 2 * TILE + 1024);
+                    tma_load_3d(sb + SM_Q + s * TILE, &tmQ, bq, 0, I * BM, bh);
+                    tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, bh);
+                    bulk_load(sb + SM_VEC1 + 512 * s, p.lse2p + (size_t)bh * p.Tp + I * BM, 512, bq);
+                    bulk_load(sb + SM_VEC2 + 512 * s, p.dvecp + (size_t)bh * p.Tp + I * BM, 512, bq);
+                } else {
+                    mbar_expect_tx(bq, TILE + 512);
+                    tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, bh);
+                    bulk_load(sb + SM_VEC1 + 512 * s, p.w.rsc + (size_t)slot * p.w.Tp + I * BM, 512, bq);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // K-major x K-major, 128 x 128
+            const uint32_t idTS = idesc_bf16(128, 64, 0, 1);   // TMEM A x MN-major B, 128 x 64
+            const uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // MN-major A x MN-major B
+            const uint64_t dK = sw128_desc(sb + SM_K), dVd = sw128_desc(sb + SM_V);
+            const uint64_t dDS = sw128_desc(sb + SM_DS, 16384);
+            bool ok = rep || mbar_wait(bar_kv, 0, kWaitLimit);
+            if (!ok) report(p.err, 0x1201);
+            int t = 0;
+            for (; ok && t < ntiles; ++t) {
+                const int s = t & 1, n = t >> 1;
+                if (!mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x1202); ok = false; break; }
+                tc_fence_after();
+                const uint64_t dQs = sw128_desc(sb + SM_Q + s * TILE), dDOs = sw128_desc(sb + SM_DO + s * TILE);
+                if (!rep) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQs + 2 * k, idSS, k > 0);
+                    mma_commit(bar_s);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOs + 2 * k, idSS, k > 0);
+                    mma_commit(bar_dp);
+                    if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1203); ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tmem + C_DV, tmem + C_S + 8 * k, dDOs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+                    if (!mbar_wait(bar_ds, t & 1, kWaitLimit)) { report(p.err, 0x1204); ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tmem + C_DK, tmem + C_DP + 8 * k, dQs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+                    const int b = t & 1, nb = t >> 1;
+                    if (!mbar_wait(bar_dqe + 8 * b, (nb & 1) ^ 1, kWaitLimit)) { report(p.err, 0x1205); ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t cdq = b ? C_DQ1 : C_DQ0;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mma_ss(tmem + cdq, dDS + 128 * k, dK + 128 * k, idDQ, k > 0);
+                    mma_commit(bar_dqf + 8 * b);
+                } else {
+                    if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1206); ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tmem + C_DV, tmem + C_S + 8 * k, dDOs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mma_ts(tmem + C_DV, tmem + C_S + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
+                }
+                mma_commit(bar_dsc);
+                mma_commit(bar_qe + 8 * s);
+            }
+            if (ok) mma_commit(bar_acc);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ key rows
+        const int quarter = warp & 3;
+        const int jl = quarter * 32 + lane;  // key within the block = TMEM lane
+        const int j = J * BN + jl;
+        const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+        const uint32_t tS = tmem + lo + C_S, tDP = tmem + lo + C_DP;
+        const float* vec1 = reinterpret_cast<const float*>(smem + SM_VEC1);
+        const float* vec2 = reinterpret_cast<const float*>(smem + SM_VEC2);
+        bool ok = true;
+        for (int t = 0; t < ntiles; ++t) {
+            const int I = J + t, s = t & 1, n = t >> 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit));
+            if (!ok) { report(p.err, 0x1301); break; }
+            const float* v1 = vec1 + 128 * s;
+            if (!rep) {
+                const float* v2 = vec2 + 128 * s;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_s, t & 1, kWaitLimit));
+                if (!ok) { report(p.err, 0x1302); break; }
+                tc_fence_after();
+                const bool diag = (t == 0);
+                const bool key_ok = j < T;
+                uint32_t pw[64];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tS + 32 * c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int ql = 32 * c + e;
+                        float p0 = ex2(__uint_as_float(v[e]) * p.scale_log2 - v1[ql]);
+                        float p1 = ex2(__uint_as_float(v[e + 1]) * p.scale_log2 - v1[ql + 1]);
+                        if (!key_ok || (diag && ql < jl)) p0 = 0.f;
+                        if (!key_ok || (diag && ql + 1 < jl)) p1 = 0.f;
+                        pw[16 * c + e / 2] = pack_bf16x2(p0, p1);
+                    }
+                    if (c == 1) {
+                        uint32_t a[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) a[e] = pw[e];
+                        tmem_st32(tS, a);
+                    }
+                }
+                {
+                    uint32_t a[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = pw[32 + e];
+                    tmem_st32(tS + 32, a);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_p);
+                // dS^T = P^T o (dP^T - D)
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, t & 1, kWaitLimit));
+                if (!ok) { report(p.err, 0x1303); break; }
+                tc_fence_after();
+                uint32_t dsw[64];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tDP + 32 * c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int ql = 32 * c + e;
+                        const float2 pp = unpack_bf16x2(pw[16 * c + e / 2]);
+                        const float d0 = pp.x * (__uint_as_float(v[e]) - v2[ql]);
+                        const float d1 = pp.y * (__uint_as_float(v[e + 1]) - v2[ql + 1]);
+                        dsw[16 * c + e / 2] = pack_bf16x2(d0, d1);
+                    }
+                    // the same values, as row jl of the MN-major A operand of dQ = dS K
+                    const uint32_t blk = sb + SM_DS + (c >> 1) * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int cc = (c & 1) * 4 + u;
+                        const uint32_t addr = blk + ((cc ^ (jl & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
+                                     "r"(dsw[16 * c + 4 * u]), "r"(dsw[16 * c + 4 * u + 1]),
+                                     "r"(dsw[16 * c + 4 * u + 2]), "r"(dsw[16 * c + 4 * u + 3])
+                                     : "memory");
+                    }
+                    if (c == 1) {
+                        uint32_t a[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) a[e] = dsw[e];
+                        tmem_st32(tDP, a);
+                    }
+                }
+                {
+                    uint32_t a[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = dsw[32 + e];
+                    tmem_st32(tDP + 32, a);
+                }
+                fence_proxy_async_smem();
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_ds);
+            } else {
+                // W^T(j, i) = E[i-j] r_i, hi + lo bf16
+                if (t > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dsc, (t - 1) & 1, kWaitLimit));
+                    if (!ok) { report(p.err, 0x1304); break; }
+                }
+                tc_fence_after();
+                const float* ef = p.w.ef + (size_t)slot * p.w.Lp + 128 + (I - J) * BM - jl;
+                uint32_t hw[64], lw[64];
+#pragma unroll
+                for (int e = 0; e < 128; e += 2) {
+                    const float w0 = __ldg(ef + e) * v1[e];
+                    const float w1 = __ldg(ef + e + 1) * v1[e + 1];
+                    const uint32_t hb = pack_bf16x2(w0, w1);
+                    const float2 hf = unpack_bf16x2(hb);
+                    hw[e / 2] = hb;
+                    lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                }
+                {
+                    uint32_t a[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = hw[e];
+                    tmem_st32(tS, a);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = hw[32 + e];
+                    tmem_st32(tS + 32, a);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = lw[e];
+                    tmem_st32(tS + 64, a);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = lw[32 + e];
+                    tmem_st32(tS + 96, a);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_p);
+            }
+        }
+        // dK, dV epilogue
+        if (ok) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_acc, 0, kWaitLimit));
+            if (!ok) report(p.err, 0x1305);
+        }
+        tc_fence_after();
+        if (ok) {
+            float vals[64];
+            const float cj = (rep && j < T) ? p.w.cf[(size_t)slot * p.w.Tp + j] : 1.f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lo + C_DV + 32 * c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) vals[32 * c + e] = __uint_as_float(v[e]) * cj;
+            }
+            if (j < T) store_row(p.dv, p.grad_fp32, (size_t)bh * T + j, vals);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lo + C_DK + 32 * c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) vals[32 * c + e] = rep ? 0.f : __uint_as_float(v[e]) * p.scale;
+            }
+            if (j < T) store_row(p.dk, p.grad_fp32, (size_t)bh * T + j, vals);
+        }
+    } else if (!rep) {
+        // ------------------------------------------------ dQ tiles -> global accumulator
+        const int quarter = warp & 3;
+        const int ql = quarter * 32 + lane;
+        const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+        const bool leader = (warp == 6 && lane == 0);
+        bool ok = true;
+        // every thread passes both named barriers of every tile, even after a
+        // timed-out wait (then it only skips the work), so none is left behind
+        for (int t = 0; t < ntiles; ++t) {
+            const int I = J + t, b = t & 1, nb = t >> 1;
+            if (ok) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_dqf + 8 * b, nb & 1, kWaitLimit));
+                if (!ok) report(p.err, 0x1401);
+            }
+            if (!ok) {
+                named_sync(1, 128);
+                named_sync(1, 128);
+                continue;
+            }
+            tc_fence_after();
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tmem + lo + (b ? C_DQ1 : C_DQ0), v0);
+            tmem_ld32(tmem + lo + (b ? C_DQ1 : C_DQ0) + 32, v1);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar_dqe + 8 * b);
+            // row ql of the [128][64] fp32 staging tile; chunk order rotated by row
+            const uint32_t rowa = sb + SM_DQ + ql * 256;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int ch = (u + ql) & 15;
+                const uint32_t* src = (ch < 8) ? &v0[4 * ch] : &v1[4 * (ch - 8)];
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowa + (ch << 4)), "r"(src[0]),
+                             "r"(src[1]), "r"(src[2]), "r"(src[3])
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            named_sync(1, 128);
+            if (leader) {
+                tma_reduce_add_3d(&tmDQ, sb + SM_DQ, 0, I * BM, bh);
+                bulk_commit();
+                bulk_wait_read0();
+            }
+            named_sync(1, 128);
+        }
+        if (leader) bulk_wait0();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// rows of [BH, Tp]: lse2 = lse*log2(e) (+inf past T), D = rowsum(dO o O) (0
+// past T); zero the dQ accumulator rows.  8 threads per row.
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ dout,
+                                                      const float* __restrict__ lse, int T, int Tp, int64_t rows,
+                                                      float* __restrict__ lse2p, float* __restrict__ dvecp,
+                                                      float* __restrict__ dqacc) {
+    const int64_t r = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);
+    const int part = threadIdx.x & 7;
+    if (r >= rows) return;
+    const int64_t bh = r / Tp;
+    const int i = (int)(r - bh * Tp);
+    float acc = 0.f;
+    if (i < T) {
+        const int64_t row = bh * T + i;
+        const uint4 ov = *reinterpret_cast<const uint4*>(o + row * kHeadDim + part * 8);
+        const uint4 dv = *reinterpret_cast<const uint4*>(dout + row * kHeadDim + part * 8);
+        const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 a = unpack_bf16x2(ow[e]), b = unpack_bf16x2(dw[e]);
+            acc = fmaf(a.x, b.x, acc);
+            acc = fmaf(a.y, b.y, acc);
+        }
+        float4* z = reinterpret_cast<float4*>(dqacc + row * kHeadDim + part * 8);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (part == 0) {
+        dvecp[r] = i < T ? acc : 0.f;
+        lse2p[r] = i < T ? lse[bh * T + i] * kLog2e : -kNegInf;
+    }
+}
+
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc, void* __restrict__ dq,
+                                                         int64_t n4, int grad_fp32, float scale) {
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n4;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4*>(acc)[idx];
+        if (grad_fp32) {
+            reinterpret_cast<float4*>(dq)[idx] = make_float4(a.x * scale, a.y * scale, a.z * scale, a.w * scale);
+        } else {
+            reinterpret_cast<uint2*>(dq)[idx] =
+                make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+        }
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+}  // namespace
+
+// [BH, T, 64] fp32 as a 3-D tensor (d, t, bh); 128 x 64 boxes, no swizzle.
+bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out) {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {64 * 4, (cuuint64_t)T * 64 * 4};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int BH, int T,
+                           float* lse2p, float* dvecp, float* dqacc, cudaStream_t stream) {
+    const int Tp = round_up128(T);
+    const int64_t rows = (int64_t)BH * Tp;
+    if (rows == 0) return cudaSuccess;
+    launch_begin(KID_BWD_PRE, stream);
+    bwd_pre_kernel<<<(unsigned)((rows + 31) / 32), 256, 0, stream>>>(o, dout, lse, T, Tp, rows, lse2p, dvecp, dqacc);
+    launch_end(KID_BWD_PRE, stream);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream) {
+    const int64_t n4 = rows * kHeadDim / 4;
+    if (n4 == 0) return cudaSuccess;
+    const int64_t blocks = (n4 + 255) / 256;
+    launch_begin(KID_DQ_CONVERT, stream);
+    dq_convert_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, stream>>>(dqacc, dq, n4,
+                                                                                            grad_fp32, 0.125f);
+    launch_end(KID_DQ_CONVERT, stream);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                          const __nv_bfloat16* dout, const float* lse2p, const float* dvecp, float* dqacc,
+                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, void* dk, void* dv,
+                          int grad_fp32, unsigned int* err, cudaStream_t stream) {
+    const int BH = B * H;
+    CUtensorMap mq, mk, mv, mdo, mdq;
+    if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, BH, T, &mk) || !make_tmap_bhtd(v, BH, T, &mv) ||
+        !make_tmap_bhtd(dout, BH, T, &mdo) || !make_tmap_bhtd_f32(dqacc, BH, T, &mdq))
+        return cudaErrorNotSupported;
+    BwdTcParams p;
+    p.lse2p = lse2p;
+    p.dvecp = dvecp;
+    p.w = w;
+    p.dk = dk;
+    p.dv = dv;
+    p.err = err;
+    int slot = 0;
+    for (int hh = 0; hh < kMaxHeads; ++hh) p.slot_of_head[hh] = -1;
+    for (int hh = 0; hh < H; ++hh)
+        if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
+    p.H = H;
+    p.T = T;
+    p.Tp = round_up128(T);
+    p.nqb = (T + BM - 1) / BM;
+    p.grad_fp32 = grad_fp32;
+    p.scale = 0.125f;
+    p.scale_log2 = kLog2e * 0.125f;
+    const int smem = SM_TOTAL + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    launch_begin(KID_BWD_TC, stream);
+    bwd_tc_kernel<<<dim3(BH, p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
+    launch_end(KID_BWD_TC, stream);
+    return cudaGetLastError();
+}
+
+}  // namespace saf

@@ -1,6 +1,7 @@
 // Shared definitions of the sm_100a mixed-head attention library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -50,6 +51,9 @@ struct WsLayout {
     size_t logz;     // [H, T] fp32 (used when the caller passes logz = NULL)
     size_t dvec;     // [B, H, T] fp32 row terms rowsum(dO o O) (backward only)
     size_t epair, ef, cpair, cf, rsc, flag;  // factored replaced-head arrays (H slots)
+    size_t lse2p;    // [B*H, Tp] fp32 lse * log2(e), +inf past T   (backward)
+    size_t dvecp;    // [B*H, Tp] fp32 rowsum(dO o O), 0 past T      (backward)
+    size_t dqacc;    // [B*H, T, 64] fp32 dQ accumulator              (backward)
     size_t total;
 };
 
@@ -68,6 +72,12 @@ inline WsLayout ws_layout(int B, int H, int T, int is_bwd) {
     L.cf = off; off = align256(off + 4 * (size_t)H * Tp);
     L.rsc = off; off = align256(off + 4 * (size_t)H * Tp);
     L.flag = off; off = align256(off + 4 * (size_t)H);
+    if (is_bwd) {
+        const size_t BH = (size_t)B * H;
+        L.lse2p = off; off = align256(off + 4 * BH * Tp);
+        L.dvecp = off; off = align256(off + 4 * BH * Tp);
+        L.dqacc = off; off = align256(off + 4 * BH * (size_t)T * kHeadDim);
+    }
     L.total = off;
     return L;
 }
@@ -114,6 +124,19 @@ cudaError_t launch_prep_replaced(const float* a, const float* r, const float* lo
 cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           __nv_bfloat16* o, float* lse, const float* logz, const HeadList& hl,
                           const ReplacedWs& w, int B, int H, int T, unsigned int* err, cudaStream_t stream);
+// Backward preprocessing for the tensor-core backward: padded lse*log2(e) and
+// rowsum(dO o O), and a zeroed dQ accumulator.
+cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int BH, int T,
+                           float* lse2p, float* dvecp, float* dqacc, cudaStream_t stream);
+// Tensor-core backward (dK, dV written; dQ reduced into dqacc).
+cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                          const __nv_bfloat16* dout, const float* lse2p, const float* dvecp, float* dqacc,
+                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, void* dk, void* dv,
+                          int grad_fp32, unsigned int* err, cudaStream_t stream);
+// dq = dqacc / sqrt(d_h) in the requested dtype.
+cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream);
+bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out);
+bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out);
 // head_only_flag != nullptr: run only replaced heads h with head_only_flag[h] != 0.
 cudaError_t launch_fwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, __nv_bfloat16* o, float* lse,
@@ -127,6 +150,7 @@ cudaError_t launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const float* lse, const float* dvec,
                            const float* a, const float* r, const float* logz,
                            const HeadList& hl, int B, int H, int T,
-                           void* dq, void* dk, void* dv, int grad_fp32, cudaStream_t stream);
+                           void* dq, void* dk, void* dv, int grad_fp32, cudaStream_t stream,
+                           const int* head_only_flag = nullptr);
 
 }  // namespace saf

@@ -61,6 +61,27 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// 3-D tiled reduce-add shared memory -> global (fp32), bulk-group completion.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+// Plain bulk copy global -> shared (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+// Barrier among `count` threads (a multiple of 32) with id 1..15.
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -113,15 +134,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // (rows = M or N index, 64 K elements per row) and an MN-major operand
 // (rows = K index, 64 MN elements per row): sbo = 1024 bytes between 8-row
 // groups.  lbo (unused for a single 128-byte-wide atom) is set to 16 bytes.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_byte_addr) {
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_byte_addr, uint32_t lbo_bytes = 16) {
     uint64_t d = 0;
     d |= (uint64_t)((smem_byte_addr >> 4) & 0x3FFF);  // start address
-    d |= (uint64_t)1 << 16;                            // leading byte offset (16 B)
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;  // leading byte offset
     d |= (uint64_t)(1024 >> 4) << 32;                  // stride byte offset
     d |= (uint64_t)1 << 46;                            // descriptor version (sm_100)
     d |= (uint64_t)2 << 61;                            // 128-byte swizzle
     return d;
 }
+// For an MN-major operand wider than one 64-element atom, `lbo_bytes` is the
+// distance between consecutive atoms along M (or N).
 
 // Instruction descriptor: bf16 x bf16 -> fp32, M x N, operand majorness.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
