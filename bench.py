@@ -4,9 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference]
 
-One step is the whole hot path on one batch: the forward call (replaced-head
-log-normalisers + fused forward) and the backward call (log-normalisers,
-row terms, fused backward), all through the C ABI, inputs resident in HBM.
+One step is the whole hot path on one batch, all through the C ABI with the
+inputs resident in HBM: the replaced heads' log-normalisers (computed once
+per step and reused by both passes, like lse), the forward call and the
+backward call (row terms, fused backward, dQ conversion).
 Default workload: the 124M-shape layer B=8, H=12 (3 replaced), T=4096,
 d_h=64, forward + backward.
 
@@ -273,10 +274,18 @@ def our_arm(args, world, rank, local):
     ws_b = saf.new_workspace(B, H, T, dev, backward=True) if w.backward else None
     stream = torch.cuda.current_stream(dev)
 
+    logz = torch.zeros(H, T, dtype=torch.float32, device=dev)
+
     def step():
-        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, out=o, lse=lse, workspace=ws_f)
+        # one training step of the layer: the replaced heads' log-normalisers
+        # once (the backward reuses them, like lse), then forward and backward
+        if n_r:
+            saf.replaced_lognorm(x["alpha"], x["rho"], mask, out=logz)
+        lz = logz if n_r else None
+        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, logz=lz, out=o, lse=lse,
+                           workspace=ws_f)
         if w.backward:
-            saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask,
+            saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask, logz=lz,
                                grad_dtype=gd, dq=dq, dk=dk, dv=dv, workspace=ws_b)
 
     torch.cuda.synchronize()
@@ -306,8 +315,8 @@ def our_arm(args, world, rank, local):
 
     # ---- per-kernel timing (separate pass, same steps, events around each launch)
     prof_steps = min(args.steps, 20)
-    per_launch = 6 if w.backward else 2
-    saf.profile_enable(prof_steps * (per_launch + 4))
+    per_step = max(1, launches // max(1, args.steps))
+    saf.profile_enable(prof_steps * per_step + 16)
     for _ in range(prof_steps):
         step()
     torch.cuda.synchronize()

@@ -44,8 +44,10 @@ constexpr uint32_t SM_V = SM_K + TILE;
 constexpr uint32_t SM_Q = SM_V + TILE;        // 2 stages
 constexpr uint32_t SM_DO = SM_Q + 2 * TILE;   // 2 stages
 constexpr uint32_t SM_DS = SM_DO + 2 * TILE;  // 32 KB: dS^T as two 64-query atoms
-constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;  // 32 KB fp32 [128][64] staging
-constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;  // 2 x 512 B: lse2 (ordinary) / r (replaced)
+// dQ staging, 2 buffers x 32 KB: each buffer is two [128][32] fp32 boxes
+// (columns 0..31 and 32..63) with the 128-byte swizzle of the reduce map
+constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;
+constexpr uint32_t SM_VEC1 = SM_DQ + 4 * TILE;  // 2 x 512 B: lse2 (ordinary) / r (replaced)
 constexpr uint32_t SM_VEC2 = SM_VEC1 + 1024;    // 2 x 512 B: D
 constexpr uint32_t SM_BAR = SM_VEC2 + 1024;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
@@ -69,6 +71,30 @@ __device__ __forceinline__ void report(unsigned int* err, unsigned int code) {
 
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// P^T for queries [32c, 32c + 32) of key row jl: exp2(S^T * scale - lse2),
+// packed as 16 bf16 pairs over TMEM columns [16c, 16c + 16) of the S^T region.
+// MASK: zero where the query precedes the key on the diagonal tile, or where
+// the key lies past T.
+template <bool MASK>
+__device__ __forceinline__ void p_chunk(uint32_t tS, int c, const float* lse2, float scale, int jl, bool diag,
+                                        bool key_ok) {
+    uint32_t v[32], pw[16];
+    tmem_ld32(tS + 32 * c, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        const int ql = 32 * c + e;
+        float p0 = ex2(fmaf(__uint_as_float(v[e]), scale, -lse2[ql]));
+        float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, -lse2[ql + 1]));
+        if (MASK) {
+            if (!key_ok || (diag && ql < jl)) p0 = 0.f;
+            if (!key_ok || (diag && ql + 1 < jl)) p1 = 0.f;
+        }
+        pw[e / 2] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(tS + 16 * c, pw);
 }
 
 // Stores one 64-wide row of an fp32 accumulator (already scaled) as bf16 or fp32.
@@ -107,13 +133,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 192);
 
     const int T = p.T;
-    const int bh = blockIdx.x;
-    const int J = (int)blockIdx.y;
+    // head-major order: the key blocks of one (b, h) run together and share
+    // its Q/dO tiles and dQ accumulator rows in L2; longest walks first
+    const int bh = (int)(blockIdx.x / (unsigned)p.nqb);
+    const int J = (int)(blockIdx.x % (unsigned)p.nqb);
     const int h = bh % p.H;
     const int slot = p.slot_of_head[h];
     const bool rep = slot >= 0;
     if (rep && p.w.flag[h] != 0) return;  // handled by the per-element exp path
     const int ntiles = p.nqb - J;
+    const bool ragged_keys = (J + 1) * BN > T;  // the key block runs past T
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -244,80 +273,47 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_s, t & 1, kWaitLimit));
                 if (!ok) { report(p.err, 0x1302); break; }
                 tc_fence_after();
-                const bool diag = (t == 0);
-                const bool key_ok = j < T;
-                uint32_t pw[64];
+                // P^T, 32 queries at a time: bf16 pairs written over the S^T
+                // columns already read (chunk c -> columns [16c, 16c + 16)).
+                // Masks only on the diagonal tile and in a ragged last key
+                // block (a warp-uniform choice: the TMEM ops are collective).
+                if (t == 0 || ragged_keys) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tS + 32 * c, v);
-                    tmem_wait_ld();
+                    for (int c = 0; c < 4; ++c) p_chunk<true>(tS, c, v1, p.scale_log2, jl, t == 0, j < T);
+                } else {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int ql = 32 * c + e;
-                        float p0 = ex2(__uint_as_float(v[e]) * p.scale_log2 - v1[ql]);
-                        float p1 = ex2(__uint_as_float(v[e + 1]) * p.scale_log2 - v1[ql + 1]);
-                        if (!key_ok || (diag && ql < jl)) p0 = 0.f;
-                        if (!key_ok || (diag && ql + 1 < jl)) p1 = 0.f;
-                        pw[16 * c + e / 2] = pack_bf16x2(p0, p1);
-                    }
-                    if (c == 1) {
-                        uint32_t a[32];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) a[e] = pw[e];
-                        tmem_st32(tS, a);
-                    }
-                }
-                {
-                    uint32_t a[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = pw[32 + e];
-                    tmem_st32(tS + 32, a);
+                    for (int c = 0; c < 4; ++c) p_chunk<false>(tS, c, v1, p.scale_log2, jl, false, true);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar_p);
-                // dS^T = P^T o (dP^T - D)
+                // dS^T = P^T o (dP^T - D): P^T read back from TMEM, dS^T written over
+                // the dP^T columns already read and, as row jl of the MN-major A
+                // operand of dQ = dS K, into shared memory
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, t & 1, kWaitLimit));
                 if (!ok) { report(p.err, 0x1303); break; }
                 tc_fence_after();
-                uint32_t dsw[64];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
+                    uint32_t v[32], pp[16], dsw[16];
                     tmem_ld32(tDP + 32 * c, v);
+                    tmem_ld16(tS + 16 * c, pp);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int ql = 32 * c + e;
-                        const float2 pp = unpack_bf16x2(pw[16 * c + e / 2]);
-                        const float d0 = pp.x * (__uint_as_float(v[e]) - v2[ql]);
-                        const float d1 = pp.y * (__uint_as_float(v[e + 1]) - v2[ql + 1]);
-                        dsw[16 * c + e / 2] = pack_bf16x2(d0, d1);
+                        const float2 pf = unpack_bf16x2(pp[e / 2]);
+                        dsw[e / 2] = pack_bf16x2(pf.x * (__uint_as_float(v[e]) - v2[ql]),
+                                                 pf.y * (__uint_as_float(v[e + 1]) - v2[ql + 1]));
                     }
-                    // the same values, as row jl of the MN-major A operand of dQ = dS K
+                    tmem_st16(tDP + 16 * c, dsw);
                     const uint32_t blk = sb + SM_DS + (c >> 1) * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const int cc = (c & 1) * 4 + u;
-                        const uint32_t addr = blk + ((cc ^ (jl & 7)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
-                                     "r"(dsw[16 * c + 4 * u]), "r"(dsw[16 * c + 4 * u + 1]),
-                                     "r"(dsw[16 * c + 4 * u + 2]), "r"(dsw[16 * c + 4 * u + 3])
-                                     : "memory");
+                        st_shared_v4(blk + ((cc ^ (jl & 7)) << 4), dsw[4 * u], dsw[4 * u + 1], dsw[4 * u + 2],
+                                     dsw[4 * u + 3]);
                     }
-                    if (c == 1) {
-                        uint32_t a[32];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) a[e] = dsw[e];
-                        tmem_st32(tDP, a);
-                    }
-                }
-                {
-                    uint32_t a[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = dsw[32 + e];
-                    tmem_st32(tDP + 32, a);
                 }
                 fence_proxy_async_smem();
                 tmem_wait_st();
@@ -331,30 +327,21 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 tc_fence_after();
                 const float* ef = p.w.ef + (size_t)slot * p.w.Lp + 128 + (I - J) * BM - jl;
-                uint32_t hw[64], lw[64];
 #pragma unroll
-                for (int e = 0; e < 128; e += 2) {
-                    const float w0 = __ldg(ef + e) * v1[e];
-                    const float w1 = __ldg(ef + e + 1) * v1[e + 1];
-                    const uint32_t hb = pack_bf16x2(w0, w1);
-                    const float2 hf = unpack_bf16x2(hb);
-                    hw[e / 2] = hb;
-                    lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
-                }
-                {
-                    uint32_t a[32];
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t hw[16], lw[16];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = hw[e];
-                    tmem_st32(tS, a);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = hw[32 + e];
-                    tmem_st32(tS + 32, a);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = lw[e];
-                    tmem_st32(tS + 64, a);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) a[e] = lw[32 + e];
-                    tmem_st32(tS + 96, a);
+                    for (int e = 0; e < 32; e += 2) {
+                        const int ql = 32 * c + e;
+                        const float w0 = __ldg(ef + ql) * v1[ql];
+                        const float w1 = __ldg(ef + ql + 1) * v1[ql + 1];
+                        const uint32_t hb = pack_bf16x2(w0, w1);
+                        const float2 hf = unpack_bf16x2(hb);
+                        hw[e / 2] = hb;
+                        lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                    }
+                    tmem_st16(tS + 16 * c, hw);
+                    tmem_st16(tS + 64 + 16 * c, lw);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -416,24 +403,27 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar_dqe + 8 * b);
-            // row ql of the [128][64] fp32 staging tile; chunk order rotated by row
-            const uint32_t rowa = sb + SM_DQ + ql * 256;
+            // staging buffer t&1 was last reduced from two tiles ago: the leader
+            // lets at most the newest reduce still be reading shared memory
+            if (leader) bulk_wait_read1();
+            named_sync(1, 128);
+            // row ql of the two [128][32] fp32 boxes, 16-byte chunks XOR-swizzled
+            // by row (the reduce map's 128-byte swizzle; conflict-free stores)
+            const uint32_t stg = sb + SM_DQ + (t & 1) * 32768 + ql * 128;
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int ch = (u + ql) & 15;
-                const uint32_t* src = (ch < 8) ? &v0[4 * ch] : &v1[4 * (ch - 8)];
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(rowa + (ch << 4)), "r"(src[0]),
-                             "r"(src[1]), "r"(src[2]), "r"(src[3])
-                             : "memory");
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t off = (uint32_t)((u ^ (ql & 7)) << 4);
+                st_shared_v4(stg + off, v0[4 * u], v0[4 * u + 1], v0[4 * u + 2], v0[4 * u + 3]);
+                st_shared_v4(stg + 16384 + off, v1[4 * u], v1[4 * u + 1], v1[4 * u + 2], v1[4 * u + 3]);
             }
             fence_proxy_async_smem();
             named_sync(1, 128);
             if (leader) {
-                tma_reduce_add_3d(&tmDQ, sb + SM_DQ, 0, I * BM, bh);
+                const uint32_t box = sb + SM_DQ + (t & 1) * 32768;
+                tma_reduce_add_3d(&tmDQ, box, 0, I * BM, bh);
+                tma_reduce_add_3d(&tmDQ, box + 16384, 32, I * BM, bh);
                 bulk_commit();
-                bulk_wait_read0();
             }
-            named_sync(1, 128);
         }
         if (leader) bulk_wait0();
     }
@@ -502,7 +492,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 }  // namespace
 
-// [BH, T, 64] fp32 as a 3-D tensor (d, t, bh); 128 x 64 boxes, no swizzle.
+// [BH, T, 64] fp32 as a 3-D tensor (d, t, bh); 128 x 32 boxes (128-byte rows)
+// with the 128-byte swizzle.
 bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out) {
     static EncodeTiledFn fn = nullptr;
     static bool tried = false;
@@ -517,10 +508,10 @@ bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out) {
     if (!fn) return false;
     cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)BH};
     cuuint64_t strides[2] = {64 * 4, (cuuint64_t)T * 64 * 4};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {32, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -577,7 +568,7 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     launch_begin(KID_BWD_TC, stream);
-    bwd_tc_kernel<<<dim3(BH, p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
+    bwd_tc_kernel<<<dim3((unsigned)BH * p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
     launch_end(KID_BWD_TC, stream);
     return cudaGetLastError();
 }

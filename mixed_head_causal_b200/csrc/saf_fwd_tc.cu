@@ -60,6 +60,75 @@ __device__ __forceinline__ void report(unsigned int* err, unsigned int code) {
     atomicCAS(err + 1, 0u, code);
 }
 
+// Row max of one 128-key block of raw scores in TMEM.  MASK: the diagonal
+// block, where keys past the row (or past T) do not count.
+template <bool MASK>
+__device__ __forceinline__ float row_max(uint32_t tS, int kbase, int i, int T) {
+    float mx = kNegInf;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            float s = __uint_as_float(v[e]);
+            if (MASK) {
+                const int key = kbase + 32 * c + e;
+                if (key > i || key >= T) s = kNegInf;
+            }
+            mx = fmaxf(mx, s);
+        }
+    }
+    return mx;
+}
+
+// P = exp2(s * scale - m) for keys [c0, c0 + 64) of the block, packed as 32
+// bf16 pairs; returns the sum of the (unrounded) probabilities.
+template <bool MASK>
+__device__ __forceinline__ float exp_half(uint32_t tS, int c0, int kbase, int i, int T, float scale, float m,
+                                          uint32_t (&pw)[32]) {
+    float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + c0 + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            float p0 = ex2(fmaf(__uint_as_float(v[e]), scale, -m));
+            float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, -m));
+            if (MASK) {
+                const int key = kbase + c0 + 32 * c + e;
+                if (key > i || key >= T) p0 = 0.f;
+                if (key + 1 > i || key + 1 >= T) p1 = 0.f;
+            }
+            l0 += p0;
+            l1 += p1;
+            pw[16 * c + e / 2] = pack_bf16x2(p0, p1);
+        }
+    }
+    return l0 + l1;
+}
+
+// W(i, j) = E[i-j] c_j for 64 keys (q0 = 0 or 8 selects the half): bf16 pair
+// products of the padded E pairs (walking down from row i) and the c pairs.
+__device__ __forceinline__ void build_w_half(const uint32_t* ep, const uint4* cp, int q0, uint32_t (&pw)[32]) {
+#pragma unroll
+    for (int q4 = 0; q4 < 8; ++q4) {
+        const uint4 c4 = __ldg(cp + q0 + q4);
+        const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int mm = 4 * (q0 + q4) + u;  // key pair (2mm, 2mm+1)
+            const uint32_t e2 = __ldg(ep - 2 * mm);
+            __nv_bfloat162 prod = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e2),
+                                          *reinterpret_cast<const __nv_bfloat162*>(&cw[u]));
+            pw[4 * q4 + u] = *reinterpret_cast<uint32_t*>(&prod);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(NTHREADS, 2)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const FwdTcParams p) {
@@ -76,8 +145,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 128);
 
     const int T = p.T;
-    const int bh = blockIdx.x;
-    const int I = p.nqb - 1 - (int)blockIdx.y;
+    // head-major order: the query blocks of one (b, h) run together and share
+    // its K/V tiles in L2; within a head, longest rows first
+    const int bh = (int)(blockIdx.x / (unsigned)p.nqb);
+    const int I = p.nqb - 1 - (int)(blockIdx.x % (unsigned)p.nqb);
     const int h = bh % p.H;
     const int slot = p.slot_of_head[h];
     const bool rep = slot >= 0;
@@ -171,28 +242,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float m = kNegInf, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
-            uint32_t pw[64];
+            uint32_t pw0[32], pw1[32];  // P (or W) as bf16 pairs: keys 0..63, 64..127
             if (!rep) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, kWaitLimit));
                 if (!ok) { report(p.err, 0x301); break; }
                 tc_fence_after();
                 const bool diag = (j == I);
                 const int kbase = j * BN;
-                // pass 1: row max of the scaled scores
-                float mx = kNegInf;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tS + 32 * c, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int key = kbase + 32 * c + e;
-                        float x = __uint_as_float(v[e]) * p.scale_log2;
-                        if (diag && (key > i || key >= T)) x = kNegInf;
-                        mx = fmaxf(mx, x);
-                    }
-                }
+                // pass 1: row max of the raw scores (the scale is positive);
+                // only the diagonal block has masked entries
+                const float mx = (diag ? row_max<true>(tS, kbase, i, T) : row_max<false>(tS, kbase, i, T)) *
+                                 p.scale_log2;
                 // the S -> P hand-off also needs the previous P.V finished
                 if (j > 0) {
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, kWaitLimit));
@@ -220,25 +280,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         tmem_st32(tO + 32 * c, v);
                     }
                 }
-                // pass 2: P = exp2(x - m) as bf16 pairs
-                const float mref = (m == kNegInf) ? 0.f : m;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tS + 32 * c, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int key = kbase + 32 * c + e;
-                        float x0 = __uint_as_float(v[e]) * p.scale_log2;
-                        float x1 = __uint_as_float(v[e + 1]) * p.scale_log2;
-                        float p0 = ex2(x0 - mref), p1 = ex2(x1 - mref);
-                        if (diag && (key > i || key >= T)) p0 = 0.f;
-                        if (diag && (key + 1 > i || key + 1 >= T)) p1 = 0.f;
-                        if (m == kNegInf) { p0 = 0.f; p1 = 0.f; }
-                        l += p0 + p1;
-                        pw[16 * c + e / 2] = pack_bf16x2(p0, p1);
-                    }
+                // pass 2: P = exp2(s * scale - m) as bf16 pairs (every row of
+                // a visited block has at least one visible key, so m is finite)
+                if (diag) {
+                    l += exp_half<true>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
+                    l += exp_half<true>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
+                } else {
+                    l += exp_half<false>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
+                    l += exp_half<false>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
                 }
             } else {
                 if (j > 0) {
@@ -248,28 +297,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 // W(i,j) = E[i-j] c_j, bf16 pairs
                 const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
                 const uint4* cp = reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
-#pragma unroll
-                for (int q4 = 0; q4 < 16; ++q4) {
-                    const uint4 c4 = __ldg(cp + q4);
-                    const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int mm = 4 * q4 + u;  // key pair (2mm, 2mm+1)
-                        const uint32_t e2 = __ldg(ep - 2 * mm);
-                        __nv_bfloat162 prod = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e2),
-                                                      *reinterpret_cast<const __nv_bfloat162*>(&cw[u]));
-                        pw[mm] = *reinterpret_cast<uint32_t*>(&prod);
-                    }
-                }
+                build_w_half(ep, cp, 0, pw0);
+                build_w_half(ep, cp, 8, pw1);
             }
             // P (or W) -> TMEM, then hand it to the MMA warp
-            {
-                uint32_t lo[32], hi[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) { lo[e] = pw[e]; hi[e] = pw[32 + e]; }
-                tmem_st32(tP, lo);
-                tmem_st32(tP + 32, hi);
-            }
+            tmem_st32(tP, pw0);
+            tmem_st32(tP + 32, pw1);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p);
@@ -382,7 +415,7 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     launch_begin(KID_FWD_TC, stream);
-    fwd_tc_kernel<<<dim3(BH, p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, p);
+    fwd_tc_kernel<<<dim3((unsigned)BH * p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, p);
     launch_end(KID_FWD_TC, stream);
     return cudaGetLastError();
 }
