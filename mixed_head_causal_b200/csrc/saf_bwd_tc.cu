@@ -79,8 +79,8 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
 // the key lies past T.
 template <bool MASK>
 __device__ __forceinline__ void p_chunk(uint32_t tS, int c, const float* lse2, float scale, int jl, bool diag,
-                                        bool key_ok) {
-    uint32_t v[32], pw[16];
+                                        bool key_ok, uint32_t (&pw)[16]) {
+    uint32_t v[32];
     tmem_ld32(tS + 32 * c, v);
     tmem_wait_ld();
 #pragma unroll
@@ -209,24 +209,46 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint64_t dDS = sw128_desc(sb + SM_DS, 16384);
             bool ok = rep || mbar_wait(bar_kv, 0, kWaitLimit);
             if (!ok) report(p.err, 0x1201);
+            // Ordinary heads run one tile ahead: S^T of tile t+1 is issued right
+            // after dV_t (the last reader of the P^T columns it overwrites) and
+            // dP^T of tile t+1 right after dQ_t, so the tensor cores work on the
+            // next tile while the row threads finish this one.  The tensor pipe
+            // executes one thread's MMAs in order, which orders those reuses.
+            auto issue_s = [&](int tt) {
+                const uint64_t dQn = sw128_desc(sb + SM_Q + (tt & 1) * TILE);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQn + 2 * k, idSS, k > 0);
+                mma_commit(bar_s);
+            };
+            auto issue_dp = [&](int tt) {
+                const uint64_t dDOn = sw128_desc(sb + SM_DO + (tt & 1) * TILE);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOn + 2 * k, idSS, k > 0);
+                mma_commit(bar_dp);
+            };
+            if (ok && !rep) {
+                if (!mbar_wait(bar_qf, 0, kWaitLimit)) { report(p.err, 0x1202); ok = false; }
+                tc_fence_after();
+                if (ok) { issue_s(0); issue_dp(0); }
+            }
             int t = 0;
             for (; ok && t < ntiles; ++t) {
                 const int s = t & 1, n = t >> 1;
-                if (!mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x1202); ok = false; break; }
-                tc_fence_after();
                 const uint64_t dQs = sw128_desc(sb + SM_Q + s * TILE), dDOs = sw128_desc(sb + SM_DO + s * TILE);
                 if (!rep) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQs + 2 * k, idSS, k > 0);
-                    mma_commit(bar_s);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOs + 2 * k, idSS, k > 0);
-                    mma_commit(bar_dp);
                     if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1203); ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
                         mma_ts(tmem + C_DV, tmem + C_S + 8 * k, dDOs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+                    const bool more = t + 1 < ntiles;
+                    if (more) {
+                        if (!mbar_wait(bar_qf + 8 * ((t + 1) & 1), ((t + 1) >> 1) & 1, kWaitLimit)) {
+                            report(p.err, 0x1207); ok = false; break;
+                        }
+                        tc_fence_after();
+                        issue_s(t + 1);
+                    }
                     if (!mbar_wait(bar_ds, t & 1, kWaitLimit)) { report(p.err, 0x1204); ok = false; break; }
                     tc_fence_after();
 #pragma unroll
@@ -239,7 +261,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                     for (int k = 0; k < 8; ++k) mma_ss(tmem + cdq, dDS + 128 * k, dK + 128 * k, idDQ, k > 0);
                     mma_commit(bar_dqf + 8 * b);
+                    if (more) issue_dp(t + 1);
                 } else {
+                    if (!mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x1202); ok = false; break; }
+                    tc_fence_after();
                     if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1206); ok = false; break; }
                     tc_fence_after();
 #pragma unroll
@@ -277,12 +302,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 // columns already read (chunk c -> columns [16c, 16c + 16)).
                 // Masks only on the diagonal tile and in a ragged last key
                 // block (a warp-uniform choice: the TMEM ops are collective).
+                // P^T stays in registers for dS^T: the S^T columns are reused by
+                // the next tile's S^T as soon as dV has read them.
+                uint32_t pw[4][16];
                 if (t == 0 || ragged_keys) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) p_chunk<true>(tS, c, v1, p.scale_log2, jl, t == 0, j < T);
+                    for (int c = 0; c < 4; ++c) p_chunk<true>(tS, c, v1, p.scale_log2, jl, t == 0, j < T, pw[c]);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) p_chunk<false>(tS, c, v1, p.scale_log2, jl, false, true);
+                    for (int c = 0; c < 4; ++c) p_chunk<false>(tS, c, v1, p.scale_log2, jl, false, true, pw[c]);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -295,14 +323,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32], pp[16], dsw[16];
+                    uint32_t v[32], dsw[16];
                     tmem_ld32(tDP + 32 * c, v);
-                    tmem_ld16(tS + 16 * c, pp);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int ql = 32 * c + e;
-                        const float2 pf = unpack_bf16x2(pp[e / 2]);
+                        const float2 pf = unpack_bf16x2(pw[c][e / 2]);
                         dsw[e / 2] = pack_bf16x2(pf.x * (__uint_as_float(v[e]) - v2[ql]),
                                                  pf.y * (__uint_as_float(v[e + 1]) - v2[ql + 1]));
                     }
