@@ -8,8 +8,9 @@
 //   warp 0      TMA producer: K, V once; Q, dO and the per-query vectors of
 //               each query block through a 2-stage ring
 //   warp 1      TMEM owner and MMA issuer (one thread)
-//   warps 2..5  one key row per thread: P^T, dS^T, dK/dV epilogue
-//   warps 6..9  one query row per thread: dQ tile TMEM -> smem -> reduce-add
+//   warps 2..9  key rows, two warps per row quarter (query columns 0..63 and
+//               64..127 of each tile): P^T, dS^T, and the dK/dV epilogue
+//   warps 10..13 one query row per thread: dQ tile TMEM -> smem -> reduce-add
 //
 // Ordinary head, per tile (rows = keys j, columns = queries i; the textbook
 // softmax-attention gradients, section 二.4 of the reading notes):
@@ -33,7 +34,7 @@ using namespace tc;
 
 constexpr int BM = 128;  // queries per block
 constexpr int BN = 128;  // keys per CTA
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 448;  // producer, MMA, 8 key-row warps, 4 dQ warps
 constexpr uint32_t TILE = 128 * 64 * 2;  // 16 KB bf16 tile
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ0 = 384, C_DQ1 = 448;
@@ -73,8 +74,15 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
+// TMEM column (relative to its fp32 region) of the bf16 pairs of query chunk
+// c: queries 0..63 pack into columns 0..31, queries 64..127 into 64..95, so
+// each half of a row only ever overwrites columns it has already read itself.
+__device__ __forceinline__ uint32_t packed_col(int c) { return c < 2 ? 16 * c : 64 + 16 * (c - 2); }
+// A-operand column of MMA k-step k (16 queries) in that packing.
+__device__ __forceinline__ uint32_t packed_kcol(int k) { return k < 4 ? 8 * k : 64 + 8 * (k - 4); }
+
 // P^T for queries [32c, 32c + 32) of key row jl: exp2(S^T * scale - lse2),
-// packed as 16 bf16 pairs over TMEM columns [16c, 16c + 16) of the S^T region.
+// packed as 16 bf16 pairs over TMEM columns packed_col(c) of the S^T region.
 // MASK: zero where the query precedes the key on the diagonal tile, or where
 // the key lies past T.
 template <bool MASK>
@@ -94,7 +102,7 @@ __device__ __forceinline__ void p_chunk(uint32_t tS, int c, const float* lse2, f
         }
         pw[e / 2] = pack_bf16x2(p0, p1);
     }
-    tmem_st16(tS + 16 * c, pw);
+    tmem_st16(tS + packed_col(c), pw);
 }
 
 // Stores one 64-wide row of an fp32 accumulator (already scaled) as bf16 or fp32.
@@ -155,8 +163,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
-        mbar_init(bar_p, 128);
-        mbar_init(bar_ds, 128);
+        mbar_init(bar_p, 256);
+        mbar_init(bar_ds, 256);
         mbar_init(bar_dsc, 1);
         mbar_init(bar_acc, 1);
         fence_mbar_init();
@@ -240,7 +248,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DV, tmem + C_S + 8 * k, dDOs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+                        mma_ts(tmem + C_DV, tmem + C_S + packed_kcol(k), dDOs + 128 * k, idTS,
+                               (t > 0 || k > 0) ? 1u : 0u);
                     const bool more = t + 1 < ntiles;
                     if (more) {
                         if (!mbar_wait(bar_qf + 8 * ((t + 1) & 1), ((t + 1) >> 1) & 1, kWaitLimit)) {
@@ -253,7 +262,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DK, tmem + C_DP + 8 * k, dQs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+                        mma_ts(tmem + C_DK, tmem + C_DP + packed_kcol(k), dQs + 128 * k, idTS,
+                               (t > 0 || k > 0) ? 1u : 0u);
                     const int b = t & 1, nb = t >> 1;
                     if (!mbar_wait(bar_dqe + 8 * b, (nb & 1) ^ 1, kWaitLimit)) { report(p.err, 0x1205); ok = false; break; }
                     tc_fence_after();
@@ -278,9 +288,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             if (ok) mma_commit(bar_acc);
         }
-    } else if (warp < 6) {
+    } else if (warp < 10) {
         // ------------------------------------------------ key rows
+        // two warps per TMEM lane quarter: `half` 0 takes query columns 0..63,
+        // half 1 columns 64..127 (all the work on a 32-column chunk is local)
         const int quarter = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int jl = quarter * 32 + lane;  // key within the block = TMEM lane
         const int j = J * BN + jl;
         const uint32_t lo = (uint32_t)(quarter * 32) << 16;
@@ -304,41 +317,45 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 // block (a warp-uniform choice: the TMEM ops are collective).
                 // P^T stays in registers for dS^T: the S^T columns are reused by
                 // the next tile's S^T as soon as dV has read them.
-                uint32_t pw[4][16];
+                uint32_t pw[2][16];
                 if (t == 0 || ragged_keys) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) p_chunk<true>(tS, c, v1, p.scale_log2, jl, t == 0, j < T, pw[c]);
+                    for (int cc = 0; cc < 2; ++cc)
+                        p_chunk<true>(tS, 2 * half + cc, v1, p.scale_log2, jl, t == 0, j < T, pw[cc]);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) p_chunk<false>(tS, c, v1, p.scale_log2, jl, false, true, pw[c]);
+                    for (int cc = 0; cc < 2; ++cc)
+                        p_chunk<false>(tS, 2 * half + cc, v1, p.scale_log2, jl, false, true, pw[cc]);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar_p);
-                // dS^T = P^T o (dP^T - D): P^T read back from TMEM, dS^T written over
-                // the dP^T columns already read and, as row jl of the MN-major A
-                // operand of dQ = dS K, into shared memory
+                // dS^T = P^T o (dP^T - D), P^T from registers; dS^T goes over the
+                // dP^T columns this warp has read and, as row jl of the MN-major
+                // A operand of dQ = dS K, into shared memory
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, t & 1, kWaitLimit));
                 if (!ok) { report(p.err, 0x1303); break; }
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * half + cc;
                     uint32_t v[32], dsw[16];
                     tmem_ld32(tDP + 32 * c, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int ql = 32 * c + e;
-                        const float2 pf = unpack_bf16x2(pw[c][e / 2]);
+                        const float2 pf = unpack_bf16x2(pw[cc][e / 2]);
                         dsw[e / 2] = pack_bf16x2(pf.x * (__uint_as_float(v[e]) - v2[ql]),
                                                  pf.y * (__uint_as_float(v[e + 1]) - v2[ql + 1]));
                     }
-                    tmem_st16(tDP + 16 * c, dsw);
-                    const uint32_t blk = sb + SM_DS + (c >> 1) * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
+                    tmem_st16(tDP + packed_col(c), dsw);
+                    // queries [64 half, 64 half + 64) form the MN atom `half`
+                    const uint32_t blk = sb + SM_DS + half * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int cc = (c & 1) * 4 + u;
-                        st_shared_v4(blk + ((cc ^ (jl & 7)) << 4), dsw[4 * u], dsw[4 * u + 1], dsw[4 * u + 2],
+                        const int ch = cc * 4 + u;
+                        st_shared_v4(blk + ((ch ^ (jl & 7)) << 4), dsw[4 * u], dsw[4 * u + 1], dsw[4 * u + 2],
                                      dsw[4 * u + 3]);
                     }
                 }
@@ -355,7 +372,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tc_fence_after();
                 const float* ef = p.w.ef + (size_t)slot * p.w.Lp + 128 + (I - J) * BM - jl;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * half + cc;
                     uint32_t hw[16], lw[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
@@ -382,33 +400,29 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         tc_fence_after();
         if (ok) {
+            // half 0 writes the dV row (times c_j for a replaced head), half 1
+            // the dK row (times 1/sqrt(d); zero for a replaced head)
             float vals[64];
-            const float cj = (rep && j < T) ? p.w.cf[(size_t)slot * p.w.Tp + j] : 1.f;
+            float mul;
+            if (half == 0) mul = (rep && j < T) ? p.w.cf[(size_t)slot * p.w.Tp + j] : 1.f;
+            else mul = rep ? 0.f : p.scale;
+            const uint32_t col = half == 0 ? C_DV : C_DK;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lo + C_DV + 32 * c, v);
+                tmem_ld32(tmem + lo + col + 32 * c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) vals[32 * c + e] = __uint_as_float(v[e]) * cj;
+                for (int e = 0; e < 32; ++e) vals[32 * c + e] = __uint_as_float(v[e]) * mul;
             }
-            if (j < T) store_row(p.dv, p.grad_fp32, (size_t)bh * T + j, vals);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lo + C_DK + 32 * c, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) vals[32 * c + e] = rep ? 0.f : __uint_as_float(v[e]) * p.scale;
-            }
-            if (j < T) store_row(p.dk, p.grad_fp32, (size_t)bh * T + j, vals);
+            if (j < T) store_row(half == 0 ? p.dv : p.dk, p.grad_fp32, (size_t)bh * T + j, vals);
         }
     } else if (!rep) {
         // ------------------------------------------------ dQ tiles -> global accumulator
         const int quarter = warp & 3;
         const int ql = quarter * 32 + lane;
         const uint32_t lo = (uint32_t)(quarter * 32) << 16;
-        const bool leader = (warp == 6 && lane == 0);
+        const bool leader = (warp == 10 && lane == 0);
         bool ok = true;
         // every thread passes both named barriers of every tile, even after a
         // timed-out wait (then it only skips the work), so none is left behind
