@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--grad-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head-cost", action="store_true",
+                    help="instead of the headline line, time the workload's shape with 0, 25, 50 and 100%% of "
+                         "the heads replaced and fit t = t0 + c_o n_o + c_r n_r per pass")
     return ap.parse_args()
 
 
@@ -403,11 +406,72 @@ def our_arm(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def head_cost(args, local):
+    """Per-head cost of each head kind: the workload's shape timed with
+    n_r = 0, H/4, H/2 and H replaced heads (the first n_r heads), forward and
+    backward separately, and a least-squares fit t = t0 + c_o n_o + c_r n_r."""
+    import numpy as np
+    from mixed_head_causal_b200 import saf
+    dev = torch.device("cuda", local)
+    base = I.WORKLOADS[args.workload]
+    rows = []
+    for n_r in sorted({0, base.H // 4, base.H // 2, base.H}):
+        w = I.custom(base.B, base.H, base.T, list(range(n_r)))
+        x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
+        mask = x["mask"]
+        lz = torch.zeros(w.H, w.T, dtype=torch.float32, device=dev)
+        if n_r:
+            saf.replaced_lognorm(x["alpha"], x["rho"], mask, out=lz)
+        lzp = lz if n_r else None
+        o = torch.empty_like(x["v"])
+        lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
+        g = [torch.empty_like(x["v"]) for _ in range(3)]
+        wsf = saf.new_workspace(w.B, w.H, w.T, dev, backward=False)
+        wsb = saf.new_workspace(w.B, w.H, w.T, dev, backward=True)
+
+        def fwd():
+            saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, logz=lzp, out=o, lse=lse,
+                               workspace=wsf)
+
+        def bwd():
+            saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask, logz=lzp,
+                               dq=g[0], dk=g[1], dv=g[2], workspace=wsb)
+
+        times = {}
+        for name, fn in (("fwd", fwd), ("bwd", bwd)):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(args.steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            times[name] = e0.elapsed_time(e1) / args.steps
+        rows.append((w.H - n_r, n_r, times["fwd"], times["bwd"]))
+        del x, o, lse, g, wsf, wsb
+        torch.cuda.empty_cache()
+    A = np.array([[1.0, r[0], r[1]] for r in rows])
+    out = {"metric": "per-head cost of ordinary vs replaced heads (ms per head per step)",
+           "config": {"workload": args.workload, "B": base.B, "H": base.H, "T": base.T, "d_h": base.d,
+                      "n_replaced_points": [r[1] for r in rows]},
+           "times_ms": [{"n_o": r[0], "n_r": r[1], "fwd": r[2], "bwd": r[3]} for r in rows]}
+    for name, col in (("fwd", 2), ("bwd", 3), ("fwd+bwd", None)):
+        y = np.array([r[2] + r[3] if col is None else r[col] for r in rows])
+        t0, c_o, c_r = np.linalg.lstsq(A, y, rcond=None)[0]
+        out[name] = {"t0_ms": t0, "c_o_ms": c_o, "c_r_ms": c_r, "c_r_over_c_o": c_r / c_o if c_o else None}
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
-        if args.impl == "reference":
+        if args.head_cost:
+            if rank == 0:
+                head_cost(args, local)
+        elif args.impl == "reference":
             reference_arm(args, world, rank)
         else:
             our_arm(args, world, rank, local)

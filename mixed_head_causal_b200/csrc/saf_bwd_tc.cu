@@ -138,6 +138,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_dqf = bar_dsc + 8;  // [2]
     const uint32_t bar_dqe = bar_dqf + 16; // [2] 128 arrivals
     const uint32_t bar_acc = bar_dqe + 16;
+    const uint32_t bar_wb = bar_acc + 8;   // [2] replaced head: W buffer b consumed
+    const uint32_t bar_pb = bar_wb + 16;   // [2] replaced head: W buffer b written (256 arrivals)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 192);
 
     const int T = p.T;
@@ -166,6 +168,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(bar_p, 256);
         mbar_init(bar_ds, 256);
         mbar_init(bar_dsc, 1);
+        mbar_init(bar_wb, 1);
+        mbar_init(bar_wb + 8, 1);
+        mbar_init(bar_pb, 256);
+        mbar_init(bar_pb + 8, 256);
         mbar_init(bar_acc, 1);
         fence_mbar_init();
     }
@@ -275,13 +281,21 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 } else {
                     if (!mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x1202); ok = false; break; }
                     tc_fence_after();
-                    if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1206); ok = false; break; }
+                    if (!mbar_wait(bar_pb + 8 * (t & 1), (t >> 1) & 1, kWaitLimit)) {
+                        report(p.err, 0x1206);
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
+                    // W of tile t sits in buffer t & 1 (the S^T or the dP^T
+                    // columns, both unused by a replaced head): hi, then lo
+                    const uint32_t wcol = C_S + 128 * (t & 1);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DV, tmem + C_S + 8 * k, dDOs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+                        mma_ts(tmem + C_DV, tmem + wcol + 8 * k, dDOs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) mma_ts(tmem + C_DV, tmem + C_S + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
+                    for (int k = 0; k < 8; ++k) mma_ts(tmem + C_DV, tmem + wcol + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
+                    mma_commit(bar_wb + 8 * (t & 1));
                 }
                 mma_commit(bar_dsc);
                 mma_commit(bar_qe + 8 * s);
@@ -364,9 +378,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tc_fence_before();
                 mbar_arrive(bar_ds);
             } else {
-                // W^T(j, i) = E[i-j] r_i, hi + lo bf16
-                if (t > 0) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dsc, (t - 1) & 1, kWaitLimit));
+                // W^T(j, i) = E[i-j] r_i, hi + lo bf16, into buffer t & 1; that
+                // buffer was last read by the MMAs of tile t - 2 (one barrier per
+                // buffer, so neither can run two phases ahead of this wait)
+                const uint32_t tW = tmem + lo + C_S + 128 * (t & 1);
+                if (t >= 2) {
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(bar_wb + 8 * (t & 1), ((t >> 1) & 1) ^ 1, kWaitLimit));
                     if (!ok) { report(p.err, 0x1304); break; }
                 }
                 tc_fence_after();
@@ -385,12 +403,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         hw[e / 2] = hb;
                         lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
                     }
-                    tmem_st16(tS + 16 * c, hw);
-                    tmem_st16(tS + 64 + 16 * c, lw);
+                    tmem_st16(tW + 16 * c, hw);
+                    tmem_st16(tW + 64 + 16 * c, lw);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar_p);
+                mbar_arrive(bar_pb + 8 * (t & 1));
             }
         }
         // dK, dV epilogue

@@ -111,6 +111,34 @@ __device__ __forceinline__ float exp_half(uint32_t tS, int c0, int kbase, int i,
     return l0 + l1;
 }
 
+// One pass over an off-diagonal block against a reference max m: P = exp2(s *
+// scale - m) as bf16 pairs for all 128 keys (64 TMEM columns per load batch),
+// the row sum in `l`, and the block's raw row max returned so the caller can
+// tell whether m was too small (then it redoes the block with two passes).
+__device__ __forceinline__ float exp_block_1pass(uint32_t tS, uint32_t tP, float scale, float m, float& l) {
+    float mx0 = kNegInf, mx1 = kNegInf, l0 = 0.f, l1 = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[64], pw[32];
+        tmem_ld32(tS + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tS + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+            const float s0 = __uint_as_float(v[e]), s1 = __uint_as_float(v[e + 1]);
+            mx0 = fmaxf(mx0, s0);
+            mx1 = fmaxf(mx1, s1);
+            const float p0 = ex2(fmaf(s0, scale, -m)), p1 = ex2(fmaf(s1, scale, -m));
+            l0 += p0;
+            l1 += p1;
+            pw[e / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tP + 32 * hh, pw);  // overwritten again if the block is redone
+    }
+    l += l0 + l1;
+    return fmaxf(mx0, mx1);
+}
+
 // W(i, j) = E[i-j] c_j for 64 keys (q0 = 0 or 8 selects the half): bf16 pair
 // products of the padded E pairs (walking down from row i) and the c pairs.
 __device__ __forceinline__ void build_w_half(const uint32_t* ep, const uint4* cp, int q0, uint32_t (&pw)[32]) {
@@ -141,7 +169,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_ke = bar_vf + 8 * NST;     // [NST] stage free
     const uint32_t bar_s = bar_ke + 8 * NST;      // S ready
     const uint32_t bar_p = bar_s + 8;             // P written (128 arrivals)
-    const uint32_t bar_o = bar_p + 8;             // P.V done
+    const uint32_t bar_o = bar_p + 8;             // P.V done (ordinary head)
+    const uint32_t bar_ob = bar_o + 8;            // [2] P.V of W buffer b done (replaced head)
+    const uint32_t bar_pb = bar_ob + 16;          // [2] W buffer b written (replaced head, 128 arrivals)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 128);
 
     const int T = p.T;
@@ -166,6 +196,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(bar_s, 1);
         mbar_init(bar_p, 128);
         mbar_init(bar_o, 1);
+        mbar_init(bar_ob, 1);
+        mbar_init(bar_ob + 8, 1);
+        mbar_init(bar_pb, 128);
+        mbar_init(bar_pb + 8, 128);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -220,13 +254,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     mma_commit(bar_s);
                 }
                 if (!mbar_wait(bar_vf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x203); break; }
-                if (!mbar_wait(bar_p, j & 1, kWaitLimit)) { report(p.err, 0x204); break; }
+                if (!(rep ? mbar_wait(bar_pb + 8 * (j & 1), (j >> 1) & 1, kWaitLimit)
+                          : mbar_wait(bar_p, j & 1, kWaitLimit))) {
+                    report(p.err, 0x204);
+                    break;
+                }
                 tc_fence_after();
                 const uint64_t dv = sw128_desc(sbase + SM_V + s * TILE_BYTES);
+                // a replaced head's W alternates between two buffers in the S
+                // columns (unused there), so building W_{j+1} overlaps this MMA
+                const uint32_t acol = rep ? 64 * (j & 1) : TP_COL;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
-                    mma_ts(tmem + TO_COL, tmem + TP_COL + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
-                mma_commit(bar_o);
+                    mma_ts(tmem + TO_COL, tmem + acol + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
+                mma_commit(rep ? bar_ob + 8 * (j & 1) : bar_o);
                 mma_commit(bar_ke + 8 * s);
             }
         }
@@ -243,73 +284,100 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
             uint32_t pw0[32], pw1[32];  // P (or W) as bf16 pairs: keys 0..63, 64..127
+            bool stored = false;        // the one-pass path writes P to TMEM itself
             if (!rep) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, kWaitLimit));
                 if (!ok) { report(p.err, 0x301); break; }
                 tc_fence_after();
                 const bool diag = (j == I);
                 const int kbase = j * BN;
-                // pass 1: row max of the raw scores (the scale is positive);
-                // only the diagonal block has masked entries
-                const float mx = (diag ? row_max<true>(tS, kbase, i, T) : row_max<false>(tS, kbase, i, T)) *
-                                 p.scale_log2;
-                // the S -> P hand-off also needs the previous P.V finished
+                // the S -> P hand-off also needs the previous P.V finished (it
+                // is: S_j was issued after it, and MMAs complete in order)
                 if (j > 0) {
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, kWaitLimit));
                     if (!ok) { report(p.err, 0x302); break; }
                 }
                 tc_fence_after();
-                float f = 1.f;
-                if (m == kNegInf) {
-                    m = mx;
-                } else if (mx > m + 8.f) {
-                    f = ex2(m - mx);
-                    l *= f;
-                    m = mx;
-                }
-                // TMEM loads/stores are warp-collective: rescale the O rows of
-                // the whole warp when any of its rows needs it (others use 1)
-                if (__any_sync(0xffffffffu, f != 1.f)) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(tO + 32 * c, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-                        tmem_st32(tO + 32 * c, v);
+                // Off-diagonal blocks after the first take one pass against the
+                // current row max m (the lazy max lets P reach 2^8); if a row's
+                // max grew past that slack the whole warp redoes the block with
+                // a max pass first (warp-uniform: TMEM ops are collective).
+                bool two_pass = diag || (m == kNegInf);
+                if (!two_pass) {
+                    float lt = 0.f;
+                    const float mx = exp_block_1pass(tS, tP, p.scale_log2, m, lt) * p.scale_log2;
+                    two_pass = __any_sync(0xffffffffu, mx > m + 8.f);
+                    if (!two_pass) {
+                        l += lt;
+                        stored = true;
                     }
                 }
-                // pass 2: P = exp2(s * scale - m) as bf16 pairs (every row of
-                // a visited block has at least one visible key, so m is finite)
-                if (diag) {
-                    l += exp_half<true>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
-                    l += exp_half<true>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
-                } else {
-                    l += exp_half<false>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
-                    l += exp_half<false>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
+                if (two_pass) {
+                    // pass 1: row max of the raw scores (the scale is positive);
+                    // only the diagonal block has masked entries
+                    const float mx =
+                        (diag ? row_max<true>(tS, kbase, i, T) : row_max<false>(tS, kbase, i, T)) * p.scale_log2;
+                    float f = 1.f;
+                    if (m == kNegInf) {
+                        m = mx;
+                    } else if (mx > m + 8.f) {
+                        f = ex2(m - mx);
+                        l *= f;
+                        m = mx;
+                    }
+                    // rescale the O rows of the whole warp when any row needs it
+                    if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t v[32];
+                            tmem_ld32(tO + 32 * c, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                            tmem_st32(tO + 32 * c, v);
+                        }
+                    }
+                    // pass 2: P = exp2(s * scale - m) as bf16 pairs (every row of
+                    // a visited block has at least one visible key, so m is finite)
+                    if (diag) {
+                        l += exp_half<true>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
+                        l += exp_half<true>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
+                    } else {
+                        l += exp_half<false>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
+                        l += exp_half<false>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
+                    }
                 }
             } else {
-                if (j > 0) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, kWaitLimit));
+                // W(i,j) = E[i-j] c_j, bf16 pairs, into buffer j & 1, last read
+                // by the P.V of block j - 2 (one barrier per buffer, so neither
+                // can run two phases ahead of this wait)
+                if (j >= 2) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_ob + 8 * (j & 1), ((j >> 1) & 1) ^ 1, kWaitLimit));
                     if (!ok) { report(p.err, 0x303); break; }
                 }
-                // W(i,j) = E[i-j] c_j, bf16 pairs
+                tc_fence_after();
                 const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
                 const uint4* cp = reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
                 build_w_half(ep, cp, 0, pw0);
                 build_w_half(ep, cp, 8, pw1);
+                tmem_st32(tS + 64 * (j & 1), pw0);
+                tmem_st32(tS + 64 * (j & 1) + 32, pw1);
+                stored = true;
             }
             // P (or W) -> TMEM, then hand it to the MMA warp
-            tmem_st32(tP, pw0);
-            tmem_st32(tP + 32, pw1);
+            if (!stored) {
+                tmem_st32(tP, pw0);
+                tmem_st32(tP + 32, pw1);
+            }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_p);
+            mbar_arrive(rep ? bar_pb + 8 * (j & 1) : bar_p);
         }
         // epilogue (TMEM reads by whole warps; rows past T are not stored)
         if (ok) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (nkb - 1) & 1, kWaitLimit));
+            const int jl = nkb - 1;  // the last P.V (MMAs complete in order)
+            ok = __all_sync(0xffffffffu, rep ? mbar_wait(bar_ob + 8 * (jl & 1), (jl >> 1) & 1, kWaitLimit)
+                                             : mbar_wait(bar_o, jl & 1, kWaitLimit));
             if (!ok) report(p.err, 0x304);
         }
         tc_fence_after();
