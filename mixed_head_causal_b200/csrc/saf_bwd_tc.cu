@@ -6,7 +6,7 @@
 // contribution is reduced into an fp32 accumulator in global memory with a
 // TMA reduce-add.  Warp roles:
 //   warp 0      TMA producer: K, V once; Q, dO and the per-query vectors of
-//               each query block through a 2-stage ring
+//               each query block through an NQS-stage ring
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2..9  key rows, two warps per row quarter (query columns 0..63 and
 //               64..127 of each tile): P^T, dS^T, and the dK/dV epilogue
@@ -42,15 +42,18 @@ constexpr long long kWaitLimit = 1ll << 31;
 
 constexpr uint32_t SM_K = 0;
 constexpr uint32_t SM_V = SM_K + TILE;
-constexpr uint32_t SM_Q = SM_V + TILE;        // 2 stages
-constexpr uint32_t SM_DO = SM_Q + 2 * TILE;   // 2 stages
-constexpr uint32_t SM_DS = SM_DO + 2 * TILE;  // 32 KB: dS^T as two 64-query atoms
-// dQ staging, 2 buffers x 32 KB: each buffer is two [128][32] fp32 boxes
-// (columns 0..31 and 32..63) with the 128-byte swizzle of the reduce map
+// Q/dO ring depth: a TMA round trip from L2 takes several tiles' worth of
+// MMA time, so the ring keeps NQS query blocks in flight
+constexpr int NQS = 3;
+constexpr uint32_t SM_Q = SM_V + TILE;          // NQS stages
+constexpr uint32_t SM_DO = SM_Q + NQS * TILE;   // NQS stages
+constexpr uint32_t SM_DS = SM_DO + NQS * TILE;  // 32 KB: dS^T as two 64-query atoms
+// dQ staging, 32 KB: two [128][32] fp32 boxes (columns 0..31 and 32..63)
+// with the 128-byte swizzle of the reduce map
 constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;
-constexpr uint32_t SM_VEC1 = SM_DQ + 4 * TILE;  // 2 x 512 B: lse2 (ordinary) / r (replaced)
-constexpr uint32_t SM_VEC2 = SM_VEC1 + 1024;    // 2 x 512 B: D
-constexpr uint32_t SM_BAR = SM_VEC2 + 1024;
+constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;     // NQS x 512 B: lse2 (ordinary) / r (replaced)
+constexpr uint32_t SM_VEC2 = SM_VEC1 + 512 * NQS;  // NQS x 512 B: D
+constexpr uint32_t SM_BAR = SM_VEC2 + 512 * NQS;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 
 struct BwdTcParams {
@@ -128,9 +131,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_addr(smem);
     const uint32_t bar_kv = sb + SM_BAR;
-    const uint32_t bar_qf = bar_kv + 8;    // [2]
-    const uint32_t bar_qe = bar_qf + 16;   // [2]
-    const uint32_t bar_s = bar_qe + 16;
+    const uint32_t bar_qf = bar_kv + 8;         // [NQS]
+    const uint32_t bar_qe = bar_qf + 8 * NQS;   // [NQS]
+    const uint32_t bar_s = bar_qe + 8 * NQS;
     const uint32_t bar_dp = bar_s + 8;
     const uint32_t bar_p = bar_dp + 8;     // 128 arrivals
     const uint32_t bar_ds = bar_p + 8;     // 128 arrivals
@@ -140,7 +143,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_acc = bar_dqe + 16;
     const uint32_t bar_wb = bar_acc + 8;   // [2] replaced head: W buffer b consumed
     const uint32_t bar_pb = bar_wb + 16;   // [2] replaced head: W buffer b written (256 arrivals)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 192);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 248);
+    static_assert(8 + 16 * NQS + 120 <= 248, "barrier area");
 
     const int T = p.T;
     // head-major order: the key blocks of one (b, h) run together and share
@@ -157,11 +161,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NQS; ++s) {
             mbar_init(bar_qf + 8 * s, 1);
             mbar_init(bar_qe + 8 * s, 1);
-            mbar_init(bar_dqf + 8 * s, 1);
-            mbar_init(bar_dqe + 8 * s, 128);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_dqf + 8 * b, 1);
+            mbar_init(bar_dqe + 8 * b, 128);
         }
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
@@ -197,7 +203,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             prefetch_tmap(&tmDO);
             for (int t = 0; t < ntiles; ++t) {
-                const int I = J + t, s = t & 1, n = t >> 1;
+                const int I = J + t, s = t % NQS, n = t / NQS;
                 if (!mbar_wait(bar_qe + 8 * s, (n & 1) ^ 1, kWaitLimit)) { report(p.err, 0x1101); break; }
                 const uint32_t bq = bar_qf + 8 * s;
                 if (!rep) {
@@ -229,13 +235,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             // next tile while the row threads finish this one.  The tensor pipe
             // executes one thread's MMAs in order, which orders those reuses.
             auto issue_s = [&](int tt) {
-                const uint64_t dQn = sw128_desc(sb + SM_Q + (tt & 1) * TILE);
+                const uint64_t dQn = sw128_desc(sb + SM_Q + (tt % NQS) * TILE);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQn + 2 * k, idSS, k > 0);
                 mma_commit(bar_s);
             };
             auto issue_dp = [&](int tt) {
-                const uint64_t dDOn = sw128_desc(sb + SM_DO + (tt & 1) * TILE);
+                const uint64_t dDOn = sw128_desc(sb + SM_DO + (tt % NQS) * TILE);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOn + 2 * k, idSS, k > 0);
                 mma_commit(bar_dp);
@@ -247,7 +253,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             int t = 0;
             for (; ok && t < ntiles; ++t) {
-                const int s = t & 1, n = t >> 1;
+                const int s = t % NQS, n = t / NQS;
                 const uint64_t dQs = sw128_desc(sb + SM_Q + s * TILE), dDOs = sw128_desc(sb + SM_DO + s * TILE);
                 if (!rep) {
                     if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1203); ok = false; break; }
@@ -258,7 +264,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                (t > 0 || k > 0) ? 1u : 0u);
                     const bool more = t + 1 < ntiles;
                     if (more) {
-                        if (!mbar_wait(bar_qf + 8 * ((t + 1) & 1), ((t + 1) >> 1) & 1, kWaitLimit)) {
+                        if (!mbar_wait(bar_qf + 8 * ((t + 1) % NQS), ((t + 1) / NQS) & 1, kWaitLimit)) {
                             report(p.err, 0x1207); ok = false; break;
                         }
                         tc_fence_after();
@@ -316,7 +322,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const float* vec2 = reinterpret_cast<const float*>(smem + SM_VEC2);
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
-            const int I = J + t, s = t & 1, n = t >> 1;
+            const int I = J + t, s = t % NQS, n = t / NQS;
             ok = __all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit));
             if (!ok) { report(p.err, 0x1301); break; }
             const float* v1 = vec1 + 128 * s;
@@ -462,13 +468,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar_dqe + 8 * b);
-            // staging buffer t&1 was last reduced from two tiles ago: the leader
-            // lets at most the newest reduce still be reading shared memory
-            if (leader) bulk_wait_read1();
+            // the staging buffer must have been read by the previous reduce
+            if (leader) bulk_wait_read0();
             named_sync(1, 128);
             // row ql of the two [128][32] fp32 boxes, 16-byte chunks XOR-swizzled
             // by row (the reduce map's 128-byte swizzle; conflict-free stores)
-            const uint32_t stg = sb + SM_DQ + (t & 1) * 32768 + ql * 128;
+            const uint32_t stg = sb + SM_DQ + ql * 128;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const uint32_t off = (uint32_t)((u ^ (ql & 7)) << 4);
@@ -478,7 +483,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             fence_proxy_async_smem();
             named_sync(1, 128);
             if (leader) {
-                const uint32_t box = sb + SM_DQ + (t & 1) * 32768;
+                const uint32_t box = sb + SM_DQ;
                 tma_reduce_add_3d(&tmDQ, box, 0, I * BM, bh);
                 tma_reduce_add_3d(&tmDQ, box + 16384, 32, I * BM, bh);
                 bulk_commit();
