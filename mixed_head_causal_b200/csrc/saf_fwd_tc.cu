@@ -4,7 +4,8 @@
 // One CTA computes one 128-row query block of one (batch, head) slice; both
 // head kinds share the grid, which is ordered longest rows first.  Warp roles:
 //   warp 0      TMA producer: Q once, then K and V tiles of 128 keys through
-//               a 2-stage shared-memory ring (K is skipped for replaced heads)
+//               separate rings (3 K stages, 2 V stages), K one block ahead of
+//               V (K is skipped for replaced heads)
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2..5  one query row per thread: softmax / pattern builder, epilogue
 //
@@ -14,6 +15,9 @@
 //   P = exp2(S*log2e/sqrt(d) - m), row max m kept lazily (the O rescale is
 //       skipped unless m grows by more than 8 in log2 units), P as bf16 into TMEM
 //   O += P V_j              tcgen05 TS MMA (A = P from TMEM), fp32 in TMEM
+// The row threads copy S_j to registers and release its TMEM columns at once,
+// so the MMA warp issues S_{j+1} while they still work on block j; the MMA
+// order is S_0, S_1, PV_0, S_2, PV_1, ...
 // Replaced head (Eq. (3), section 二.3, in factored form): the tile
 //   W(i,j) = E[i-j] c_j     (bf16 pairs multiplied in registers, no exp)
 // is written to TMEM and O += W V_j; the epilogue scales row i by r_i, giving
@@ -30,7 +34,8 @@ using namespace tc;
 
 constexpr int BM = 128;          // query rows per CTA
 constexpr int BN = 128;          // keys per block
-constexpr int NST = 2;           // K/V ring stages
+constexpr int NSK = 3;           // K ring stages
+constexpr int NSV = 2;           // V ring stages
 constexpr int NTHREADS = 192;
 constexpr uint32_t TILE_BYTES = 128 * 64 * 2;  // one 128 x 64 bf16 tile
 constexpr uint32_t TMEM_COLS = 256;
@@ -40,8 +45,8 @@ constexpr long long kWaitLimit = 1ll << 31;                 // cycles
 // shared memory map (offsets from a 1024-aligned base)
 constexpr uint32_t SM_Q = 0;
 constexpr uint32_t SM_K = SM_Q + TILE_BYTES;
-constexpr uint32_t SM_V = SM_K + NST * TILE_BYTES;
-constexpr uint32_t SM_BAR = SM_V + NST * TILE_BYTES;
+constexpr uint32_t SM_V = SM_K + NSK * TILE_BYTES;
+constexpr uint32_t SM_BAR = SM_V + NSV * TILE_BYTES;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 
 struct FwdTcParams {
@@ -60,83 +65,45 @@ __device__ __forceinline__ void report(unsigned int* err, unsigned int code) {
     atomicCAS(err + 1, 0u, code);
 }
 
-// Row max of one 128-key block of raw scores in TMEM.  MASK: the diagonal
-// block, where keys past the row (or past T) do not count.
-template <bool MASK>
-__device__ __forceinline__ float row_max(uint32_t tS, int kbase, int i, int T) {
-    float mx = kNegInf;
+// The 128 raw scores of this thread's row of S, TMEM -> registers.
+__device__ __forceinline__ void load_s_row(uint32_t tS, uint32_t (&v)[128]) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + 32 * c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            float s = __uint_as_float(v[e]);
-            if (MASK) {
-                const int key = kbase + 32 * c + e;
-                if (key > i || key >= T) s = kNegInf;
-            }
-            mx = fmaxf(mx, s);
-        }
-    }
-    return mx;
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+    tmem_wait_ld();
 }
 
-// P = exp2(s * scale - m) for keys [c0, c0 + 64) of the block, packed as 32
-// bf16 pairs; returns the sum of the (unrounded) probabilities.
+// Row max of one 128-key block of raw scores.  MASK: the diagonal block,
+// where keys past the row (or past T) do not count.
 template <bool MASK>
-__device__ __forceinline__ float exp_half(uint32_t tS, int c0, int kbase, int i, int T, float scale, float m,
-                                          uint32_t (&pw)[32]) {
-    float l0 = 0.f, l1 = 0.f;
+__device__ __forceinline__ float row_max(const uint32_t (&v)[128], int kbase, int i, int T) {
+    float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + c0 + 32 * c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-            float p0 = ex2(fmaf(__uint_as_float(v[e]), scale, -m));
-            float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, -m));
-            if (MASK) {
-                const int key = kbase + c0 + 32 * c + e;
-                if (key > i || key >= T) p0 = 0.f;
-                if (key + 1 > i || key + 1 >= T) p1 = 0.f;
-            }
-            l0 += p0;
-            l1 += p1;
-            pw[16 * c + e / 2] = pack_bf16x2(p0, p1);
-        }
+    for (int e = 0; e < 128; ++e) {
+        float s = __uint_as_float(v[e]);
+        if (MASK && (kbase + e > i || kbase + e >= T)) s = kNegInf;
+        mx[e & 3] = fmaxf(mx[e & 3], s);
     }
-    return l0 + l1;
+    return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// One pass over an off-diagonal block against a reference max m: P = exp2(s *
-// scale - m) as bf16 pairs for all 128 keys (64 TMEM columns per load batch),
-// the row sum in `l`, and the block's raw row max returned so the caller can
-// tell whether m was too small (then it redoes the block with two passes).
-__device__ __forceinline__ float exp_block_1pass(uint32_t tS, uint32_t tP, float scale, float m, float& l) {
-    float mx0 = kNegInf, mx1 = kNegInf, l0 = 0.f, l1 = 0.f;
+// P = exp2(s * scale - m) for the 128 keys of the block as 64 bf16 pairs;
+// returns the sum of the (unrounded) probabilities.
+template <bool MASK>
+__device__ __forceinline__ float exp_row(const uint32_t (&v)[128], int kbase, int i, int T, float scale, float m,
+                                         uint32_t (&pw)[64]) {
+    float l[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        uint32_t v[64], pw[32];
-        tmem_ld32(tS + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tS + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-            const float s0 = __uint_as_float(v[e]), s1 = __uint_as_float(v[e + 1]);
-            mx0 = fmaxf(mx0, s0);
-            mx1 = fmaxf(mx1, s1);
-            const float p0 = ex2(fmaf(s0, scale, -m)), p1 = ex2(fmaf(s1, scale, -m));
-            l0 += p0;
-            l1 += p1;
-            pw[e / 2] = pack_bf16x2(p0, p1);
+    for (int e = 0; e < 128; e += 2) {
+        float p0 = ex2(fmaf(__uint_as_float(v[e]), scale, -m));
+        float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, -m));
+        if (MASK) {
+            if (kbase + e > i || kbase + e >= T) p0 = 0.f;
+            if (kbase + e + 1 > i || kbase + e + 1 >= T) p1 = 0.f;
         }
-        tmem_st32(tP + 32 * hh, pw);  // overwritten again if the block is redone
+        l[(e >> 1) & 3] += p0 + p1;
+        pw[e >> 1] = pack_bf16x2(p0, p1);
     }
-    l += l0 + l1;
-    return fmaxf(mx0, mx1);
+    return (l[0] + l[1]) + (l[2] + l[3]);
 }
 
 // W(i, j) = E[i-j] c_j for 64 keys (q0 = 0 or 8 selects the half): bf16 pair
@@ -164,15 +131,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bar_q = sbase + SM_BAR;
-    const uint32_t bar_kf = bar_q + 8;            // [NST]
-    const uint32_t bar_vf = bar_kf + 8 * NST;     // [NST]
-    const uint32_t bar_ke = bar_vf + 8 * NST;     // [NST] stage free
-    const uint32_t bar_s = bar_ke + 8 * NST;      // S ready
-    const uint32_t bar_p = bar_s + 8;             // P written (128 arrivals)
+    const uint32_t bar_kf = bar_q + 8;            // [NSK] K stage full
+    const uint32_t bar_ke = bar_kf + 8 * NSK;     // [NSK] K stage free (S MMA done)
+    const uint32_t bar_vf = bar_ke + 8 * NSK;     // [NSV] V stage full
+    const uint32_t bar_ve = bar_vf + 8 * NSV;     // [NSV] V stage free (P.V MMA done)
+    const uint32_t bar_s = bar_ve + 8 * NSV;      // S ready
+    const uint32_t bar_sf = bar_s + 8;            // S copied out by the rows (128 arrivals)
+    const uint32_t bar_p = bar_sf + 8;            // P written (128 arrivals)
     const uint32_t bar_o = bar_p + 8;             // P.V done (ordinary head)
     const uint32_t bar_ob = bar_o + 8;            // [2] P.V of W buffer b done (replaced head)
     const uint32_t bar_pb = bar_ob + 16;          // [2] W buffer b written (replaced head, 128 arrivals)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 128);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 192);
 
     const int T = p.T;
     // head-major order: the query blocks of one (b, h) run together and share
@@ -188,12 +157,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        for (int s = 0; s < NST; ++s) {
+        for (int s = 0; s < NSK; ++s) {
             mbar_init(bar_kf + 8 * s, 1);
-            mbar_init(bar_vf + 8 * s, 1);
             mbar_init(bar_ke + 8 * s, 1);
         }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(bar_vf + 8 * s, 1);
+            mbar_init(bar_ve + 8 * s, 1);
+        }
         mbar_init(bar_s, 1);
+        mbar_init(bar_sf, 128);
         mbar_init(bar_p, 128);
         mbar_init(bar_o, 1);
         mbar_init(bar_ob, 1);
@@ -223,16 +196,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mbar_expect_tx(bar_q, TILE_BYTES);
                 tma_load_3d(sbase + SM_Q, &tmQ, bar_q, 0, I * BM, bh);
             }
-            for (int j = 0; j < nkb; ++j) {
-                const int s = j % NST, n = j / NST;
-                if (!mbar_wait(bar_ke + 8 * s, (n & 1) ^ 1, kWaitLimit)) { report(p.err, 0x101); break; }
-                if (!rep) {
-                    mbar_expect_tx(bar_kf + 8 * s, TILE_BYTES);
-                    tma_load_3d(sbase + SM_K + s * TILE_BYTES, &tmK, bar_kf + 8 * s, 0, j * BN, bh);
-                }
+            // K_j is consumed by S_j, which runs a block ahead of P.V_j: the
+            // K loads go one block ahead of the V loads
+            auto load_k = [&](int j) -> bool {
+                const int s = j % NSK, n = j / NSK;
+                if (!mbar_wait(bar_ke + 8 * s, (n & 1) ^ 1, kWaitLimit)) return false;
+                mbar_expect_tx(bar_kf + 8 * s, TILE_BYTES);
+                tma_load_3d(sbase + SM_K + s * TILE_BYTES, &tmK, bar_kf + 8 * s, 0, j * BN, bh);
+                return true;
+            };
+            bool ok = rep || load_k(0);
+            for (int j = 0; ok && j < nkb; ++j) {
+                if (!rep && j + 1 < nkb && !load_k(j + 1)) { ok = false; break; }
+                const int s = j % NSV, n = j / NSV;
+                if (!mbar_wait(bar_ve + 8 * s, (n & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                 mbar_expect_tx(bar_vf + 8 * s, TILE_BYTES);
                 tma_load_3d(sbase + SM_V + s * TILE_BYTES, &tmV, bar_vf + 8 * s, 0, j * BN, bh);
             }
+            if (!ok) report(p.err, 0x101);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -240,19 +221,28 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
             const uint32_t idO = idesc_bf16(128, 64, 0, 1);   // P (TMEM) x V (MN-major)
             const uint64_t dq = sw128_desc(sbase + SM_Q);
-            bool ok = true;
-            if (!rep && !mbar_wait(bar_q, 0, kWaitLimit)) { report(p.err, 0x201); ok = false; }
-            for (int j = 0; ok && j < nkb; ++j) {
-                const int s = j % NST, n = j / NST;
-                if (!rep) {
-                    if (!mbar_wait(bar_kf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x202); break; }
-                    tc_fence_after();
-                    const uint64_t dk = sw128_desc(sbase + SM_K + s * TILE_BYTES);
+            // S_j = Q K_j^T into the S columns; frees K stage j when done
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % NSK, n = j / NSK;
+                if (!mbar_wait(bar_kf + 8 * s, n & 1, kWaitLimit)) return false;
+                tc_fence_after();
+                const uint64_t dk = sw128_desc(sbase + SM_K + s * TILE_BYTES);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
-                        mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
-                    mma_commit(bar_s);
+                for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
+                    mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
+                mma_commit(bar_s);
+                mma_commit(bar_ke + 8 * s);
+                return true;
+            };
+            bool ok = true;
+            if (!rep) ok = mbar_wait(bar_q, 0, kWaitLimit) && issue_s(0);
+            if (!ok) report(p.err, 0x201);
+            for (int j = 0; ok && j < nkb; ++j) {
+                if (!rep && j + 1 < nkb) {
+                    // S_{j+1} once the rows have copied S_j out of TMEM
+                    if (!mbar_wait(bar_sf, j & 1, kWaitLimit) || !issue_s(j + 1)) { report(p.err, 0x202); break; }
                 }
+                const int s = j % NSV, n = j / NSV;
                 if (!mbar_wait(bar_vf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x203); break; }
                 if (!(rep ? mbar_wait(bar_pb + 8 * (j & 1), (j >> 1) & 1, kWaitLimit)
                           : mbar_wait(bar_p, j & 1, kWaitLimit))) {
@@ -268,7 +258,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
                     mma_ts(tmem + TO_COL, tmem + acol + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
                 mma_commit(rep ? bar_ob + 8 * (j & 1) : bar_o);
-                mma_commit(bar_ke + 8 * s);
+                mma_commit(bar_ve + 8 * s);
             }
         }
     } else {
@@ -283,70 +273,54 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         float m = kNegInf, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
-            uint32_t pw0[32], pw1[32];  // P (or W) as bf16 pairs: keys 0..63, 64..127
-            bool stored = false;        // the one-pass path writes P to TMEM itself
             if (!rep) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, kWaitLimit));
                 if (!ok) { report(p.err, 0x301); break; }
                 tc_fence_after();
+                uint32_t v[128];
+                load_s_row(tS, v);
+                tc_fence_before();
+                mbar_arrive(bar_sf);  // the MMA warp may now overwrite S
                 const bool diag = (j == I);
                 const int kbase = j * BN;
-                // the S -> P hand-off also needs the previous P.V finished (it
-                // is: S_j was issued after it, and MMAs complete in order)
+                // row max of the block (the scale is positive); every row of a
+                // visited block has a visible key, so mx is finite.  The running
+                // max m moves only when the block's max exceeds it by more than
+                // 8 (log2 units), so P stays below 2^8 and O is rarely rescaled.
+                const float mx =
+                    (diag ? row_max<true>(v, kbase, i, T) : row_max<false>(v, kbase, i, T)) * p.scale_log2;
+                float f = 1.f;
+                if (m == kNegInf) {
+                    m = mx;
+                } else if (mx > m + 8.f) {
+                    f = ex2(m - mx);
+                    l *= f;
+                    m = mx;
+                }
+                uint32_t pw[64];  // P as bf16 pairs
+                l += diag ? exp_row<true>(v, kbase, i, T, p.scale_log2, m, pw)
+                          : exp_row<false>(v, kbase, i, T, p.scale_log2, m, pw);
+                // P_j replaces P_{j-1} in TMEM once P.V_{j-1} has read it; the
+                // O rows are rescaled (by the whole warp, when any row needs
+                // it) once that P.V has landed in O
                 if (j > 0) {
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, kWaitLimit));
                     if (!ok) { report(p.err, 0x302); break; }
+                    tc_fence_after();
                 }
-                tc_fence_after();
-                // Off-diagonal blocks after the first take one pass against the
-                // current row max m (the lazy max lets P reach 2^8); if a row's
-                // max grew past that slack the whole warp redoes the block with
-                // a max pass first (warp-uniform: TMEM ops are collective).
-                bool two_pass = diag || (m == kNegInf);
-                if (!two_pass) {
-                    float lt = 0.f;
-                    const float mx = exp_block_1pass(tS, tP, p.scale_log2, m, lt) * p.scale_log2;
-                    two_pass = __any_sync(0xffffffffu, mx > m + 8.f);
-                    if (!two_pass) {
-                        l += lt;
-                        stored = true;
-                    }
-                }
-                if (two_pass) {
-                    // pass 1: row max of the raw scores (the scale is positive);
-                    // only the diagonal block has masked entries
-                    const float mx =
-                        (diag ? row_max<true>(tS, kbase, i, T) : row_max<false>(tS, kbase, i, T)) * p.scale_log2;
-                    float f = 1.f;
-                    if (m == kNegInf) {
-                        m = mx;
-                    } else if (mx > m + 8.f) {
-                        f = ex2(m - mx);
-                        l *= f;
-                        m = mx;
-                    }
-                    // rescale the O rows of the whole warp when any row needs it
-                    if (__any_sync(0xffffffffu, f != 1.f)) {
+                if (__any_sync(0xffffffffu, f != 1.f)) {
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            uint32_t v[32];
-                            tmem_ld32(tO + 32 * c, v);
-                            tmem_wait_ld();
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + 32 * c, ov);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-                            tmem_st32(tO + 32 * c, v);
-                        }
-                    }
-                    // pass 2: P = exp2(s * scale - m) as bf16 pairs (every row of
-                    // a visited block has at least one visible key, so m is finite)
-                    if (diag) {
-                        l += exp_half<true>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
-                        l += exp_half<true>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
-                    } else {
-                        l += exp_half<false>(tS, 0, kbase, i, T, p.scale_log2, m, pw0);
-                        l += exp_half<false>(tS, 64, kbase, i, T, p.scale_log2, m, pw1);
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+                        tmem_st32(tO + 32 * c, ov);
                     }
                 }
+                tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
+                tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
             } else {
                 // W(i,j) = E[i-j] c_j, bf16 pairs, into buffer j & 1, last read
                 // by the P.V of block j - 2 (one barrier per buffer, so neither
@@ -356,19 +330,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     if (!ok) { report(p.err, 0x303); break; }
                 }
                 tc_fence_after();
+                uint32_t pw0[32], pw1[32];
                 const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
                 const uint4* cp = reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
                 build_w_half(ep, cp, 0, pw0);
                 build_w_half(ep, cp, 8, pw1);
                 tmem_st32(tS + 64 * (j & 1), pw0);
                 tmem_st32(tS + 64 * (j & 1) + 32, pw1);
-                stored = true;
             }
-            // P (or W) -> TMEM, then hand it to the MMA warp
-            if (!stored) {
-                tmem_st32(tP, pw0);
-                tmem_st32(tP + 32, pw1);
-            }
+            // hand P (or W) to the MMA warp
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(rep ? bar_pb + 8 * (j & 1) : bar_p);

@@ -6,52 +6,84 @@
 //    depends on a and r only, so it is computed once per head, not per batch.
 //  * dot: the backward row term D[i] = sum_c dO[i,c] O[i,c] of softmax
 //    attention (equal to sum_j P[i,j] dP[i,j]), one fp32 value per row.
+#include <algorithm>
+
 #include "saf_common.cuh"
 
 namespace saf {
 namespace {
 
 
-// Merge two (max, sum-of-exp2) pairs of a log2-domain log-sum-exp.
-__device__ __forceinline__ void lse2_merge(float& m, float& s, float m2, float s2) {
-    float M = fmaxf(m, m2);
-    if (M == kNegInf) return;  // both empty
-    float a = (m == kNegInf) ? 0.f : s * exp2f(m - M);
-    float b = (m2 == kNegInf) ? 0.f : s2 * exp2f(m2 - M);
-    m = M;
-    s = a + b;
-}
+// Tiling of the log-normaliser: a block owns 32 consecutive rows i (one per
+// lane) of one replaced head and walks k in chunks of kLnChunk staged in
+// shared memory; its 8 warps split each chunk 8 ways.  In a warp every lane
+// reads the same a[k] (a broadcast) and consecutive r[i-k] (no bank
+// conflicts).  Each lane keeps a log2-domain (max, sum) pair updated once per
+// 8 terms; the 8 per-warp partials of a row are merged at the end.
+constexpr int kLnRows = 32;
+constexpr int kLnWarps = 8;
+constexpr int kLnChunk = 256;
+constexpr int kLnSpan = kLnChunk + kLnRows;  // distinct d = i - k in one chunk
+constexpr float kLnFloor = -3.402823466e38f;  // finite "no term yet" maximum
 
-// One warp per row i of one replaced head; lanes stride over k and keep an
-// online (max, sum) pair, merged across the warp at the end.
-__global__ void __launch_bounds__(256) lognorm_kernel(const float* __restrict__ a,
-                                                      const float* __restrict__ r,
-                                                      HeadList hl, int T,
-                                                      float* __restrict__ logz) {
+__global__ void __launch_bounds__(kLnWarps * 32) lognorm_kernel(const float* __restrict__ a,
+                                                               const float* __restrict__ r,
+                                                               HeadList hl, int T,
+                                                               float* __restrict__ logz) {
+    __shared__ float sa[kLnChunk];
+    __shared__ float sr[kLnSpan];
+    __shared__ float pm[kLnWarps][32], ps[kLnWarps][32];
     const int h = hl.heads[blockIdx.y];
-    const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (i >= T) return;
+    const int i0 = blockIdx.x * kLnRows;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* ah = a + (size_t)h * T;
     const float* rh = r + (size_t)h * T;
-    float m = kNegInf, s = 0.f;
-    for (int k = lane; k <= i; k += 32) {
-        float x = (ah[k] + rh[i - k]) * kLog2e;
-        if (x == kNegInf) continue;
-        if (x > m) {
-            s = (m == kNegInf ? 0.f : s * exp2f(m - x)) + 1.f;
-            m = x;
-        } else {
-            s += exp2f(x - m);
+    const int kend = min(i0 + kLnRows, T);  // every k a row of this tile can reach
+    float m = kLnFloor, s = 0.f;
+    for (int k0 = 0; k0 < kend; k0 += kLnChunk) {
+        // sa[u] = a[k0 + u] and sr[q] = r[d] for d = i0 - k0 - (kLnChunk - 1) + q,
+        // both in log2 units; out-of-range entries are -inf (no term)
+        const int dbase = i0 - k0 - (kLnChunk - 1);
+        for (int u = threadIdx.x; u < kLnChunk; u += blockDim.x)
+            sa[u] = (k0 + u < kend) ? ah[k0 + u] * kLog2e : kNegInf;
+        for (int q = threadIdx.x; q < kLnSpan; q += blockDim.x) {
+            const int d = dbase + q;
+            sr[q] = (d >= 0 && d < T) ? rh[d] * kLog2e : kNegInf;
         }
-    }
+        __syncthreads();
+        // row i = i0 + lane, k = k0 + u: d - dbase = lane + (kLnChunk - 1) - u
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        float m2 = __shfl_xor_sync(0xffffffffu, m, off);
-        float s2 = __shfl_xor_sync(0xffffffffu, s, off);
-        lse2_merge(m, s, m2, s2);
+        for (int g = 0; g < kLnChunk / kLnWarps; g += 8) {
+            const int u0 = warp * (kLnChunk / kLnWarps) + g;
+            float x[8];
+            float mx = kNegInf;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                x[e] = sa[u0 + e] + sr[lane + (kLnChunk - 1) - (u0 + e)];
+                mx = fmaxf(mx, x[e]);
+            }
+            if (mx > m) {
+                s *= exp2f(m - mx);
+                m = mx;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s += exp2f(x[e] - m);
+        }
+        __syncthreads();
     }
-    if (lane == 0) logz[(size_t)h * T + i] = (m == kNegInf) ? kNegInf : (m + log2f(s)) * kLn2;
+    pm[warp][lane] = m;
+    ps[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0) {
+        float M = kLnFloor;
+#pragma unroll
+        for (int w = 0; w < kLnWarps; ++w) M = fmaxf(M, pm[w][lane]);
+        float S = 0.f;
+#pragma unroll
+        for (int w = 0; w < kLnWarps; ++w) S += ps[w][lane] * exp2f(pm[w][lane] - M);
+        const int i = i0 + lane;
+        if (i < T) logz[(size_t)h * T + i] = (S > 0.f) ? (M + log2f(S)) * kLn2 : kNegInf;
+    }
 }
 
 // 8 threads per row, 16 bytes (8 bf16) of O and dO each.
@@ -80,71 +112,72 @@ __global__ void __launch_bounds__(256) dot_kernel(const __nv_bfloat16* __restric
     if (row < rows && part == 0) dvec[row] = acc;
 }
 
-__device__ float block_reduce(float v, bool is_max, float* red) {
+// Block-wide reduction of four values at once: max, min, max, min.
+__device__ float4 block_reduce_mmmm(float4 v, float4* red) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-        float o = __shfl_xor_sync(0xffffffffu, v, off);
-        v = is_max ? fmaxf(v, o) : fminf(v, o);
+        v.x = fmaxf(v.x, __shfl_xor_sync(0xffffffffu, v.x, off));
+        v.y = fminf(v.y, __shfl_xor_sync(0xffffffffu, v.y, off));
+        v.z = fmaxf(v.z, __shfl_xor_sync(0xffffffffu, v.z, off));
+        v.w = fminf(v.w, __shfl_xor_sync(0xffffffffu, v.w, off));
     }
     if (lane == 0) red[wid] = v;
     __syncthreads();
-    if (wid == 0) {
-        v = lane < (int)(blockDim.x >> 5) ? red[lane] : (is_max ? kNegInf : -kNegInf);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            float o = __shfl_xor_sync(0xffffffffu, v, off);
-            v = is_max ? fmaxf(v, o) : fminf(v, o);
-        }
-        if (lane == 0) red[32] = v;
+    v = red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+        const float4 o = red[w];
+        v.x = fmaxf(v.x, o.x);
+        v.y = fminf(v.y, o.y);
+        v.z = fmaxf(v.z, o.z);
+        v.w = fminf(v.w, o.w);
     }
-    __syncthreads();
-    v = red[32];
-    __syncthreads();
     return v;
 }
 
 // Factored form of a replaced head's pattern,
 //   P(i,j) = r_i * E[i-j] * c_j,  E[d] = exp(r[d] - R),  c_j = exp(a[j] - A),
 //   r_i = exp(A + R - log Z(i)),  A = max a, R = max r,
-// which is Eq. (3) rearranged (exp of a sum is the product of exps).  One CTA
-// per replaced head writes, for the tensor-core kernels:
+// which is Eq. (3) rearranged (exp of a sum is the product of exps).  A row of
+// blocks per replaced head (grid.y = head slot) writes, for the tensor-core
+// kernels:
 //   epair[x + 128] = {bf16 E[x], bf16 E[x-1]}  for x in [-128, Tp + 128)
 //   ef[x + 128]    = E[x] (fp32), same range;  E outside [0, T) is 0
 //   cpair[m]       = {bf16 c[2m], bf16 c[2m+1]}, cf[j] = c[j]; 0 for j >= T
 //   rsc[i]         = r_i (fp32; 0 where log Z(i) = -inf)
 //   flag[h]        = 1 when the factors leave fp32 range for terms that matter
 //                    (then the head runs the per-element exp path instead).
-__global__ void __launch_bounds__(1024) prep_replaced_kernel(const float* __restrict__ a,
-                                                             const float* __restrict__ r,
-                                                             const float* __restrict__ logz, HeadList hl,
-                                                             int T, int Tp, int Lp, uint32_t* __restrict__ epair,
-                                                             float* __restrict__ ef, uint32_t* __restrict__ cpair,
-                                                             float* __restrict__ cf, float* __restrict__ rsc,
-                                                             int* __restrict__ flag) {
-    __shared__ float red[33];
-    const int slot = blockIdx.x;
+__global__ void __launch_bounds__(256) prep_replaced_kernel(const float* __restrict__ a,
+                                                            const float* __restrict__ r,
+                                                            const float* __restrict__ logz, HeadList hl,
+                                                            int T, int Tp, int Lp, uint32_t* __restrict__ epair,
+                                                            float* __restrict__ ef, uint32_t* __restrict__ cpair,
+                                                            float* __restrict__ cf, float* __restrict__ rsc,
+                                                            int* __restrict__ flag) {
+    __shared__ float4 red[8];
+    const int slot = blockIdx.y;
     const int h = hl.heads[slot];
     const float* ah = a + (size_t)h * T;
     const float* rh = r + (size_t)h * T;
     const float* lz = logz + (size_t)h * T;
-    float amax = kNegInf, amin = -kNegInf, rmax = kNegInf, lzmin = -kNegInf;
+    // every block of the head reduces the whole head (a few KB from L2), then
+    // writes its own share of the outputs
+    float4 v = make_float4(kNegInf, -kNegInf, kNegInf, -kNegInf);  // max a, min a, max r, min log Z
     for (int k = threadIdx.x; k < T; k += blockDim.x) {
         const float av = ah[k], rv = rh[k], lv = lz[k];
-        amax = fmaxf(amax, av);
-        if (av != kNegInf) amin = fminf(amin, av);
-        rmax = fmaxf(rmax, rv);
-        if (lv != kNegInf) lzmin = fminf(lzmin, lv);
+        v.x = fmaxf(v.x, av);
+        if (av != kNegInf) v.y = fminf(v.y, av);
+        v.z = fmaxf(v.z, rv);
+        if (lv != kNegInf) v.w = fminf(v.w, lv);
     }
-    amax = block_reduce(amax, true, red);
-    amin = block_reduce(amin, false, red);
-    rmax = block_reduce(rmax, true, red);
-    lzmin = block_reduce(lzmin, false, red);
-    const float A = (amax == kNegInf) ? 0.f : amax;
-    const float R = (rmax == kNegInf) ? 0.f : rmax;
+    v = block_reduce_mmmm(v, red);
+    const float amin = v.y, lzmin = v.w;
+    const float A = (v.x == kNegInf) ? 0.f : v.x;
+    const float R = (v.z == kNegInf) ? 0.f : v.z;
+    const int g0 = blockIdx.x * blockDim.x + threadIdx.x, gs = gridDim.x * blockDim.x;
     uint32_t* ep = epair + (size_t)slot * Lp;
     float* efs = ef + (size_t)slot * Lp;
-    for (int x = (int)threadIdx.x - 128; x < Tp + 128; x += blockDim.x) {
+    for (int x = g0 - 128; x < Tp + 128; x += gs) {
         const float e0 = (x >= 0 && x < T) ? expf(rh[x] - R) : 0.f;
         const float e1 = (x - 1 >= 0 && x - 1 < T) ? expf(rh[x - 1] - R) : 0.f;
         __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
@@ -153,7 +186,7 @@ __global__ void __launch_bounds__(1024) prep_replaced_kernel(const float* __rest
     }
     uint32_t* cp = cpair + (size_t)slot * (Tp / 2);
     float* cfs = cf + (size_t)slot * Tp;
-    for (int m = threadIdx.x; m < Tp / 2; m += blockDim.x) {
+    for (int m = g0; m < Tp / 2; m += gs) {
         const int j = 2 * m;
         const float c0 = j < T ? expf(ah[j] - A) : 0.f;
         const float c1 = j + 1 < T ? expf(ah[j + 1] - A) : 0.f;
@@ -163,11 +196,11 @@ __global__ void __launch_bounds__(1024) prep_replaced_kernel(const float* __rest
         cfs[j + 1] = c1;
     }
     float* rs = rsc + (size_t)slot * Tp;
-    for (int i = threadIdx.x; i < Tp; i += blockDim.x) {
+    for (int i = g0; i < Tp; i += gs) {
         const float lv = i < T ? lz[i] : kNegInf;
         rs[i] = (lv == kNegInf) ? 0.f : expf(A + R - lv);
     }
-    if (threadIdx.x == 0) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
         // forward: r_i = exp(A + R - log Z(i)) and backward: 1 / c_j = exp(A - a_j)
         // must stay well inside fp32 for every term of size > ~1e-15
         const bool ok = (lzmin == -kNegInf || A + R - lzmin <= 80.f) && (amin == -kNegInf || A - amin <= 80.f);
@@ -181,7 +214,9 @@ cudaError_t launch_prep_replaced(const float* a, const float* r, const float* lo
                                  const ReplacedWs& w, cudaStream_t stream) {
     if (hl.n == 0 || T == 0) return cudaSuccess;
     launch_begin(KID_PREP_REPLACED, stream);
-    prep_replaced_kernel<<<hl.n, 1024, 0, stream>>>(a, r, logz, hl, T, w.Tp, w.Lp, w.epair, w.ef, w.cpair, w.cf,
+    // enough 256-thread blocks per head for about 4 output entries per thread
+    const int nb = std::max(1, std::min(16, (w.Lp + 1023) / 1024));
+    prep_replaced_kernel<<<dim3(nb, hl.n), 256, 0, stream>>>(a, r, logz, hl, T, w.Tp, w.Lp, w.epair, w.ef, w.cpair, w.cf,
                                                     w.rsc, w.flag);
     launch_end(KID_PREP_REPLACED, stream);
     return cudaGetLastError();
@@ -190,9 +225,9 @@ cudaError_t launch_prep_replaced(const float* a, const float* r, const float* lo
 cudaError_t launch_lognorm(const float* a, const float* r, const HeadList& hl, int T,
                            float* logz, cudaStream_t stream) {
     if (hl.n == 0 || T == 0) return cudaSuccess;
-    dim3 grid((T + 7) / 8, hl.n);
+    dim3 grid((T + kLnRows - 1) / kLnRows, hl.n);
     launch_begin(KID_LOGNORM, stream);
-    lognorm_kernel<<<grid, 256, 0, stream>>>(a, r, hl, T, logz);
+    lognorm_kernel<<<grid, kLnWarps * 32, 0, stream>>>(a, r, hl, T, logz);
     launch_end(KID_LOGNORM, stream);
     return cudaGetLastError();
 }

@@ -128,6 +128,30 @@ def test_lognorm_entry_point_and_explicit_logz():
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("T", [1, 31, 32, 257, 545, 4101])
+def test_lognorm_tiles_and_special_values(T):
+    """log Z over ragged row tiles and several k chunks, with -inf terms
+    (a masked key, a forbidden distance) and offsets of +-50."""
+    gen = torch.Generator().manual_seed(T)
+    a = torch.randn(3, T, generator=gen) * 4
+    r = torch.randn(3, T, generator=gen) * 4
+    a[1] += 50.0
+    r[2] -= 50.0
+    a[0, ::7] = float("-inf")
+    r[0, 1::5] = float("-inf")
+    if T > 3:
+        a[2, :3] = float("-inf")  # rows 0..2 of head 2 have no term: log Z = -inf
+        r[2, 0] = float("-inf")
+    mask = torch.ones(3, dtype=torch.bool)
+    lz = saf.replaced_lognorm(a.cuda(), r.cuda(), mask).cpu().double().numpy()
+    ref = oracle.lognorm(a, r)
+    fin = np.isfinite(ref)
+    assert (np.isfinite(lz) == fin).all()
+    assert (lz[~fin] == -np.inf).all()
+    err = np.abs(lz[fin] - ref[fin])
+    assert err.max() < 1e-4 * max(1.0, np.abs(ref[fin]).max())
+
+
 def test_repeatable():
     w = I.custom(1, 3, 700, [1])
     x = I.make_inputs(w, 2)
