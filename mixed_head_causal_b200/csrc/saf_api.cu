@@ -180,11 +180,11 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
     }
     const ReplacedWs rw = replaced_ws(ws, L, T);
     if (hl.n > 0 && launch_prep_replaced(a, r, lz, hl, T, rw, s) != cudaSuccess) return SAF_ERR_CUDA;
-    float* lse2p = reinterpret_cast<float*>(ws + L.lse2p);
+    float* nlse2p = reinterpret_cast<float*>(ws + L.nlse2p);
     float* dvecp = reinterpret_cast<float*>(ws + L.dvecp);
     float* dqacc = reinterpret_cast<float*>(ws + L.dqacc);
-    if (launch_bwd_pre(ob, dob, lse, B * H, T, lse2p, dvecp, dqacc, s) != cudaSuccess) return SAF_ERR_CUDA;
-    cudaError_t e = launch_bwd_tc(qb, kb, vb, dob, lse2p, dvecp, dqacc, hl, rw, B, H, T, dk, dv, grad_dtype,
+    if (launch_bwd_pre(ob, dob, lse, B * H, T, nlse2p, dvecp, dqacc, s) != cudaSuccess) return SAF_ERR_CUDA;
+    cudaError_t e = launch_bwd_tc(qb, kb, vb, dob, nlse2p, dvecp, dqacc, hl, rw, B, H, T, dk, dv, grad_dtype,
                                   reinterpret_cast<unsigned int*>(ws), s);
     if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return SAF_ERR_CUDA;

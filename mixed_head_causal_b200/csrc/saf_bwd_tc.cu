@@ -51,13 +51,13 @@ constexpr uint32_t SM_DS = SM_DO + NQS * TILE;  // 32 KB: dS^T as two 64-query a
 // dQ staging, 32 KB: two [128][32] fp32 boxes (columns 0..31 and 32..63)
 // with the 128-byte swizzle of the reduce map
 constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;
-constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;     // NQS x 512 B: lse2 (ordinary) / r (replaced)
+constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;     // NQS x 512 B: -lse2 (ordinary) / r (replaced)
 constexpr uint32_t SM_VEC2 = SM_VEC1 + 512 * NQS;  // NQS x 512 B: D
 constexpr uint32_t SM_BAR = SM_VEC2 + 512 * NQS;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 
 struct BwdTcParams {
-    const float* lse2p;
+    const float* nlse2p;
     const float* dvecp;
     ReplacedWs w;
     void* dk;
@@ -86,19 +86,23 @@ __device__ __forceinline__ uint32_t packed_kcol(int k) { return k < 4 ? 8 * k : 
 
 // P^T for queries [32c, 32c + 32) of key row jl: exp2(S^T * scale - lse2),
 // packed as 16 bf16 pairs over TMEM columns packed_col(c) of the S^T region.
-// MASK: zero where the query precedes the key on the diagonal tile, or where
-// the key lies past T.
+// nlse2 holds -lse2 per query (read as pairs); the scale-and-shift runs on
+// paired fp32 FMAs.  MASK: zero where the query precedes the key on the
+// diagonal tile, or where the key lies past T.
 template <bool MASK>
-__device__ __forceinline__ void p_chunk(uint32_t tS, int c, const float* lse2, float scale, int jl, bool diag,
+__device__ __forceinline__ void p_chunk(uint32_t tS, int c, const float* nlse2, float scale, int jl, bool diag,
                                         bool key_ok, uint32_t (&pw)[16]) {
     uint32_t v[32];
     tmem_ld32(tS + 32 * c, v);
     tmem_wait_ld();
+    const uint64_t sc2 = f32x2(scale, scale);
+    const uint64_t* nl = reinterpret_cast<const uint64_t*>(nlse2 + 32 * c);
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
         const int ql = 32 * c + e;
-        float p0 = ex2(fmaf(__uint_as_float(v[e]), scale, -lse2[ql]));
-        float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, -lse2[ql + 1]));
+        const float2 x =
+            split_f32x2(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nl[e / 2]));
+        float p0 = ex2(x.x), p1 = ex2(x.y);
         if (MASK) {
             if (!key_ok || (diag && ql < jl)) p0 = 0.f;
             if (!key_ok || (diag && ql + 1 < jl)) p1 = 0.f;
@@ -210,7 +214,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     mbar_expect_tx(bq, 2 * TILE + 1024);
                     tma_load_3d(sb + SM_Q + s * TILE, &tmQ, bq, 0, I * BM, bh);
                     tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, bh);
-                    bulk_load(sb + SM_VEC1 + 512 * s, p.lse2p + (size_t)bh * p.Tp + I * BM, 512, bq);
+                    bulk_load(sb + SM_VEC1 + 512 * s, p.nlse2p + (size_t)bh * p.Tp + I * BM, 512, bq);
                     bulk_load(sb + SM_VEC2 + 512 * s, p.dvecp + (size_t)bh * p.Tp + I * BM, 512, bq);
                 } else {
                     mbar_expect_tx(bq, TILE + 512);
@@ -362,12 +366,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     uint32_t v[32], dsw[16];
                     tmem_ld32(tDP + 32 * c, v);
                     tmem_wait_ld();
+                    const uint64_t* d2 = reinterpret_cast<const uint64_t*>(v2 + 32 * c);
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const int ql = 32 * c + e;
+                        // (dP - D) paired, times P (bf16, widened), one rounding
                         const float2 pf = unpack_bf16x2(pw[cc][e / 2]);
-                        dsw[e / 2] = pack_bf16x2(pf.x * (__uint_as_float(v[e]) - v2[ql]),
-                                                 pf.y * (__uint_as_float(v[e + 1]) - v2[ql + 1]));
+                        const uint64_t g = sub_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), d2[e / 2]);
+                        const float2 ds = split_f32x2(mul_f32x2(f32x2(pf.x, pf.y), g));
+                        dsw[e / 2] = pack_bf16x2(ds.x, ds.y);
                     }
                     tmem_st16(tDP + packed_col(c), dsw);
                     // queries [64 half, 64 half + 64) form the MN atom `half`
@@ -499,12 +505,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
 }
 
-// rows of [BH, Tp]: lse2 = lse*log2(e) (+inf past T), D = rowsum(dO o O) (0
+// rows of [BH, Tp]: -lse2 = -lse*log2(e) (-inf past T), D = rowsum(dO o O) (0
 // past T); zero the dQ accumulator rows.  8 threads per row.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       const float* __restrict__ lse, int T, int Tp, int64_t rows,
-                                                      float* __restrict__ lse2p, float* __restrict__ dvecp,
+                                                      float* __restrict__ nlse2p, float* __restrict__ dvecp,
                                                       float* __restrict__ dqacc) {
     const int64_t r = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);
     const int part = threadIdx.x & 7;
@@ -532,7 +538,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
     acc += __shfl_xor_sync(0xffffffffu, acc, 4);
     if (part == 0) {
         dvecp[r] = i < T ? acc : 0.f;
-        lse2p[r] = i < T ? lse[bh * T + i] * kLog2e : -kNegInf;
+        nlse2p[r] = i < T ? -lse[bh * T + i] * kLog2e : kNegInf;
     }
 }
 
@@ -580,12 +586,12 @@ bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out) {
 }
 
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int BH, int T,
-                           float* lse2p, float* dvecp, float* dqacc, cudaStream_t stream) {
+                           float* nlse2p, float* dvecp, float* dqacc, cudaStream_t stream) {
     const int Tp = round_up128(T);
     const int64_t rows = (int64_t)BH * Tp;
     if (rows == 0) return cudaSuccess;
     launch_begin(KID_BWD_PRE, stream);
-    bwd_pre_kernel<<<(unsigned)((rows + 31) / 32), 256, 0, stream>>>(o, dout, lse, T, Tp, rows, lse2p, dvecp, dqacc);
+    bwd_pre_kernel<<<(unsigned)((rows + 31) / 32), 256, 0, stream>>>(o, dout, lse, T, Tp, rows, nlse2p, dvecp, dqacc);
     launch_end(KID_BWD_PRE, stream);
     return cudaGetLastError();
 }
@@ -602,7 +608,7 @@ cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int gr
 }
 
 cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                          const __nv_bfloat16* dout, const float* lse2p, const float* dvecp, float* dqacc,
+                          const __nv_bfloat16* dout, const float* nlse2p, const float* dvecp, float* dqacc,
                           const HeadList& hl, const ReplacedWs& w, int B, int H, int T, void* dk, void* dv,
                           int grad_fp32, unsigned int* err, cudaStream_t stream) {
     const int BH = B * H;
@@ -611,7 +617,7 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
         !make_tmap_bhtd(dout, BH, T, &mdo) || !make_tmap_bhtd_f32(dqacc, BH, T, &mdq))
         return cudaErrorNotSupported;
     BwdTcParams p;
-    p.lse2p = lse2p;
+    p.nlse2p = nlse2p;
     p.dvecp = dvecp;
     p.w = w;
     p.dk = dk;

@@ -51,7 +51,7 @@ struct WsLayout {
     size_t logz;     // [H, T] fp32 (used when the caller passes logz = NULL)
     size_t dvec;     // [B, H, T] fp32 row terms rowsum(dO o O) (backward only)
     size_t epair, ef, cpair, cf, rsc, flag;  // factored replaced-head arrays (H slots)
-    size_t lse2p;    // [B*H, Tp] fp32 lse * log2(e), +inf past T   (backward)
+    size_t nlse2p;    // [B*H, Tp] fp32 -lse * log2(e), -inf past T  (backward)
     size_t dvecp;    // [B*H, Tp] fp32 rowsum(dO o O), 0 past T      (backward)
     size_t dqacc;    // [B*H, T, 64] fp32 dQ accumulator              (backward)
     size_t total;
@@ -74,7 +74,7 @@ inline WsLayout ws_layout(int B, int H, int T, int is_bwd) {
     L.flag = off; off = align256(off + 4 * (size_t)H);
     if (is_bwd) {
         const size_t BH = (size_t)B * H;
-        L.lse2p = off; off = align256(off + 4 * BH * Tp);
+        L.nlse2p = off; off = align256(off + 4 * BH * Tp);
         L.dvecp = off; off = align256(off + 4 * BH * Tp);
         L.dqacc = off; off = align256(off + 4 * BH * (size_t)T * kHeadDim);
     }
@@ -127,10 +127,10 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
 // Backward preprocessing for the tensor-core backward: padded lse*log2(e) and
 // rowsum(dO o O), and a zeroed dQ accumulator.
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int BH, int T,
-                           float* lse2p, float* dvecp, float* dqacc, cudaStream_t stream);
+                           float* nlse2p, float* dvecp, float* dqacc, cudaStream_t stream);
 // Tensor-core backward (dK, dV written; dQ reduced into dqacc).
 cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                          const __nv_bfloat16* dout, const float* lse2p, const float* dvecp, float* dqacc,
+                          const __nv_bfloat16* dout, const float* nlse2p, const float* dvecp, float* dqacc,
                           const HeadList& hl, const ReplacedWs& w, int B, int H, int T, void* dk, void* dv,
                           int grad_fp32, unsigned int* err, cudaStream_t stream);
 // dq = dqacc / sqrt(d_h) in the requested dtype.

@@ -73,37 +73,45 @@ __device__ __forceinline__ void load_s_row(uint32_t tS, uint32_t (&v)[128]) {
 }
 
 // Row max of one 128-key block of raw scores.  MASK: the diagonal block,
-// where keys past the row (or past T) do not count.
+// where keys past the row (or past T) do not count.  Three-input max, four
+// independent chains.
 template <bool MASK>
 __device__ __forceinline__ float row_max(const uint32_t (&v)[128], int kbase, int i, int T) {
     float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
-    for (int e = 0; e < 128; ++e) {
-        float s = __uint_as_float(v[e]);
-        if (MASK && (kbase + e > i || kbase + e >= T)) s = kNegInf;
-        mx[e & 3] = fmaxf(mx[e & 3], s);
+    for (int e = 0; e < 128; e += 2) {
+        float s0 = __uint_as_float(v[e]), s1 = __uint_as_float(v[e + 1]);
+        if (MASK) {
+            if (kbase + e > i || kbase + e >= T) s0 = kNegInf;
+            if (kbase + e + 1 > i || kbase + e + 1 >= T) s1 = kNegInf;
+        }
+        mx[(e >> 1) & 3] = max3(mx[(e >> 1) & 3], s0, s1);
     }
     return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
 // P = exp2(s * scale - m) for the 128 keys of the block as 64 bf16 pairs;
-// returns the sum of the (unrounded) probabilities.
+// returns the sum of the (unrounded) probabilities.  The scale-and-shift and
+// the running sums use the paired fp32 instructions (same rounding as the
+// scalar ones).
 template <bool MASK>
 __device__ __forceinline__ float exp_row(const uint32_t (&v)[128], int kbase, int i, int T, float scale, float m,
                                          uint32_t (&pw)[64]) {
-    float l[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint64_t sc2 = f32x2(scale, scale), nm2 = f32x2(-m, -m);
+    uint64_t l2[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int e = 0; e < 128; e += 2) {
-        float p0 = ex2(fmaf(__uint_as_float(v[e]), scale, -m));
-        float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, -m));
+        const float2 x = split_f32x2(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nm2));
+        float p0 = ex2(x.x), p1 = ex2(x.y);
         if (MASK) {
             if (kbase + e > i || kbase + e >= T) p0 = 0.f;
             if (kbase + e + 1 > i || kbase + e + 1 >= T) p1 = 0.f;
         }
-        l[(e >> 1) & 3] += p0 + p1;
+        l2[(e >> 1) & 3] = add_f32x2(l2[(e >> 1) & 3], f32x2(p0, p1));
         pw[e >> 1] = pack_bf16x2(p0, p1);
     }
-    return (l[0] + l[1]) + (l[2] + l[3]);
+    const float2 a = split_f32x2(add_f32x2(add_f32x2(l2[0], l2[1]), add_f32x2(l2[2], l2[3])));
+    return a.x + a.y;
 }
 
 // W(i, j) = E[i-j] c_j for 64 keys (q0 = 0 or 8 selects the half): bf16 pair
