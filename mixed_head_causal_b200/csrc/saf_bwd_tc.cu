@@ -64,7 +64,7 @@ struct BwdTcParams {
     void* dv;
     unsigned int* err;
     int16_t slot_of_head[kMaxHeads];
-    int H, T, Tp, nqb, grad_fp32;
+    int H, BH, T, Tp, nqb, grad_fp32;
     float scale, scale_log2;
 };
 
@@ -139,22 +139,21 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_qe = bar_qf + 8 * NQS;   // [NQS]
     const uint32_t bar_s = bar_qe + 8 * NQS;
     const uint32_t bar_dp = bar_s + 8;
-    const uint32_t bar_p = bar_dp + 8;     // 128 arrivals
-    const uint32_t bar_ds = bar_p + 8;     // 128 arrivals
-    const uint32_t bar_dsc = bar_ds + 8;   // tile's MMAs done with P/W/dS
-    const uint32_t bar_dqf = bar_dsc + 8;  // [2]
+    const uint32_t bar_p = bar_dp + 8;     // 256 arrivals
+    const uint32_t bar_ds = bar_p + 8;     // 256 arrivals
+    const uint32_t bar_dqf = bar_ds + 8;   // [2]
     const uint32_t bar_dqe = bar_dqf + 16; // [2] 128 arrivals
     const uint32_t bar_acc = bar_dqe + 16;
     const uint32_t bar_wb = bar_acc + 8;   // [2] replaced head: W buffer b consumed
     const uint32_t bar_pb = bar_wb + 16;   // [2] replaced head: W buffer b written (256 arrivals)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 248);
-    static_assert(8 + 16 * NQS + 120 <= 248, "barrier area");
+    static_assert(8 + 16 * NQS + 104 <= 248, "barrier area");
 
     const int T = p.T;
-    // head-major order: the key blocks of one (b, h) run together and share
-    // its Q/dO tiles and dQ accumulator rows in L2; longest walks first
-    const int bh = (int)(blockIdx.x / (unsigned)p.nqb);
-    const int J = (int)(blockIdx.x % (unsigned)p.nqb);
+    // grouped, longest-first order (key block J walks nqb - J query blocks);
+    // a group's Q/dO tiles and dQ accumulator rows stay in L2
+    int bh, J;
+    grouped_order(blockIdx.x, p.BH, p.nqb, bh, J);
     const int h = bh % p.H;
     const int slot = p.slot_of_head[h];
     const bool rep = slot >= 0;
@@ -177,7 +176,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(bar_dp, 1);
         mbar_init(bar_p, 256);
         mbar_init(bar_ds, 256);
-        mbar_init(bar_dsc, 1);
         mbar_init(bar_wb, 1);
         mbar_init(bar_wb + 8, 1);
         mbar_init(bar_pb, 256);
@@ -307,7 +305,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     for (int k = 0; k < 8; ++k) mma_ts(tmem + C_DV, tmem + wcol + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
                     mma_commit(bar_wb + 8 * (t & 1));
                 }
-                mma_commit(bar_dsc);
                 mma_commit(bar_qe + 8 * s);
             }
             if (ok) mma_commit(bar_acc);
@@ -628,6 +625,7 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     for (int hh = 0; hh < H; ++hh)
         if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
     p.H = H;
+    p.BH = BH;
     p.T = T;
     p.Tp = round_up128(T);
     p.nqb = (T + BM - 1) / BM;

@@ -43,6 +43,21 @@ struct ReplacedWs {
 
 __host__ __device__ inline int round_up128(int x) { return (x + 127) & ~127; }
 
+// CTA order of the tensor-core kernels.  A CTA does one block-row of one
+// (batch, head) slice; its work shrinks with its causal rank (rank 0 = the
+// longest).  Slices are taken kHeadGroup at a time, so the tiles they share
+// stay in L2, and inside a group the CTAs run longest first across all its
+// slices, so the last CTAs to start are the shortest and the tail is small.
+constexpr int kHeadGroup = 16;
+__device__ __forceinline__ void grouped_order(unsigned b, int BH, int nblk, int& bh, int& rank) {
+    const unsigned per_group = (unsigned)kHeadGroup * (unsigned)nblk;
+    const int g = (int)(b / per_group);
+    const int r = (int)(b - (unsigned)g * per_group);
+    const int heads = min(kHeadGroup, BH - g * kHeadGroup);
+    rank = r / heads;
+    bh = g * kHeadGroup + (r - rank * heads);
+}
+
 // ---------------------------------------------------------------- workspace
 // Offsets of the scratch regions inside the caller's workspace.  Every region
 // starts on a 256-byte boundary.

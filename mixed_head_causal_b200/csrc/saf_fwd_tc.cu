@@ -56,7 +56,7 @@ struct FwdTcParams {
     ReplacedWs w;
     unsigned int* err;
     int16_t slot_of_head[kMaxHeads];
-    int H, T, nqb;
+    int H, BH, T, nqb;
     float scale_log2;
 };
 
@@ -152,10 +152,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 192);
 
     const int T = p.T;
-    // head-major order: the query blocks of one (b, h) run together and share
-    // its K/V tiles in L2; within a head, longest rows first
-    const int bh = (int)(blockIdx.x / (unsigned)p.nqb);
-    const int I = p.nqb - 1 - (int)(blockIdx.x % (unsigned)p.nqb);
+    // grouped, longest-first order (query block I visits I + 1 key blocks)
+    int bh, rank;
+    grouped_order(blockIdx.x, p.BH, p.nqb, bh, rank);
+    const int I = p.nqb - 1 - rank;
     const int h = bh % p.H;
     const int slot = p.slot_of_head[h];
     const bool rep = slot >= 0;
@@ -454,6 +454,7 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     for (int hh = 0; hh < H; ++hh)
         if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
     p.H = H;
+    p.BH = BH;
     p.T = T;
     p.nqb = (T + BM - 1) / BM;
     p.scale_log2 = kLog2e / 8.0f;
