@@ -9,6 +9,7 @@
 #include <algorithm>
 
 #include "saf_common.cuh"
+#include "tc_util.cuh"
 
 namespace saf {
 namespace {
@@ -16,13 +17,14 @@ namespace {
 
 // Tiling of the log-normaliser: a block owns 32 consecutive rows i (one per
 // lane) of one replaced head and walks k in chunks of kLnChunk staged in
-// shared memory; its 8 warps split each chunk 8 ways.  In a warp every lane
+// shared memory; its 8 warps split each chunk 8 ways.  Blocks start with the
+// last rows (the longest sums).  In a warp every lane
 // reads the same a[k] (a broadcast) and consecutive r[i-k] (no bank
 // conflicts).  Each lane keeps a log2-domain (max, sum) pair updated once per
 // 8 terms; the 8 per-warp partials of a row are merged at the end.
 constexpr int kLnRows = 32;
 constexpr int kLnWarps = 8;
-constexpr int kLnChunk = 256;
+constexpr int kLnChunk = 1024;
 constexpr int kLnSpan = kLnChunk + kLnRows;  // distinct d = i - k in one chunk
 constexpr float kLnFloor = -3.402823466e38f;  // finite "no term yet" maximum
 
@@ -34,7 +36,7 @@ __global__ void __launch_bounds__(kLnWarps * 32) lognorm_kernel(const float* __r
     __shared__ float sr[kLnSpan];
     __shared__ float pm[kLnWarps][32], ps[kLnWarps][32];
     const int h = hl.heads[blockIdx.y];
-    const int i0 = blockIdx.x * kLnRows;
+    const int i0 = (gridDim.x - 1 - blockIdx.x) * kLnRows;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* ah = a + (size_t)h * T;
     const float* rh = r + (size_t)h * T;
@@ -63,11 +65,11 @@ __global__ void __launch_bounds__(kLnWarps * 32) lognorm_kernel(const float* __r
                 mx = fmaxf(mx, x[e]);
             }
             if (mx > m) {
-                s *= exp2f(m - mx);
+                s *= tc::ex2(m - mx);
                 m = mx;
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s += exp2f(x[e] - m);
+            for (int e = 0; e < 8; ++e) s += tc::ex2(x[e] - m);
         }
         __syncthreads();
     }
@@ -147,14 +149,14 @@ __device__ float4 block_reduce_mmmm(float4 v, float4* red) {
 //   rsc[i]         = r_i (fp32; 0 where log Z(i) = -inf)
 //   flag[h]        = 1 when the factors leave fp32 range for terms that matter
 //                    (then the head runs the per-element exp path instead).
-__global__ void __launch_bounds__(256) prep_replaced_kernel(const float* __restrict__ a,
+__global__ void __launch_bounds__(1024) prep_replaced_kernel(const float* __restrict__ a,
                                                             const float* __restrict__ r,
                                                             const float* __restrict__ logz, HeadList hl,
                                                             int T, int Tp, int Lp, uint32_t* __restrict__ epair,
                                                             float* __restrict__ ef, uint32_t* __restrict__ cpair,
                                                             float* __restrict__ cf, float* __restrict__ rsc,
                                                             int* __restrict__ flag) {
-    __shared__ float4 red[8];
+    __shared__ float4 red[32];
     const int slot = blockIdx.y;
     const int h = hl.heads[slot];
     const float* ah = a + (size_t)h * T;
@@ -214,9 +216,9 @@ cudaError_t launch_prep_replaced(const float* a, const float* r, const float* lo
                                  const ReplacedWs& w, cudaStream_t stream) {
     if (hl.n == 0 || T == 0) return cudaSuccess;
     launch_begin(KID_PREP_REPLACED, stream);
-    // enough 256-thread blocks per head for about 4 output entries per thread
-    const int nb = std::max(1, std::min(16, (w.Lp + 1023) / 1024));
-    prep_replaced_kernel<<<dim3(nb, hl.n), 256, 0, stream>>>(a, r, logz, hl, T, w.Tp, w.Lp, w.epair, w.ef, w.cpair, w.cf,
+    // enough 1024-thread blocks per head for about 2 output entries per thread
+    const int nb = std::max(1, std::min(16, (w.Lp + 2047) / 2048));
+    prep_replaced_kernel<<<dim3(nb, hl.n), 1024, 0, stream>>>(a, r, logz, hl, T, w.Tp, w.Lp, w.epair, w.ef, w.cpair, w.cf,
                                                     w.rsc, w.flag);
     launch_end(KID_PREP_REPLACED, stream);
     return cudaGetLastError();
