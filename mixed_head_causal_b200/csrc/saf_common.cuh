@@ -116,6 +116,13 @@ struct WsHeader {
     unsigned int where;       // which wait (kernel-specific code)
     unsigned int counters[62];
 };
+// Work-queue counters of the persistent kernels, as word indices into the
+// header: the next unclaimed item and the number of CTAs that have finished
+// (the last one resets both to zero for the next launch).
+constexpr int kCtrFwdNext = 2, kCtrFwdDone = 3, kCtrBwdNext = 4, kCtrBwdDone = 5;
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
 
 // ---------------------------------------------------------------- accounting
 // Kernel ids of the launch accounting (names in saf_profile.cu).

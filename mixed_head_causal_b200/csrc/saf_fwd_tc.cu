@@ -24,6 +24,8 @@
 //   O_i = sum_j exp(a[j] + r[i-j] - log Z(i)) V_j.
 // Causal tile skipping: key blocks past the diagonal are never visited; the
 // diagonal block is masked (ordinary) or zero by construction (E[d<0] = 0).
+#include <algorithm>
+
 #include "saf_common.cuh"
 #include "tc_util.cuh"
 
@@ -34,7 +36,7 @@ using namespace tc;
 
 constexpr int BM = 128;          // query rows per CTA
 constexpr int BN = 128;          // keys per block
-constexpr int NSK = 3;           // K ring stages
+constexpr int NSK = 2;           // K ring stages
 constexpr int NSV = 2;           // V ring stages
 constexpr int NTHREADS = 192;
 constexpr uint32_t TILE_BYTES = 128 * 64 * 2;  // one 128 x 64 bf16 tile
@@ -44,7 +46,7 @@ constexpr long long kWaitLimit = 1ll << 31;                 // cycles
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr uint32_t SM_Q = 0;
-constexpr uint32_t SM_K = SM_Q + TILE_BYTES;
+constexpr uint32_t SM_K = SM_Q + 2 * TILE_BYTES;  // Q: two buffers (this item, next item)
 constexpr uint32_t SM_V = SM_K + NSK * TILE_BYTES;
 constexpr uint32_t SM_BAR = SM_V + NSV * TILE_BYTES;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
@@ -138,8 +140,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
-    const uint32_t bar_q = sbase + SM_BAR;
-    const uint32_t bar_kf = bar_q + 8;            // [NSK] K stage full
+    const uint32_t bar_itf = sbase + SM_BAR;      // [2] work item slot full
+    const uint32_t bar_ite = bar_itf + 16;        // [2] work item slot read (5 arrivals)
+    const uint32_t bar_qf = bar_ite + 16;         // [2] Q buffer full
+    const uint32_t bar_qe = bar_qf + 16;          // [2] Q buffer free (last S MMA of its item done)
+    const uint32_t bar_kf = bar_qe + 16;          // [NSK] K stage full
     const uint32_t bar_ke = bar_kf + 8 * NSK;     // [NSK] K stage free (S MMA done)
     const uint32_t bar_vf = bar_ke + 8 * NSK;     // [NSV] V stage full
     const uint32_t bar_ve = bar_vf + 8 * NSV;     // [NSV] V stage free (P.V MMA done)
@@ -149,22 +154,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_o = bar_p + 8;             // P.V done (ordinary head)
     const uint32_t bar_ob = bar_o + 8;            // [2] P.V of W buffer b done (replaced head)
     const uint32_t bar_pb = bar_ob + 16;          // [2] W buffer b written (replaced head, 128 arrivals)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 192);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 232);
+    int* item_slot = reinterpret_cast<int*>(smem + SM_BAR + 240);  // [2]
+    static_assert(16 * 4 + 16 * NSK + 16 * NSV + 32 + 32 <= 232, "barrier area");
 
     const int T = p.T;
-    // grouped, longest-first order (query block I visits I + 1 key blocks)
-    int bh, rank;
-    grouped_order(blockIdx.x, p.BH, p.nqb, bh, rank);
-    const int I = p.nqb - 1 - rank;
-    const int h = bh % p.H;
-    const int slot = p.slot_of_head[h];
-    const bool rep = slot >= 0;
-    if (rep && p.w.flag[h] != 0) return;  // handled by the per-element exp path
-    const int nkb = I + 1;
+    const int total = p.BH * p.nqb;  // work items: one query block of one (b, h) slice
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_q, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_itf + 8 * b, 1);
+            mbar_init(bar_ite + 8 * b, 5);
+            mbar_init(bar_qf + 8 * b, 1);
+            mbar_init(bar_qe + 8 * b, 1);
+            mbar_init(bar_ob + 8 * b, 1);
+            mbar_init(bar_pb + 8 * b, 128);
+        }
         for (int s = 0; s < NSK; ++s) {
             mbar_init(bar_kf + 8 * s, 1);
             mbar_init(bar_ke + 8 * s, 1);
@@ -177,10 +183,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(bar_sf, 128);
         mbar_init(bar_p, 128);
         mbar_init(bar_o, 1);
-        mbar_init(bar_ob, 1);
-        mbar_init(bar_ob + 8, 1);
-        mbar_init(bar_pb, 128);
-        mbar_init(bar_pb + 8, 128);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -192,204 +194,302 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    // Work item n of this CTA (-1: none left), published by the producer
+    // through a 2-slot ring; every consumer warp acknowledges it.
+    auto take_item = [&](int n, int& item) -> bool {
+        if (!mbar_wait(bar_itf + 8 * (n & 1), (n >> 1) & 1, kWaitLimit)) return false;
+        item = *reinterpret_cast<volatile int*>(item_slot + (n & 1));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ite + 8 * (n & 1));
+        return true;
+    };
+    // (b, h) slice and query block of an item, grouped longest-first order
+    // (query block I visits I + 1 key blocks)
+    struct Item {
+        int bh, I, h, slot;
+        bool rep, skip;
+    };
+    auto decode = [&](int item) {
+        Item it;
+        int rank;
+        grouped_order((unsigned)item, p.BH, p.nqb, it.bh, rank);
+        it.I = p.nqb - 1 - rank;
+        it.h = it.bh % p.H;
+        it.slot = p.slot_of_head[it.h];
+        it.rep = it.slot >= 0;
+        it.skip = it.rep && p.w.flag[it.h] != 0;  // handled by the per-element exp path
+        return it;
+    };
+
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            if (!rep) {
-                prefetch_tmap(&tmQ);
-                prefetch_tmap(&tmK);
-            }
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            if (!rep) {
-                mbar_expect_tx(bar_q, TILE_BYTES);
-                tma_load_3d(sbase + SM_Q, &tmQ, bar_q, 0, I * BM, bh);
-            }
-            // K_j is consumed by S_j, which runs a block ahead of P.V_j: the
-            // K loads go one block ahead of the V loads
-            auto load_k = [&](int j) -> bool {
-                const int s = j % NSK, n = j / NSK;
-                if (!mbar_wait(bar_ke + 8 * s, (n & 1) ^ 1, kWaitLimit)) return false;
-                mbar_expect_tx(bar_kf + 8 * s, TILE_BYTES);
-                tma_load_3d(sbase + SM_K + s * TILE_BYTES, &tmK, bar_kf + 8 * s, 0, j * BN, bh);
-                return true;
-            };
-            bool ok = rep || load_k(0);
-            for (int j = 0; ok && j < nkb; ++j) {
-                if (!rep && j + 1 < nkb && !load_k(j + 1)) { ok = false; break; }
-                const int s = j % NSV, n = j / NSV;
-                if (!mbar_wait(bar_ve + 8 * s, (n & 1) ^ 1, kWaitLimit)) { ok = false; break; }
-                mbar_expect_tx(bar_vf + 8 * s, TILE_BYTES);
-                tma_load_3d(sbase + SM_V + s * TILE_BYTES, &tmV, bar_vf + 8 * s, 0, j * BN, bh);
+            int gk = 0, gv = 0, nq = 0;  // K blocks, V blocks, ordinary items so far
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
+                const int w = (int)atomicAdd(p.err + kCtrFwdNext, 1u);
+                const int item = w < total ? w : -1;
+                if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                *reinterpret_cast<volatile int*>(item_slot + (n & 1)) = item;
+                mbar_arrive(bar_itf + 8 * (n & 1));
+                if (item < 0) break;
+                const Item it = decode(item);
+                if (it.skip) continue;
+                const int nkb = it.I + 1;
+                if (!it.rep) {
+                    const int b = nq & 1;
+                    if (!mbar_wait(bar_qe + 8 * b, ((nq >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                    mbar_expect_tx(bar_qf + 8 * b, TILE_BYTES);
+                    tma_load_3d(sbase + SM_Q + b * TILE_BYTES, &tmQ, bar_qf + 8 * b, 0, it.I * BM, it.bh);
+                    ++nq;
+                }
+                // K_j is consumed by S_j, which runs a block ahead of P.V_j: the
+                // K loads go one block ahead of the V loads
+                auto load_k = [&](int j) -> bool {
+                    const int g = gk + j, s = g % NSK, u = g / NSK;
+                    if (!mbar_wait(bar_ke + 8 * s, (u & 1) ^ 1, kWaitLimit)) return false;
+                    mbar_expect_tx(bar_kf + 8 * s, TILE_BYTES);
+                    tma_load_3d(sbase + SM_K + s * TILE_BYTES, &tmK, bar_kf + 8 * s, 0, j * BN, it.bh);
+                    return true;
+                };
+                if (!it.rep && !load_k(0)) { ok = false; break; }
+                for (int j = 0; j < nkb; ++j) {
+                    if (!it.rep && j + 1 < nkb && !load_k(j + 1)) { ok = false; break; }
+                    const int g = gv + j, s = g % NSV, u = g / NSV;
+                    if (!mbar_wait(bar_ve + 8 * s, (u & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                    mbar_expect_tx(bar_vf + 8 * s, TILE_BYTES);
+                    tma_load_3d(sbase + SM_V + s * TILE_BYTES, &tmV, bar_vf + 8 * s, 0, j * BN, it.bh);
+                }
+                if (!it.rep) gk += nkb;
+                gv += nkb;
             }
             if (!ok) report(p.err, 0x101);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
-            const uint32_t idO = idesc_bf16(128, 64, 0, 1);   // P (TMEM) x V (MN-major)
-            const uint64_t dq = sw128_desc(sbase + SM_Q);
-            // S_j = Q K_j^T into the S columns; frees K stage j when done
-            auto issue_s = [&](int j) -> bool {
-                const int s = j % NSK, n = j / NSK;
-                if (!mbar_wait(bar_kf + 8 * s, n & 1, kWaitLimit)) return false;
-                tc_fence_after();
-                const uint64_t dk = sw128_desc(sbase + SM_K + s * TILE_BYTES);
+        const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
+        const uint32_t idO = idesc_bf16(128, 64, 0, 1);   // P (TMEM) x V (MN-major)
+        int gk = 0, gv = 0, go = 0, gr = 0, nq = 0;  // K, V, ordinary, replaced blocks; ordinary items
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            int item;
+            ok = __all_sync(0xffffffffu, take_item(n, item));
+            if (!ok) { if (lane == 0) report(p.err, 0x205); break; }
+            if (item < 0) break;
+            const Item it = decode(item);
+            if (it.skip) continue;
+            const int nkb = it.I + 1;
+            if (lane == 0) {
+                const int b = nq & 1;
+                const uint64_t dq = sw128_desc(sbase + SM_Q + b * TILE_BYTES);
+                // S_j = Q K_j^T into the S columns; frees K stage j when done,
+                // and the Q buffer after the item's last block
+                auto issue_s = [&](int j) -> bool {
+                    const int g = gk + j, s = g % NSK, u = g / NSK;
+                    if (!mbar_wait(bar_kf + 8 * s, u & 1, kWaitLimit)) return false;
+                    tc_fence_after();
+                    const uint64_t dk = sw128_desc(sbase + SM_K + s * TILE_BYTES);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
-                    mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
-                mma_commit(bar_s);
-                mma_commit(bar_ke + 8 * s);
-                return true;
-            };
-            bool ok = true;
-            if (!rep) ok = mbar_wait(bar_q, 0, kWaitLimit) && issue_s(0);
-            if (!ok) report(p.err, 0x201);
-            for (int j = 0; ok && j < nkb; ++j) {
-                if (!rep && j + 1 < nkb) {
-                    // S_{j+1} once the rows have copied S_j out of TMEM
-                    if (!mbar_wait(bar_sf, j & 1, kWaitLimit) || !issue_s(j + 1)) { report(p.err, 0x202); break; }
-                }
-                const int s = j % NSV, n = j / NSV;
-                if (!mbar_wait(bar_vf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x203); break; }
-                if (!(rep ? mbar_wait(bar_pb + 8 * (j & 1), (j >> 1) & 1, kWaitLimit)
-                          : mbar_wait(bar_p, j & 1, kWaitLimit))) {
-                    report(p.err, 0x204);
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t dv = sw128_desc(sbase + SM_V + s * TILE_BYTES);
-                // a replaced head's W alternates between two buffers in the S
-                // columns (unused there), so building W_{j+1} overlaps this MMA
-                const uint32_t acol = rep ? 64 * (j & 1) : TP_COL;
+                    for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
+                        mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
+                    mma_commit(bar_s);
+                    mma_commit(bar_ke + 8 * s);
+                    if (j == nkb - 1) mma_commit(bar_qe + 8 * b);
+                    return true;
+                };
+                if (!it.rep) ok = mbar_wait(bar_qf + 8 * b, (nq >> 1) & 1, kWaitLimit) && issue_s(0);
+                if (!ok) report(p.err, 0x201);
+                for (int j = 0; ok && j < nkb; ++j) {
+                    if (!it.rep && j + 1 < nkb) {
+                        // S_{j+1} once the rows have copied S_j out of TMEM
+                        if (!mbar_wait(bar_sf, (go + j) & 1, kWaitLimit) || !issue_s(j + 1)) {
+                            report(p.err, 0x202);
+                            ok = false;
+                            break;
+                        }
+                    }
+                    const int g = gv + j, s = g % NSV, u = g / NSV;
+                    if (!mbar_wait(bar_vf + 8 * s, u & 1, kWaitLimit)) { report(p.err, 0x203); ok = false; break; }
+                    const int wb = (gr + j) & 1;
+                    if (!(it.rep ? mbar_wait(bar_pb + 8 * wb, ((gr + j) >> 1) & 1, kWaitLimit)
+                                 : mbar_wait(bar_p, (go + j) & 1, kWaitLimit))) {
+                        report(p.err, 0x204);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t dv = sw128_desc(sbase + SM_V + s * TILE_BYTES);
+                    // a replaced head's W alternates between two buffers in the S
+                    // columns (unused there), so building W_{j+1} overlaps this MMA
+                    const uint32_t acol = it.rep ? 64 * wb : TP_COL;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
-                    mma_ts(tmem + TO_COL, tmem + acol + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
-                mma_commit(rep ? bar_ob + 8 * (j & 1) : bar_o);
-                mma_commit(bar_ve + 8 * s);
+                    for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
+                        mma_ts(tmem + TO_COL, tmem + acol + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(it.rep ? bar_ob + 8 * wb : bar_o);
+                    mma_commit(bar_ve + 8 * s);
+                }
             }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (it.rep) {
+                gr += nkb;
+            } else {
+                gk += nkb;
+                go += nkb;
+                ++nq;
+            }
+            gv += nkb;
         }
     } else {
         // ------------------------------------------------ row threads
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // TMEM lane = query row within the block
-        const int i = I * BM + row;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lane_off + TS_COL;
         const uint32_t tO = tmem + lane_off + TO_COL;
         const uint32_t tP = tmem + lane_off + TP_COL;
-        float m = kNegInf, l = 0.f;
+        int go = 0, gr = 0;  // ordinary and replaced blocks so far
         bool ok = true;
-        for (int j = 0; j < nkb; ++j) {
-            if (!rep) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, kWaitLimit));
-                if (!ok) { report(p.err, 0x301); break; }
-                tc_fence_after();
-                uint32_t v[128];
-                load_s_row(tS, v);
-                tc_fence_before();
-                mbar_arrive(bar_sf);  // the MMA warp may now overwrite S
-                const bool diag = (j == I);
-                const int kbase = j * BN;
-                // row max of the block (the scale is positive); every row of a
-                // visited block has a visible key, so mx is finite.  The running
-                // max m moves only when the block's max exceeds it by more than
-                // 8 (log2 units), so P stays below 2^8 and O is rarely rescaled.
-                const float mx =
-                    (diag ? row_max<true>(v, kbase, i, T) : row_max<false>(v, kbase, i, T)) * p.scale_log2;
-                float f = 1.f;
-                if (m == kNegInf) {
-                    m = mx;
-                } else if (mx > m + 8.f) {
-                    f = ex2(m - mx);
-                    l *= f;
-                    m = mx;
-                }
-                uint32_t pw[64];  // P as bf16 pairs
-                l += diag ? exp_row<true>(v, kbase, i, T, p.scale_log2, m, pw)
-                          : exp_row<false>(v, kbase, i, T, p.scale_log2, m, pw);
-                // P_j replaces P_{j-1} in TMEM once P.V_{j-1} has read it; the
-                // O rows are rescaled (by the whole warp, when any row needs
-                // it) once that P.V has landed in O
-                if (j > 0) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (j - 1) & 1, kWaitLimit));
-                    if (!ok) { report(p.err, 0x302); break; }
+        for (int n = 0; ok; ++n) {
+            int item;
+            ok = __all_sync(0xffffffffu, take_item(n, item));
+            if (!ok) { report(p.err, 0x305); break; }
+            if (item < 0) break;
+            int I, slot;
+            bool rep;
+            {
+                const Item it = decode(item);
+                if (it.skip) continue;
+                I = it.I;
+                slot = it.slot;
+                rep = it.rep;
+            }
+            const int nkb = I + 1;
+            const int i = I * BM + row;
+            float m = kNegInf, l = 0.f;
+            for (int j = 0; j < nkb; ++j) {
+                if (!rep) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s, (go + j) & 1, kWaitLimit));
+                    if (!ok) { report(p.err, 0x301); break; }
                     tc_fence_after();
+                    uint32_t v[128];
+                    load_s_row(tS, v);
+                    tc_fence_before();
+                    mbar_arrive(bar_sf);  // the MMA warp may now overwrite S
+                    const bool diag = (j == I);
+                    const int kbase = j * BN;
+                    // row max of the block (the scale is positive); every row of a
+                    // visited block has a visible key, so mx is finite.  The running
+                    // max m moves only when the block's max exceeds it by more than
+                    // 8 (log2 units), so P stays below 2^8 and O is rarely rescaled.
+                    const float mx =
+                        (diag ? row_max<true>(v, kbase, i, T) : row_max<false>(v, kbase, i, T)) * p.scale_log2;
+                    float f = 1.f;
+                    if (m == kNegInf) {
+                        m = mx;
+                    } else if (mx > m + 8.f) {
+                        f = ex2(m - mx);
+                        l *= f;
+                        m = mx;
+                    }
+                    uint32_t pw[64];  // P as bf16 pairs
+                    l += diag ? exp_row<true>(v, kbase, i, T, p.scale_log2, m, pw)
+                              : exp_row<false>(v, kbase, i, T, p.scale_log2, m, pw);
+                    // P_j replaces P_{j-1} in TMEM once P.V_{j-1} has read it (the
+                    // previous item's last P.V was waited for by its epilogue); the
+                    // O rows are rescaled (by the whole warp, when any row needs
+                    // it) once that P.V has landed in O
+                    if (j > 0) {
+                        ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (go + j - 1) & 1, kWaitLimit));
+                        if (!ok) { report(p.err, 0x302); break; }
+                        tc_fence_after();
+                    }
+                    if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t ov[32];
+                            tmem_ld32(tO + 32 * c, ov);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+                            tmem_st32(tO + 32 * c, ov);
+                        }
+                    }
+                    tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
+                    tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
+                } else {
+                    // W(i,j) = E[i-j] c_j, bf16 pairs, into buffer g & 1 (g counts
+                    // replaced blocks), last read by the P.V of block g - 2 (one
+                    // barrier per buffer, so neither runs two phases ahead)
+                    const int g = gr + j;
+                    if (g >= 2) {
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(bar_ob + 8 * (g & 1), ((g >> 1) & 1) ^ 1, kWaitLimit));
+                        if (!ok) { report(p.err, 0x303); break; }
+                    }
+                    tc_fence_after();
+                    uint32_t pw0[32], pw1[32];
+                    const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
+                    const uint4* cp =
+                        reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
+                    build_w_half(ep, cp, 0, pw0);
+                    build_w_half(ep, cp, 8, pw1);
+                    tmem_st32(tS + 64 * (g & 1), pw0);
+                    tmem_st32(tS + 64 * (g & 1) + 32, pw1);
                 }
-                if (__any_sync(0xffffffffu, f != 1.f)) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t ov[32];
-                        tmem_ld32(tO + 32 * c, ov);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-                        tmem_st32(tO + 32 * c, ov);
+                // hand P (or W) to the MMA warp
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(rep ? bar_pb + 8 * ((gr + j) & 1) : bar_p);
+            }
+            // epilogue (TMEM reads by whole warps; rows past T are not stored)
+            if (ok) {
+                const int gl = (rep ? gr : go) + nkb - 1;  // the last P.V (MMAs complete in order)
+                ok = __all_sync(0xffffffffu, rep ? mbar_wait(bar_ob + 8 * (gl & 1), (gl >> 1) & 1, kWaitLimit)
+                                                 : mbar_wait(bar_o, gl & 1, kWaitLimit));
+                if (!ok) report(p.err, 0x304);
+            }
+            tc_fence_after();
+            const Item it = decode(item);
+            const int bh = it.bh;
+            if (ok) {
+                float scale = 0.f, lse_v = kNegInf;
+                if (i < T) {
+                    if (!rep) {
+                        scale = l > 0.f ? 1.f / l : 0.f;
+                        lse_v = (m == kNegInf || l <= 0.f) ? kNegInf : (m + log2f(l)) * kLn2;
+                    } else {
+                        scale = p.w.rsc[(size_t)slot * p.w.Tp + i];
+                        lse_v = p.logz[(size_t)it.h * T + i];
                     }
                 }
-                tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
-                tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
-            } else {
-                // W(i,j) = E[i-j] c_j, bf16 pairs, into buffer j & 1, last read
-                // by the P.V of block j - 2 (one barrier per buffer, so neither
-                // can run two phases ahead of this wait)
-                if (j >= 2) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(bar_ob + 8 * (j & 1), ((j >> 1) & 1) ^ 1, kWaitLimit));
-                    if (!ok) { report(p.err, 0x303); break; }
-                }
-                tc_fence_after();
-                uint32_t pw0[32], pw1[32];
-                const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
-                const uint4* cp = reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
-                build_w_half(ep, cp, 0, pw0);
-                build_w_half(ep, cp, 8, pw1);
-                tmem_st32(tS + 64 * (j & 1), pw0);
-                tmem_st32(tS + 64 * (j & 1) + 32, pw1);
-            }
-            // hand P (or W) to the MMA warp
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(rep ? bar_pb + 8 * (j & 1) : bar_p);
-        }
-        // epilogue (TMEM reads by whole warps; rows past T are not stored)
-        if (ok) {
-            const int jl = nkb - 1;  // the last P.V (MMAs complete in order)
-            ok = __all_sync(0xffffffffu, rep ? mbar_wait(bar_ob + 8 * (jl & 1), (jl >> 1) & 1, kWaitLimit)
-                                             : mbar_wait(bar_o, jl & 1, kWaitLimit));
-            if (!ok) report(p.err, 0x304);
-        }
-        tc_fence_after();
-        if (ok) {
-            float scale = 0.f, lse_v = kNegInf;
-            if (i < T) {
-                if (!rep) {
-                    scale = l > 0.f ? 1.f / l : 0.f;
-                    lse_v = (m == kNegInf || l <= 0.f) ? kNegInf : (m + log2f(l)) * kLn2;
-                } else {
-                    scale = p.w.rsc[(size_t)slot * p.w.Tp + i];
-                    lse_v = p.logz[(size_t)h * T + i];
-                }
-            }
-            __nv_bfloat16* orow = p.o + ((size_t)bh * T + (i < T ? i : 0)) * kHeadDim;
+                __nv_bfloat16* orow = p.o + ((size_t)bh * T + (i < T ? i : 0)) * kHeadDim;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tO + 32 * c, v);
-                tmem_wait_ld();
-                uint32_t packed[16];
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tO + 32 * c, v);
+                    tmem_wait_ld();
+                    uint32_t packed[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    packed[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * scale, __uint_as_float(v[2 * e + 1]) * scale);
-                if (i < T) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+                    for (int e = 0; e < 16; ++e)
+                        packed[e] =
+                            pack_bf16x2(__uint_as_float(v[2 * e]) * scale, __uint_as_float(v[2 * e + 1]) * scale);
+                    if (i < T) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] =
+                                make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                    }
                 }
+                if (i < T) p.lse[(size_t)bh * T + i] = lse_v;
+            } else if (i < T) {
+                p.lse[(size_t)bh * T + i] = __int_as_float(0x7fc00000);  // NaN marks the failed rows
             }
-            if (i < T) p.lse[(size_t)bh * T + i] = lse_v;
-        } else if (i < T) {
-            p.lse[(size_t)bh * T + i] = __int_as_float(0x7fc00000);  // NaN marks the failed rows
+            if (rep) gr += nkb;
+            else go += nkb;
         }
     }
     tc_fence_before();
@@ -397,6 +497,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
+    }
+    // the last CTA to finish resets the work counters for the next launch
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.err + kCtrFwdDone, 1u) == gridDim.x - 1) {
+            atomicExch(p.err + kCtrFwdNext, 0u);
+            atomicExch(p.err + kCtrFwdDone, 0u);
+        }
     }
 }
 
@@ -420,6 +528,19 @@ EncodeTiledFn encode_fn() {
 }
 
 }  // namespace
+
+int sm_count() {
+    constexpr int kMaxDev = 64;
+    static int cached[kMaxDev] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
 
 // [BH, T, 64] bf16 viewed as a 3-D tensor (d, t, bh); 128 x 64 boxes with the
 // 128-byte swizzle; rows past T read as zeros.
@@ -461,8 +582,12 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     const int smem = SM_TOTAL + 1024;
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // persistent: two CTAs per SM pull work items from a counter in the
+    // workspace header
+    const int items = BH * p.nqb;
+    const int grid = std::min(items, 2 * sm_count());
     launch_begin(KID_FWD_TC, stream);
-    fwd_tc_kernel<<<dim3((unsigned)BH * p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, p);
+    fwd_tc_kernel<<<dim3((unsigned)grid), NTHREADS, smem, stream>>>(mq, mk, mv, p);
     launch_end(KID_FWD_TC, stream);
     return cudaGetLastError();
 }
