@@ -127,11 +127,10 @@ saf_status saf_mixed_attn_fwd(const void* q, const void* k, const void* v, void*
     if (force_mma_path()) return cuda_status(launch_fwd_mma(qb, kb, vb, ob, lse, a, r, lz, hl, B, H, T, s));
     const ReplacedWs rw = replaced_ws(ws, L, T);
     if (hl.n > 0 && launch_prep_replaced(a, r, lz, hl, T, rw, s) != cudaSuccess) return SAF_ERR_CUDA;
-    cudaError_t e = launch_fwd_tc(qb, kb, vb, ob, lse, lz, hl, rw, B, H, T, reinterpret_cast<unsigned int*>(ws), s);
+    cudaError_t e =
+        launch_fwd_tc(qb, kb, vb, ob, lse, a, r, lz, hl, rw, B, H, T, reinterpret_cast<unsigned int*>(ws), s);
     if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return SAF_ERR_CUDA;
-    // replaced heads whose factored form would leave fp32 range
-    if (hl.n > 0) return cuda_status(launch_fwd_mma(qb, kb, vb, ob, lse, a, r, lz, hl, B, H, T, s, rw.flag));
     return SAF_OK;
 }
 
@@ -184,15 +183,11 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
     float* dvecp = reinterpret_cast<float*>(ws + L.dvecp);
     float* dqacc = reinterpret_cast<float*>(ws + L.dqacc);
     if (launch_bwd_pre(ob, dob, lse, B * H, T, nlse2p, dvecp, dqacc, s) != cudaSuccess) return SAF_ERR_CUDA;
-    cudaError_t e = launch_bwd_tc(qb, kb, vb, dob, nlse2p, dvecp, dqacc, hl, rw, B, H, T, dk, dv, grad_dtype,
-                                  reinterpret_cast<unsigned int*>(ws), s);
+    cudaError_t e = launch_bwd_tc(qb, kb, vb, dob, nlse2p, dvecp, dqacc, a, r, lz, hl, rw, B, H, T, dk, dv,
+                                  grad_dtype, reinterpret_cast<unsigned int*>(ws), s);
     if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return SAF_ERR_CUDA;
     if (launch_dq_convert(dqacc, dq, (int64_t)B * H * T, grad_dtype, s) != cudaSuccess) return SAF_ERR_CUDA;
-    // replaced heads whose factored form would leave fp32 range
-    if (hl.n > 0)
-        return cuda_status(launch_bwd_mma(qb, kb, vb, dob, lse, dvecp, a, r, lz, hl, B, H, T, dq, dk, dv,
-                                          grad_dtype, s, rw.flag));
     return SAF_OK;
 }
 

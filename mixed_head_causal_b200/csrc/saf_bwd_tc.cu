@@ -24,6 +24,8 @@
 // fed to the tensor cores as a hi + lo bf16 pair (two TS MMAs) so that a
 // column with large weights over many rows (a sink) keeps its precision;
 // c_j is applied in the epilogue.  dK = 0 there, and dQ gets no contribution.
+// A replaced head whose factors would leave fp32 range (flag set by the prep
+// kernel) uses P^T itself, one exp per element, and no c_j.
 #include "saf_common.cuh"
 #include "tc_util.cuh"
 
@@ -59,6 +61,9 @@ constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 struct BwdTcParams {
     const float* nlse2p;
     const float* dvecp;
+    const float* a;  // [H, T] pattern vectors and log Z (read for flag-1 replaced heads only)
+    const float* r;
+    const float* logz;
     ReplacedWs w;
     void* dk;
     void* dv;
@@ -127,6 +132,39 @@ __device__ __forceinline__ void store_row(void* base, int grad_fp32, size_t row,
     }
 }
 
+// P^T(j, i) = exp(a[j] + r[i-j] - log Z(i)) of a replaced head straight from
+// Eq. (3) (aj = a[j], -inf past T); 0 before the key, past T, or where log Z
+// is -inf.
+__device__ __forceinline__ float direct_pt(const BwdTcParams& p, int h, int T, float aj, int j, int i) {
+    if (i < j || i >= T) return 0.f;
+    const float lz = __ldg(p.logz + (size_t)h * T + i);
+    if (lz == kNegInf) return 0.f;
+    return ex2((aj + __ldg(p.r + (size_t)h * T + (i - j)) - lz) * kLog2e);
+}
+
+// The direct P^T for query columns [64 half, 64 half + 64) of this thread's
+// key row, as hi + lo bf16 pairs into the W buffer at tW (kept out of line:
+// the path is rare).
+__device__ __noinline__ void direct_pt_half(const BwdTcParams& p, int h, int T, float aj, int j, int qbase, int half,
+                                            uint32_t tW) {
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * half + cc;
+        uint32_t hw[16], lw[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const float w0 = direct_pt(p, h, T, aj, j, qbase + 32 * c + e);
+            const float w1 = direct_pt(p, h, T, aj, j, qbase + 32 * c + e + 1);
+            const uint32_t hb = pack_bf16x2(w0, w1);
+            const float2 hf = unpack_bf16x2(hb);
+            hw[e / 2] = hb;
+            lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+        }
+        tmem_st16(tW + 16 * c, hw);
+        tmem_st16(tW + 64 + 16 * c, lw);
+    }
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -157,7 +195,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int h = bh % p.H;
     const int slot = p.slot_of_head[h];
     const bool rep = slot >= 0;
-    if (rep && p.w.flag[h] != 0) return;  // handled by the per-element exp path
+    // a replaced head whose factors would leave fp32 range takes P^T itself
+    // (one exp per element) in place of W^T, and its dV rows need no c_j
+    const bool direct = rep && p.w.flag[h] != 0;
     const int ntiles = p.nqb - J;
     const bool ragged_keys = (J + 1) * BN > T;  // the key block runs past T
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -227,7 +267,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // K-major x K-major, 128 x 128
             const uint32_t idTS = idesc_bf16(128, 64, 0, 1);   // TMEM A x MN-major B, 128 x 64
             const uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // MN-major A x MN-major B
-            const uint64_t dK = sw128_desc(sb + SM_K), dVd = sw128_desc(sb + SM_V);
+            // descriptors of the tiles: one base plus (byte offset / 16)
+            const uint64_t d0 = sw128_desc(sb);
+            const uint64_t dK = d0 + (SM_K >> 4), dVd = d0 + (SM_V >> 4);
             const uint64_t dDS = sw128_desc(sb + SM_DS, 16384);
             bool ok = rep || mbar_wait(bar_kv, 0, kWaitLimit);
             if (!ok) report(p.err, 0x1201);
@@ -236,14 +278,17 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             // dP^T of tile t+1 right after dQ_t, so the tensor cores work on the
             // next tile while the row threads finish this one.  The tensor pipe
             // executes one thread's MMAs in order, which orders those reuses.
-            auto issue_s = [&](int tt) {
-                const uint64_t dQn = sw128_desc(sb + SM_Q + (tt % NQS) * TILE);
+            // The issuing thread keeps its scalar work small (the pipe stalls
+            // while it computes): ring stages and their descriptors advance
+            // incrementally (a stage is TILE bytes = TILE / 16 descriptor units).
+            constexpr uint64_t kStage = TILE >> 4;
+            const uint64_t dQ0 = d0 + (SM_Q >> 4), dDO0 = d0 + (SM_DO >> 4);
+            auto issue_s = [&](uint64_t dQn) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQn + 2 * k, idSS, k > 0);
                 mma_commit(bar_s);
             };
-            auto issue_dp = [&](int tt) {
-                const uint64_t dDOn = sw128_desc(sb + SM_DO + (tt % NQS) * TILE);
+            auto issue_dp = [&](uint64_t dDOn) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOn + 2 * k, idSS, k > 0);
                 mma_commit(bar_dp);
@@ -251,43 +296,45 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (ok && !rep) {
                 if (!mbar_wait(bar_qf, 0, kWaitLimit)) { report(p.err, 0x1202); ok = false; }
                 tc_fence_after();
-                if (ok) { issue_s(0); issue_dp(0); }
+                if (ok) { issue_s(dQ0); issue_dp(dDO0); }
             }
-            int t = 0;
-            for (; ok && t < ntiles; ++t) {
-                const int s = t % NQS, n = t / NQS;
-                const uint64_t dQs = sw128_desc(sb + SM_Q + s * TILE), dDOs = sw128_desc(sb + SM_DO + s * TILE);
+            int s = 0, ph = 0;  // ring stage of tile t and its phase parity
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const bool wrap = (s + 1 == NQS);
+                const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;  // tile t + 1
+                const uint64_t dQs = dQ0 + (uint64_t)s * kStage, dDOs = dDO0 + (uint64_t)s * kStage;
+                const uint32_t acc = t > 0 ? 1u : 0u;
                 if (!rep) {
                     if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1203); ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DV, tmem + C_S + packed_kcol(k), dDOs + 128 * k, idTS,
-                               (t > 0 || k > 0) ? 1u : 0u);
+                        mma_ts(tmem + C_DV, tmem + C_S + packed_kcol(k), dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
                     const bool more = t + 1 < ntiles;
                     if (more) {
-                        if (!mbar_wait(bar_qf + 8 * ((t + 1) % NQS), ((t + 1) / NQS) & 1, kWaitLimit)) {
-                            report(p.err, 0x1207); ok = false; break;
-                        }
+                        if (!mbar_wait(bar_qf + 8 * s1, ph1, kWaitLimit)) { report(p.err, 0x1207); ok = false; break; }
                         tc_fence_after();
-                        issue_s(t + 1);
+                        issue_s(dQ0 + (uint64_t)s1 * kStage);
                     }
                     if (!mbar_wait(bar_ds, t & 1, kWaitLimit)) { report(p.err, 0x1204); ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DK, tmem + C_DP + packed_kcol(k), dQs + 128 * k, idTS,
-                               (t > 0 || k > 0) ? 1u : 0u);
-                    const int b = t & 1, nb = t >> 1;
-                    if (!mbar_wait(bar_dqe + 8 * b, (nb & 1) ^ 1, kWaitLimit)) { report(p.err, 0x1205); ok = false; break; }
+                        mma_ts(tmem + C_DK, tmem + C_DP + packed_kcol(k), dQs + 128 * k, idTS, k > 0 ? 1u : acc);
+                    const int b = t & 1;
+                    if (!mbar_wait(bar_dqe + 8 * b, ((t >> 1) & 1) ^ 1, kWaitLimit)) {
+                        report(p.err, 0x1205);
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t cdq = b ? C_DQ1 : C_DQ0;
 #pragma unroll
                     for (int k = 0; k < 8; ++k) mma_ss(tmem + cdq, dDS + 128 * k, dK + 128 * k, idDQ, k > 0);
                     mma_commit(bar_dqf + 8 * b);
-                    if (more) issue_dp(t + 1);
+                    if (more) issue_dp(dDO0 + (uint64_t)s1 * kStage);
                 } else {
-                    if (!mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit)) { report(p.err, 0x1202); ok = false; break; }
+                    if (!mbar_wait(bar_qf + 8 * s, ph, kWaitLimit)) { report(p.err, 0x1202); ok = false; break; }
                     tc_fence_after();
                     if (!mbar_wait(bar_pb + 8 * (t & 1), (t >> 1) & 1, kWaitLimit)) {
                         report(p.err, 0x1206);
@@ -300,12 +347,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const uint32_t wcol = C_S + 128 * (t & 1);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DV, tmem + wcol + 8 * k, dDOs + 128 * k, idTS, (t > 0 || k > 0) ? 1u : 0u);
+                        mma_ts(tmem + C_DV, tmem + wcol + 8 * k, dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
 #pragma unroll
                     for (int k = 0; k < 8; ++k) mma_ts(tmem + C_DV, tmem + wcol + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
                     mma_commit(bar_wb + 8 * (t & 1));
                 }
                 mma_commit(bar_qe + 8 * s);
+                s = s1;
+                ph = ph1;
             }
             if (ok) mma_commit(bar_acc);
         }
@@ -398,22 +447,27 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 tc_fence_after();
                 const float* ef = p.w.ef + (size_t)slot * p.w.Lp + 128 + (I - J) * BM - jl;
+                const float aj = (direct && j < T) ? p.a[(size_t)h * T + j] : kNegInf;
+                if (!direct) {
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * half + cc;
-                    uint32_t hw[16], lw[16];
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = 2 * half + cc;
+                        uint32_t hw[16], lw[16];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int ql = 32 * c + e;
-                        const float w0 = __ldg(ef + ql) * v1[ql];
-                        const float w1 = __ldg(ef + ql + 1) * v1[ql + 1];
-                        const uint32_t hb = pack_bf16x2(w0, w1);
-                        const float2 hf = unpack_bf16x2(hb);
-                        hw[e / 2] = hb;
-                        lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                        for (int e = 0; e < 32; e += 2) {
+                            const int ql = 32 * c + e;
+                            const float w0 = __ldg(ef + ql) * v1[ql];
+                            const float w1 = __ldg(ef + ql + 1) * v1[ql + 1];
+                            const uint32_t hb = pack_bf16x2(w0, w1);
+                            const float2 hf = unpack_bf16x2(hb);
+                            hw[e / 2] = hb;
+                            lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                        }
+                        tmem_st16(tW + 16 * c, hw);
+                        tmem_st16(tW + 64 + 16 * c, lw);
                     }
-                    tmem_st16(tW + 16 * c, hw);
-                    tmem_st16(tW + 64 + 16 * c, lw);
+                } else {
+                    direct_pt_half(p, h, T, aj, j, I * BM, half, tW);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -431,7 +485,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             // the dK row (times 1/sqrt(d); zero for a replaced head)
             float vals[64];
             float mul;
-            if (half == 0) mul = (rep && j < T) ? p.w.cf[(size_t)slot * p.w.Tp + j] : 1.f;
+            if (half == 0) mul = (rep && !direct && j < T) ? p.w.cf[(size_t)slot * p.w.Tp + j] : 1.f;
             else mul = rep ? 0.f : p.scale;
             const uint32_t col = half == 0 ? C_DV : C_DK;
 #pragma unroll
@@ -606,8 +660,9 @@ cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int gr
 
 cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           const __nv_bfloat16* dout, const float* nlse2p, const float* dvecp, float* dqacc,
-                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, void* dk, void* dv,
-                          int grad_fp32, unsigned int* err, cudaStream_t stream) {
+                          const float* a, const float* r, const float* logz, const HeadList& hl,
+                          const ReplacedWs& w, int B, int H, int T, void* dk, void* dv, int grad_fp32,
+                          unsigned int* err, cudaStream_t stream) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mdo, mdq;
     if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, BH, T, &mk) || !make_tmap_bhtd(v, BH, T, &mv) ||
@@ -616,6 +671,9 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     BwdTcParams p;
     p.nlse2p = nlse2p;
     p.dvecp = dvecp;
+    p.a = a;
+    p.r = r;
+    p.logz = logz;
     p.w = w;
     p.dk = dk;
     p.dv = dv;

@@ -140,21 +140,24 @@ cudaError_t launch_lognorm(const float* a, const float* r, const HeadList& hl, i
                            float* logz, cudaStream_t stream);
 cudaError_t launch_prep_replaced(const float* a, const float* r, const float* logz, const HeadList& hl, int T,
                                  const ReplacedWs& w, cudaStream_t stream);
-// Tensor-core forward of every ordinary head and every replaced head whose
-// factored form is usable (flag 0); returns cudaErrorNotSupported when the
-// tensor maps cannot be built.
+// Tensor-core forward of every head (replaced heads whose factored form would
+// leave fp32 range, flag 1, take per-element exps of a + r - log Z); returns
+// cudaErrorNotSupported when the tensor maps cannot be built.
 cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                          __nv_bfloat16* o, float* lse, const float* logz, const HeadList& hl,
-                          const ReplacedWs& w, int B, int H, int T, unsigned int* err, cudaStream_t stream);
+                          __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
+                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, unsigned int* err,
+                          cudaStream_t stream);
 // Backward preprocessing for the tensor-core backward: padded lse*log2(e) and
 // rowsum(dO o O), and a zeroed dQ accumulator.
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int BH, int T,
                            float* nlse2p, float* dvecp, float* dqacc, cudaStream_t stream);
-// Tensor-core backward (dK, dV written; dQ reduced into dqacc).
+// Tensor-core backward (dK, dV written; dQ reduced into dqacc); replaced
+// heads with flag 1 take per-element exps of a + r - log Z.
 cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           const __nv_bfloat16* dout, const float* nlse2p, const float* dvecp, float* dqacc,
-                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, void* dk, void* dv,
-                          int grad_fp32, unsigned int* err, cudaStream_t stream);
+                          const float* a, const float* r, const float* logz, const HeadList& hl,
+                          const ReplacedWs& w, int B, int H, int T, void* dk, void* dv, int grad_fp32,
+                          unsigned int* err, cudaStream_t stream);
 // dq = dqacc / sqrt(d_h) in the requested dtype.
 cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream);
 bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out);

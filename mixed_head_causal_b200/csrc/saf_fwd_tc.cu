@@ -22,6 +22,8 @@
 //   W(i,j) = E[i-j] c_j     (bf16 pairs multiplied in registers, no exp)
 // is written to TMEM and O += W V_j; the epilogue scales row i by r_i, giving
 //   O_i = sum_j exp(a[j] + r[i-j] - log Z(i)) V_j.
+// A replaced head whose factors would leave fp32 range (flag set by the prep
+// kernel) takes the pattern itself, one exp per element, in the same slot.
 // Causal tile skipping: key blocks past the diagonal are never visited; the
 // diagonal block is masked (ordinary) or zero by construction (E[d<0] = 0).
 #include <algorithm>
@@ -54,6 +56,8 @@ constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 struct FwdTcParams {
     __nv_bfloat16* o;
     float* lse;
+    const float* a;  // [H, T] pattern vectors (read for flag-1 replaced heads only)
+    const float* r;
     const float* logz;
     ReplacedWs w;
     unsigned int* err;
@@ -134,6 +138,32 @@ __device__ __forceinline__ void build_w_half(const uint32_t* ep, const uint4* cp
     }
 }
 
+// A replaced head whose factored form would leave fp32 range: row i of the
+// pattern for keys [k0, k0 + 128) straight from Eq. (3), one exp per element,
+// P = exp(a[k] + r[i-k] - log Z(i)) (0 past the row, past T, or where log Z is
+// -inf), as 64 bf16 pairs stored to the W buffer at tW; the epilogue then
+// needs no row scale.  Kept out of line: the path is rare.
+__device__ __noinline__ void direct_p_row(const float* ah, const float* rh, const float* logz, int h, int T, int i,
+                                          int k0, uint32_t tW) {
+    const float lz = i < T ? logz[(size_t)h * T + i] : kNegInf;
+    const bool row_ok = lz != kNegInf;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        uint32_t pw[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+            float pr[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int k = k0 + 64 * c + e + u;
+                pr[u] = (row_ok && k <= i && k < T) ? ex2((__ldg(ah + k) + __ldg(rh + (i - k)) - lz) * kLog2e) : 0.f;
+            }
+            pw[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+        }
+        tmem_st32(tW + 32 * c, pw);
+    }
+}
+
 __global__ void __launch_bounds__(NTHREADS, 2)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const FwdTcParams p) {
@@ -149,11 +179,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_vf = bar_ke + 8 * NSK;     // [NSV] V stage full
     const uint32_t bar_ve = bar_vf + 8 * NSV;     // [NSV] V stage free (P.V MMA done)
     const uint32_t bar_s = bar_ve + 8 * NSV;      // S ready
-    const uint32_t bar_sf = bar_s + 8;            // S copied out by the rows (128 arrivals)
-    const uint32_t bar_p = bar_sf + 8;            // P written (128 arrivals)
+    const uint32_t bar_sf = bar_s + 8;            // S copied out by the rows (4 warp arrivals)
+    const uint32_t bar_p = bar_sf + 8;            // P written (4 warp arrivals)
     const uint32_t bar_o = bar_p + 8;             // P.V done (ordinary head)
     const uint32_t bar_ob = bar_o + 8;            // [2] P.V of W buffer b done (replaced head)
-    const uint32_t bar_pb = bar_ob + 16;          // [2] W buffer b written (replaced head, 128 arrivals)
+    const uint32_t bar_pb = bar_ob + 16;          // [2] W buffer b written (replaced head, 4 warp arrivals)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 232);
     int* item_slot = reinterpret_cast<int*>(smem + SM_BAR + 240);  // [2]
     static_assert(16 * 4 + 16 * NSK + 16 * NSV + 32 + 32 <= 232, "barrier area");
@@ -169,7 +199,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_init(bar_qf + 8 * b, 1);
             mbar_init(bar_qe + 8 * b, 1);
             mbar_init(bar_ob + 8 * b, 1);
-            mbar_init(bar_pb + 8 * b, 128);
+            mbar_init(bar_pb + 8 * b, 4);
         }
         for (int s = 0; s < NSK; ++s) {
             mbar_init(bar_kf + 8 * s, 1);
@@ -180,8 +210,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_init(bar_ve + 8 * s, 1);
         }
         mbar_init(bar_s, 1);
-        mbar_init(bar_sf, 128);
-        mbar_init(bar_p, 128);
+        mbar_init(bar_sf, 4);
+        mbar_init(bar_p, 4);
         mbar_init(bar_o, 1);
         fence_mbar_init();
     }
@@ -207,7 +237,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // (query block I visits I + 1 key blocks)
     struct Item {
         int bh, I, h, slot;
-        bool rep, skip;
+        bool rep, direct;
     };
     auto decode = [&](int item) {
         Item it;
@@ -217,7 +247,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         it.h = it.bh % p.H;
         it.slot = p.slot_of_head[it.h];
         it.rep = it.slot >= 0;
-        it.skip = it.rep && p.w.flag[it.h] != 0;  // handled by the per-element exp path
+        it.direct = it.rep && p.w.flag[it.h] != 0;  // per-element exps instead of the factored form
         return it;
     };
 
@@ -237,7 +267,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mbar_arrive(bar_itf + 8 * (n & 1));
                 if (item < 0) break;
                 const Item it = decode(item);
-                if (it.skip) continue;
                 const int nkb = it.I + 1;
                 if (!it.rep) {
                     const int b = nq & 1;
@@ -272,6 +301,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // ------------------------------------------------ MMA issuer
         const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
         const uint32_t idO = idesc_bf16(128, 64, 0, 1);   // P (TMEM) x V (MN-major)
+        // descriptors advance by stage (TILE_BYTES = TILE_BYTES / 16 units):
+        // the issuing thread keeps its scalar work small, the pipe waits on it
+        constexpr uint64_t kStage = TILE_BYTES >> 4;
+        const uint64_t dQ0 = sw128_desc(sbase + SM_Q), dK0 = sw128_desc(sbase + SM_K);
+        const uint64_t dV0 = sw128_desc(sbase + SM_V);
         int gk = 0, gv = 0, go = 0, gr = 0, nq = 0;  // K, V, ordinary, replaced blocks; ordinary items
         bool ok = true;
         for (int n = 0; ok; ++n) {
@@ -280,18 +314,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (!ok) { if (lane == 0) report(p.err, 0x205); break; }
             if (item < 0) break;
             const Item it = decode(item);
-            if (it.skip) continue;
             const int nkb = it.I + 1;
             if (lane == 0) {
                 const int b = nq & 1;
-                const uint64_t dq = sw128_desc(sbase + SM_Q + b * TILE_BYTES);
+                const uint64_t dq = dQ0 + (uint64_t)b * kStage;
                 // S_j = Q K_j^T into the S columns; frees K stage j when done,
                 // and the Q buffer after the item's last block
                 auto issue_s = [&](int j) -> bool {
                     const int g = gk + j, s = g % NSK, u = g / NSK;
                     if (!mbar_wait(bar_kf + 8 * s, u & 1, kWaitLimit)) return false;
                     tc_fence_after();
-                    const uint64_t dk = sw128_desc(sbase + SM_K + s * TILE_BYTES);
+                    const uint64_t dk = dK0 + (uint64_t)s * kStage;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
                         mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
@@ -321,7 +354,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t dv = sw128_desc(sbase + SM_V + s * TILE_BYTES);
+                    const uint64_t dv = dV0 + (uint64_t)s * kStage;
                     // a replaced head's W alternates between two buffers in the S
                     // columns (unused there), so building W_{j+1} overlaps this MMA
                     const uint32_t acol = it.rep ? 64 * wb : TP_COL;
@@ -357,14 +390,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             ok = __all_sync(0xffffffffu, take_item(n, item));
             if (!ok) { report(p.err, 0x305); break; }
             if (item < 0) break;
-            int I, slot;
-            bool rep;
+            int I, slot, h;
+            bool rep, direct;
             {
                 const Item it = decode(item);
-                if (it.skip) continue;
                 I = it.I;
                 slot = it.slot;
+                h = it.h;
                 rep = it.rep;
+                direct = it.direct;
             }
             const int nkb = I + 1;
             const int i = I * BM + row;
@@ -377,7 +411,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     uint32_t v[128];
                     load_s_row(tS, v);
                     tc_fence_before();
-                    mbar_arrive(bar_sf);  // the MMA warp may now overwrite S
+                    mbar_arrive_warp(bar_sf);  // the MMA warp may now overwrite S
                     const bool diag = (j == I);
                     const int kbase = j * BN;
                     // row max of the block (the scale is positive); every row of a
@@ -430,19 +464,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         if (!ok) { report(p.err, 0x303); break; }
                     }
                     tc_fence_after();
-                    uint32_t pw0[32], pw1[32];
-                    const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
-                    const uint4* cp =
-                        reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
-                    build_w_half(ep, cp, 0, pw0);
-                    build_w_half(ep, cp, 8, pw1);
-                    tmem_st32(tS + 64 * (g & 1), pw0);
-                    tmem_st32(tS + 64 * (g & 1) + 32, pw1);
+                    if (!direct) {
+                        uint32_t pw0[32], pw1[32];
+                        const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
+                        const uint4* cp =
+                            reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
+                        build_w_half(ep, cp, 0, pw0);
+                        build_w_half(ep, cp, 8, pw1);
+                        tmem_st32(tS + 64 * (g & 1), pw0);
+                        tmem_st32(tS + 64 * (g & 1) + 32, pw1);
+                    } else {
+                        direct_p_row(p.a + (size_t)h * T, p.r + (size_t)h * T, p.logz, h, T, i, j * BN,
+                                     tS + 64 * (g & 1));
+                    }
                 }
                 // hand P (or W) to the MMA warp
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(rep ? bar_pb + 8 * ((gr + j) & 1) : bar_p);
+                mbar_arrive_warp(rep ? bar_pb + 8 * ((gr + j) & 1) : bar_p);
             }
             // epilogue (TMEM reads by whole warps; rows past T are not stored)
             if (ok) {
@@ -452,8 +491,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (!ok) report(p.err, 0x304);
             }
             tc_fence_after();
-            const Item it = decode(item);
-            const int bh = it.bh;
+            const int bh = decode(item).bh;
             if (ok) {
                 float scale = 0.f, lse_v = kNegInf;
                 if (i < T) {
@@ -461,8 +499,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         scale = l > 0.f ? 1.f / l : 0.f;
                         lse_v = (m == kNegInf || l <= 0.f) ? kNegInf : (m + log2f(l)) * kLn2;
                     } else {
-                        scale = p.w.rsc[(size_t)slot * p.w.Tp + i];
-                        lse_v = p.logz[(size_t)it.h * T + i];
+                        scale = direct ? 1.f : p.w.rsc[(size_t)slot * p.w.Tp + i];
+                        lse_v = p.logz[(size_t)h * T + i];
                     }
                 }
                 __nv_bfloat16* orow = p.o + ((size_t)bh * T + (i < T ? i : 0)) * kHeadDim;
@@ -558,8 +596,9 @@ bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out) {
 }
 
 cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                          __nv_bfloat16* o, float* lse, const float* logz, const HeadList& hl,
-                          const ReplacedWs& w, int B, int H, int T, unsigned int* err, cudaStream_t stream) {
+                          __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
+                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, unsigned int* err,
+                          cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     const int BH = B * H;
     if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, BH, T, &mk) || !make_tmap_bhtd(v, BH, T, &mv))
@@ -567,6 +606,8 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     FwdTcParams p;
     p.o = o;
     p.lse = lse;
+    p.a = a;
+    p.r = r;
     p.logz = logz;
     p.w = w;
     p.err = err;

@@ -16,24 +16,26 @@ namespace {
 
 
 // Tiling of the log-normaliser: a block owns 32 consecutive rows i (one per
-// lane) of one replaced head and walks k in chunks of kLnChunk staged in
-// shared memory; its 8 warps split each chunk 8 ways.  Blocks start with the
-// last rows (the longest sums).  In a warp every lane
-// reads the same a[k] (a broadcast) and consecutive r[i-k] (no bank
-// conflicts).  Each lane keeps a log2-domain (max, sum) pair updated once per
-// 8 terms; the 8 per-warp partials of a row are merged at the end.
+// lane) of one replaced head.  It stages a[0, kend) and r[0, kend) (kend = the
+// tile's last row + 1; chunks of kLnChunk for long heads) in shared memory in
+// log2 units, all loads in flight at once, and its 8 warps split the k range
+// 8 ways.  In a warp every lane reads the same a[k] (a broadcast) and
+// consecutive r[i-k] (no bank conflicts).  Each lane keeps a log2-domain
+// (max, sum) pair updated once per 8 terms; the 8 per-warp partials of a row
+// are merged at the end.  Blocks start with the last rows (the longest sums).
 constexpr int kLnRows = 32;
 constexpr int kLnWarps = 8;
-constexpr int kLnChunk = 1024;
-constexpr int kLnSpan = kLnChunk + kLnRows;  // distinct d = i - k in one chunk
+constexpr int kLnChunk = 4096;
 constexpr float kLnFloor = -3.402823466e38f;  // finite "no term yet" maximum
 
 __global__ void __launch_bounds__(kLnWarps * 32) lognorm_kernel(const float* __restrict__ a,
                                                                const float* __restrict__ r,
-                                                               HeadList hl, int T,
+                                                               HeadList hl, int T, int chunk,
                                                                float* __restrict__ logz) {
-    __shared__ float sa[kLnChunk];
-    __shared__ float sr[kLnSpan];
+    // dynamic shared memory of 2 * chunk + kLnRows floats, chunk = min(T, kLnChunk)
+    extern __shared__ float ln_smem[];
+    float* sa = ln_smem;          // [chunk]: a[k0 + u]
+    float* sr = ln_smem + chunk;  // [chunk + kLnRows]: r[dbase + q]
     __shared__ float pm[kLnWarps][32], ps[kLnWarps][32];
     const int h = hl.heads[blockIdx.y];
     const int i0 = (gridDim.x - 1 - blockIdx.x) * kLnRows;
@@ -42,26 +44,31 @@ __global__ void __launch_bounds__(kLnWarps * 32) lognorm_kernel(const float* __r
     const float* rh = r + (size_t)h * T;
     const int kend = min(i0 + kLnRows, T);  // every k a row of this tile can reach
     float m = kLnFloor, s = 0.f;
-    for (int k0 = 0; k0 < kend; k0 += kLnChunk) {
-        // sa[u] = a[k0 + u] and sr[q] = r[d] for d = i0 - k0 - (kLnChunk - 1) + q,
-        // both in log2 units; out-of-range entries are -inf (no term)
-        const int dbase = i0 - k0 - (kLnChunk - 1);
-        for (int u = threadIdx.x; u < kLnChunk; u += blockDim.x)
-            sa[u] = (k0 + u < kend) ? ah[k0 + u] * kLog2e : kNegInf;
-        for (int q = threadIdx.x; q < kLnSpan; q += blockDim.x) {
+    for (int k0 = 0; k0 < kend; k0 += chunk) {
+        const int n = min(chunk, kend - k0);  // k of this chunk: [k0, k0 + n)
+        // sa[u] = a[k0 + u] (u < n) and sr[q] = r[d], d = dbase + q, for the
+        // d = i - k this chunk can meet; out-of-range entries are -inf (no term)
+        const int dbase = i0 - k0 - (n - 1);
+        const int span = n + kLnRows - 1;
+#pragma unroll 4
+        for (int u = threadIdx.x; u < n; u += blockDim.x) sa[u] = ah[k0 + u] * kLog2e;
+#pragma unroll 4
+        for (int q = threadIdx.x; q < span; q += blockDim.x) {
             const int d = dbase + q;
             sr[q] = (d >= 0 && d < T) ? rh[d] * kLog2e : kNegInf;
         }
         __syncthreads();
-        // row i = i0 + lane, k = k0 + u: d - dbase = lane + (kLnChunk - 1) - u
-#pragma unroll
-        for (int g = 0; g < kLnChunk / kLnWarps; g += 8) {
-            const int u0 = warp * (kLnChunk / kLnWarps) + g;
+        // warp w takes k in [w * per, (w + 1) * per) of the chunk, 8 at a time;
+        // row i = i0 + lane, k = k0 + u: d - dbase = lane + (n - 1) - u
+        const int per = ((n + 8 * kLnWarps - 1) / (8 * kLnWarps)) * 8;
+        const int ub = warp * per, ue = min(n, ub + per);
+        for (int u0 = ub; u0 < ue; u0 += 8) {
             float x[8];
             float mx = kNegInf;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                x[e] = sa[u0 + e] + sr[lane + (kLnChunk - 1) - (u0 + e)];
+                const int u = u0 + e;
+                x[e] = u < ue ? sa[u] + sr[lane + (n - 1) - u] : kNegInf;
                 mx = fmaxf(mx, x[e]);
             }
             if (mx > m) {
@@ -216,8 +223,8 @@ cudaError_t launch_prep_replaced(const float* a, const float* r, const float* lo
                                  const ReplacedWs& w, cudaStream_t stream) {
     if (hl.n == 0 || T == 0) return cudaSuccess;
     launch_begin(KID_PREP_REPLACED, stream);
-    // enough 1024-thread blocks per head for about 2 output entries per thread
-    const int nb = std::max(1, std::min(16, (w.Lp + 2047) / 2048));
+    // enough 1024-thread blocks per head for about one output entry per thread
+    const int nb = std::max(1, std::min(32, (w.Lp + 1023) / 1024));
     prep_replaced_kernel<<<dim3(nb, hl.n), 1024, 0, stream>>>(a, r, logz, hl, T, w.Tp, w.Lp, w.epair, w.ef, w.cpair, w.cf,
                                                     w.rsc, w.flag);
     launch_end(KID_PREP_REPLACED, stream);
@@ -228,8 +235,14 @@ cudaError_t launch_lognorm(const float* a, const float* r, const HeadList& hl, i
                            float* logz, cudaStream_t stream) {
     if (hl.n == 0 || T == 0) return cudaSuccess;
     dim3 grid((T + kLnRows - 1) / kLnRows, hl.n);
+    const int chunk = std::min(T, kLnChunk);
+    const int smem = (int)sizeof(float) * (2 * chunk + kLnRows);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(lognorm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
     launch_begin(KID_LOGNORM, stream);
-    lognorm_kernel<<<grid, kLnWarps * 32, 0, stream>>>(a, r, hl, T, logz);
+    lognorm_kernel<<<grid, kLnWarps * 32, smem, stream>>>(a, r, hl, T, chunk, logz);
     launch_end(KID_LOGNORM, stream);
     return cudaGetLastError();
 }

@@ -198,3 +198,16 @@ def test_factored_range_guard_falls_back(path):
     w, x = _special(777, lambda T: torch.randn(T) * 40.0, lambda T: -0.05 * torch.arange(T, dtype=torch.float32))
     got = P.run_layer(w, x)
     P.check_slices(w, x, got, _all_slices(w))
+
+
+def test_guarded_and_factored_heads_in_one_call():
+    """Two batches, heads 0 and 2 replaced: head 0 with a far beyond fp32
+    range (per-element exps), head 2 ordinary-range (factored form), a ragged
+    T spanning several tiles; every slice against the oracle."""
+    w = I.custom(2, 4, 650, [0, 2])
+    x = I.make_inputs(w, 13)
+    gen = torch.Generator().manual_seed(13)
+    x["alpha"][0] = torch.randn(650, generator=gen) * 40.0
+    x["rho"][0] = -0.02 * torch.arange(650, dtype=torch.float32) + torch.randn(650, generator=gen) * 30.0
+    got = P.run_layer(w, x)
+    P.check_slices(w, x, got, _all_slices(w))
