@@ -39,7 +39,6 @@ struct BwdParams {
     void* dk;
     void* dv;
     HeadList hl;
-    const int* head_only_flag;  // non-null: only replaced heads with a nonzero flag
     int H, T, grad_fp32;
     float scale;       // 1/sqrt(d_h)
     float scale_log2;  // log2(e)/sqrt(d_h)
@@ -87,13 +86,8 @@ __global__ void __launch_bounds__(NT) dkdv_kernel(const BwdParams p) {
 
     const int T = p.T;
     const int kb = blockIdx.y;  // key block 0 has the most query blocks: run first
-    int bh = blockIdx.x;
-    int h = bh % p.H;
-    if (p.head_only_flag != nullptr) {  // grid.x enumerates (batch, replaced head)
-        h = p.hl.heads[blockIdx.x % p.hl.n];
-        bh = (blockIdx.x / p.hl.n) * p.H + h;
-        if (p.head_only_flag[h] == 0) return;
-    }
+    const int bh = blockIdx.x;
+    const int h = bh % p.H;
     const bool rep = p.hl.replaced[h] != 0;
     const size_t base = (size_t)bh * T * kHeadDim;
     const __nv_bfloat16* Qg = p.q + base;
@@ -283,13 +277,8 @@ __global__ void __launch_bounds__(NT) dq_kernel(const BwdParams p) {
     const int T = p.T;
     const int nqb = (T + BQ - 1) / BQ;
     const int qb = nqb - 1 - (int)blockIdx.y;
-    int bh = blockIdx.x;
-    int h = bh % p.H;
-    if (p.head_only_flag != nullptr) {
-        h = p.hl.heads[blockIdx.x % p.hl.n];
-        bh = (blockIdx.x / p.hl.n) * p.H + h;
-        if (p.head_only_flag[h] == 0) return;
-    }
+    const int bh = blockIdx.x;
+    const int h = bh % p.H;
     const bool rep = p.hl.replaced[h] != 0;
     const size_t base = (size_t)bh * T * kHeadDim;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -399,11 +388,10 @@ cudaError_t launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const float* lse, const float* dvec,
                            const float* a, const float* r, const float* logz,
                            const HeadList& hl, int B, int H, int T,
-                           void* dq, void* dk, void* dv, int grad_fp32, cudaStream_t stream,
-                           const int* head_only_flag) {
-    BwdParams p{q, k, v, dout, lse, dvec, a, r, logz, dq, dk, dv, hl, head_only_flag, H, T, grad_fp32,
+                           void* dq, void* dk, void* dv, int grad_fp32, cudaStream_t stream) {
+    BwdParams p{q, k, v, dout, lse, dvec, a, r, logz, dq, dk, dv, hl, H, T, grad_fp32,
                 0.125f, kLog2e * 0.125f};
-    const int gx = head_only_flag ? B * hl.n : B * H;
+    const int gx = B * H;
     if (gx == 0) return cudaSuccess;
     const int smem1 = 2 * BK * 128 + 4 * BQ * 128 + 4 * BQ * (int)sizeof(float);
     const int smem2 = 2 * BQ * 128 + 4 * BK * 128;

@@ -162,12 +162,12 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
 cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream);
 bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out);
 bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out);
-// head_only_flag != nullptr: run only replaced heads h with head_only_flag[h] != 0.
+// Warp-level (mma.sync) forward and backward of every head, the reference
+// path selected by SAF_FORCE_MMA.
 cudaError_t launch_fwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, __nv_bfloat16* o, float* lse,
                            const float* a, const float* r, const float* logz,
-                           const HeadList& hl, int B, int H, int T, cudaStream_t stream,
-                           const int* head_only_flag = nullptr);
+                           const HeadList& hl, int B, int H, int T, cudaStream_t stream);
 cudaError_t launch_bwd_dot(const __nv_bfloat16* o, const __nv_bfloat16* dout, float* dvec,
                            const HeadList& hl, int B, int H, int T, cudaStream_t stream);
 cudaError_t launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
@@ -175,7 +175,6 @@ cudaError_t launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const float* lse, const float* dvec,
                            const float* a, const float* r, const float* logz,
                            const HeadList& hl, int B, int H, int T,
-                           void* dq, void* dk, void* dv, int grad_fp32, cudaStream_t stream,
-                           const int* head_only_flag = nullptr);
+                           void* dq, void* dk, void* dv, int grad_fp32, cudaStream_t stream);
 
 }  // namespace saf

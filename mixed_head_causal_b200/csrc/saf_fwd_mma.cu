@@ -35,7 +35,6 @@ struct FwdParams {
     const float* r;
     const float* logz;
     HeadList hl;
-    const int* head_only_flag;  // non-null: only replaced heads with a nonzero flag
     int H, T;
     float scale_log2;  // log2(e) / sqrt(d_h)
 };
@@ -49,13 +48,8 @@ __global__ void __launch_bounds__(NT) fwd_mma_kernel(const FwdParams p) {
     const int T = p.T;
     const int nqb = (T + BM - 1) / BM;
     const int qb = nqb - 1 - (int)blockIdx.y;  // longest rows first
-    int bh = blockIdx.x;
-    int h = bh % p.H;
-    if (p.head_only_flag != nullptr) {  // grid.x enumerates (batch, replaced head)
-        h = p.hl.heads[blockIdx.x % p.hl.n];
-        bh = (blockIdx.x / p.hl.n) * p.H + h;
-        if (p.head_only_flag[h] == 0) return;
-    }
+    const int bh = blockIdx.x;
+    const int h = bh % p.H;
     const bool rep = p.hl.replaced[h] != 0;
     const size_t base = (size_t)bh * T * kHeadDim;
     const __nv_bfloat16* Qg = p.q + base;
@@ -255,13 +249,12 @@ __global__ void __launch_bounds__(NT) fwd_mma_kernel(const FwdParams p) {
 cudaError_t launch_fwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, __nv_bfloat16* o, float* lse,
                            const float* a, const float* r, const float* logz,
-                           const HeadList& hl, int B, int H, int T, cudaStream_t stream,
-                           const int* head_only_flag) {
-    FwdParams p{q, k, v, o, lse, a, r, logz, hl, head_only_flag, H, T, kLog2e / 8.0f};
+                           const HeadList& hl, int B, int H, int T, cudaStream_t stream) {
+    FwdParams p{q, k, v, o, lse, a, r, logz, hl, H, T, kLog2e / 8.0f};
     const int smem = BM * 128 + 4 * BN * 128;
     cudaError_t e = cudaFuncSetAttribute(fwd_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(head_only_flag ? B * hl.n : B * H, (T + BM - 1) / BM);
+    dim3 grid(B * H, (T + BM - 1) / BM);
     if (grid.x == 0) return cudaSuccess;
     launch_begin(KID_FWD_MMA, stream);
     fwd_mma_kernel<<<grid, NT, smem, stream>>>(p);
