@@ -38,6 +38,11 @@
  *              Device-side waits are bounded; one that gives up records an
  *              error word in the workspace, which saf_device_status reports
  *              as SAF_ERR_TIMEOUT.
+ *   Workspace  Its first 256 bytes hold the device error word and the work
+ *              counters of the persistent kernels; they must be zero before
+ *              the workspace is first used (e.g. one cudaMemset), and every
+ *              call leaves the counters zero again.  The rest needs no
+ *              clearing.
  *   Outputs    Always overwritten, never accumulated into.  Inputs and outputs
  *              must not alias.  Calls that share a workspace must not overlap
  *              on the GPU.
@@ -133,6 +138,37 @@ SAF_API saf_status saf_mixed_attn_bwd(const void *q, const void *k, const void *
                               void *stream);
 
 /*
+ * Shared K/V (grouped-query attention): the same layer with k and v holding
+ * H_kv heads ([B,H_kv,T,d_h]) shared by groups of H / H_kv consecutive query
+ * heads: query head h reads K/V head h / (H / H_kv).  H_kv must divide H
+ * (SAF_ERR_INVALID_ARG otherwise); H_kv == H is the plain layer.  Replaced
+ * heads read the V head of their group.  In the backward, dk and dv are
+ * [B,H_kv,T,d_h]: the gradient of a shared K/V head is the sum over the query
+ * heads of its group (computed per query head in fp32 in the workspace, then
+ * summed).  The pages measure their attention speed-ups on this variant
+ * ("When Can Attention Heads Be Statically Defined?", Table 26); its math is
+ * the plain layer with K and V repeated over each group.  Workspace sizes come
+ * from saf_workspace_size_gqa.  Not available on the SAF_FORCE_MMA path
+ * (SAF_ERR_UNSUPPORTED).
+ */
+SAF_API size_t saf_workspace_size_gqa(int B, int H, int H_kv, int T, int d_h, int is_bwd);
+SAF_API saf_status saf_mixed_attn_fwd_gqa(const void *q, const void *k, const void *v,
+                                          void *o, float *lse,
+                                          const float *a, const float *r, const float *logz,
+                                          const uint8_t *replaced_mask,
+                                          int B, int H, int H_kv, int T, int d_h,
+                                          void *workspace, size_t workspace_bytes,
+                                          void *stream);
+SAF_API saf_status saf_mixed_attn_bwd_gqa(const void *q, const void *k, const void *v,
+                                          const void *o, const void *dout, const float *lse,
+                                          const float *a, const float *r, const float *logz,
+                                          const uint8_t *replaced_mask,
+                                          int B, int H, int H_kv, int T, int d_h,
+                                          void *dq, void *dk, void *dv, int grad_dtype,
+                                          void *workspace, size_t workspace_bytes,
+                                          void *stream);
+
+/*
  * Allocation-free backward, for callers that cannot pass a workspace: code
  * that may not call cudaMalloc (custom allocators' own callbacks, frameworks
  * that own all device memory), or that has no allocator to draw one from.
@@ -161,9 +197,9 @@ SAF_API saf_status saf_mixed_attn_bwd_noalloc(const void *q, const void *k, cons
 
 /*
  * Reads (synchronously: waits for `stream`) and clears the device error word
- * that the kernels keep in the first 256 bytes of `workspace`.  Those bytes
- * must be zero before the workspace is first used (e.g. one cudaMemset); the
- * kernels only ever set the word, and this call clears it again.
+ * that the kernels keep in the first 256 bytes of `workspace` (zero before
+ * first use, see Workspace above); the kernels only ever set the word, and
+ * this call clears it again.
  * Returns SAF_OK, SAF_ERR_TIMEOUT if a bounded device wait gave up since the
  * last check, SAF_ERR_WORKSPACE for a missing/short workspace, or SAF_ERR_CUDA.
  */

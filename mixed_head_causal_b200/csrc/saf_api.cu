@@ -45,6 +45,13 @@ saf_status build_headlist(const uint8_t* mask, int H, HeadList* hl) {
 
 inline saf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAF_OK : SAF_ERR_CUDA; }
 
+// K/V heads: at least one, dividing H (H == 0 allows any positive count).
+saf_status check_groups(int H, int H_kv) {
+    if (H_kv <= 0) return SAF_ERR_INVALID_ARG;
+    if (H > 0 && (H_kv > H || H % H_kv != 0)) return SAF_ERR_INVALID_ARG;
+    return SAF_OK;
+}
+
 // SAF_FORCE_MMA=1 in the environment routes every head through the
 // warp-level mma.sync kernels (the per-element path), for comparisons.
 bool force_mma_path() {
@@ -70,10 +77,14 @@ const char* saf_status_string(int status) {
 
 int saf_version(void) { return kVersion; }
 
-size_t saf_workspace_size(int B, int H, int T, int d_h, int is_bwd) {
-    if (check_shape(B, H, T, d_h) != SAF_OK) return (size_t)-1;
+size_t saf_workspace_size_gqa(int B, int H, int H_kv, int T, int d_h, int is_bwd) {
+    if (check_shape(B, H, T, d_h) != SAF_OK || check_groups(H, H_kv) != SAF_OK) return (size_t)-1;
     if ((int64_t)B * H * T == 0) return 0;
-    return ws_layout(B, H, T, is_bwd ? 1 : 0).total;
+    return ws_layout(B, H, T, is_bwd ? 1 : 0, H_kv).total;
+}
+
+size_t saf_workspace_size(int B, int H, int T, int d_h, int is_bwd) {
+    return saf_workspace_size_gqa(B, H, H, T, d_h, is_bwd);
 }
 
 saf_status saf_replaced_lognorm(const float* a, const float* r, const uint8_t* replaced_mask,
@@ -90,11 +101,13 @@ saf_status saf_replaced_lognorm(const float* a, const float* r, const uint8_t* r
     return cuda_status(launch_lognorm(a, r, hl, T, logz, (cudaStream_t)stream));
 }
 
-saf_status saf_mixed_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                              const float* a, const float* r, const float* logz,
-                              const uint8_t* replaced_mask, int B, int H, int T, int d_h,
-                              void* workspace, size_t workspace_bytes, void* stream) {
+saf_status saf_mixed_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  const float* a, const float* r, const float* logz,
+                                  const uint8_t* replaced_mask, int B, int H, int H_kv, int T, int d_h,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
     saf_status st = check_shape(B, H, T, d_h);
+    if (st != SAF_OK) return st;
+    st = check_groups(H, H_kv);
     if (st != SAF_OK) return st;
     if ((int64_t)B * H * T == 0) return SAF_OK;
     HeadList hl;
@@ -107,7 +120,7 @@ saf_status saf_mixed_attn_fwd(const void* q, const void* k, const void* v, void*
         if (!a || !r) return SAF_ERR_INVALID_ARG;
         if (!aligned16(a) || !aligned16(r) || (logz && !aligned16(logz))) return SAF_ERR_INVALID_ARG;
     }
-    const WsLayout L = ws_layout(B, H, T, 0);
+    const WsLayout L = ws_layout(B, H, T, 0, H_kv);
     if (!workspace || workspace_bytes < L.total) return SAF_ERR_WORKSPACE;
     if (!aligned256(workspace)) return SAF_ERR_INVALID_ARG;
 
@@ -124,22 +137,35 @@ saf_status saf_mixed_attn_fwd(const void* q, const void* k, const void* v, void*
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
     const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
     __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
-    if (force_mma_path()) return cuda_status(launch_fwd_mma(qb, kb, vb, ob, lse, a, r, lz, hl, B, H, T, s));
+    if (force_mma_path()) {
+        if (H_kv != H) return SAF_ERR_UNSUPPORTED;  // the warp-level path has no shared K/V
+        return cuda_status(launch_fwd_mma(qb, kb, vb, ob, lse, a, r, lz, hl, B, H, T, s));
+    }
     const ReplacedWs rw = replaced_ws(ws, L, T);
     if (hl.n > 0 && launch_prep_replaced(a, r, lz, hl, T, rw, s) != cudaSuccess) return SAF_ERR_CUDA;
     cudaError_t e =
-        launch_fwd_tc(qb, kb, vb, ob, lse, a, r, lz, hl, rw, B, H, T, reinterpret_cast<unsigned int*>(ws), s);
+        launch_fwd_tc(qb, kb, vb, ob, lse, a, r, lz, hl, rw, B, H, H_kv, T, reinterpret_cast<unsigned int*>(ws), s);
     if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return SAF_ERR_CUDA;
     return SAF_OK;
 }
 
-saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const void* o,
-                              const void* dout, const float* lse, const float* a, const float* r,
-                              const float* logz, const uint8_t* replaced_mask, int B, int H, int T,
-                              int d_h, void* dq, void* dk, void* dv, int grad_dtype,
+saf_status saf_mixed_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const float* a, const float* r, const float* logz,
+                              const uint8_t* replaced_mask, int B, int H, int T, int d_h,
                               void* workspace, size_t workspace_bytes, void* stream) {
+    return saf_mixed_attn_fwd_gqa(q, k, v, o, lse, a, r, logz, replaced_mask, B, H, H, T, d_h, workspace,
+                                  workspace_bytes, stream);
+}
+
+saf_status saf_mixed_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                                  const void* dout, const float* lse, const float* a, const float* r,
+                                  const float* logz, const uint8_t* replaced_mask, int B, int H, int H_kv,
+                                  int T, int d_h, void* dq, void* dk, void* dv, int grad_dtype,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
     saf_status st = check_shape(B, H, T, d_h);
+    if (st != SAF_OK) return st;
+    st = check_groups(H, H_kv);
     if (st != SAF_OK) return st;
     if (grad_dtype != 0 && grad_dtype != 1) return SAF_ERR_UNSUPPORTED;
     if ((int64_t)B * H * T == 0) return SAF_OK;
@@ -154,7 +180,7 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
         if (!a || !r) return SAF_ERR_INVALID_ARG;
         if (!aligned16(a) || !aligned16(r) || (logz && !aligned16(logz))) return SAF_ERR_INVALID_ARG;
     }
-    const WsLayout L = ws_layout(B, H, T, 1);
+    const WsLayout L = ws_layout(B, H, T, 1, H_kv);
     if (!workspace || workspace_bytes < L.total) return SAF_ERR_WORKSPACE;
     if (!aligned256(workspace)) return SAF_ERR_INVALID_ARG;
 
@@ -172,6 +198,7 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
     const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
     const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
     if (force_mma_path()) {
+        if (H_kv != H) return SAF_ERR_UNSUPPORTED;  // the warp-level path has no shared K/V
         float* dvec = reinterpret_cast<float*>(ws + L.dvec);
         if (launch_bwd_dot(ob, dob, dvec, hl, B, H, T, s) != cudaSuccess) return SAF_ERR_CUDA;
         return cuda_status(launch_bwd_mma(qb, kb, vb, dob, lse, dvec, a, r, lz, hl, B, H, T, dq, dk, dv,
@@ -183,12 +210,30 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
     float* dvecp = reinterpret_cast<float*>(ws + L.dvecp);
     float* dqacc = reinterpret_cast<float*>(ws + L.dqacc);
     if (launch_bwd_pre(ob, dob, lse, B * H, T, nlse2p, dvecp, dqacc, s) != cudaSuccess) return SAF_ERR_CUDA;
-    cudaError_t e = launch_bwd_tc(qb, kb, vb, dob, nlse2p, dvecp, dqacc, a, r, lz, hl, rw, B, H, T, dk, dv,
-                                  grad_dtype, reinterpret_cast<unsigned int*>(ws), s);
+    // shared K/V: per-query-head fp32 dK, dV into the workspace, then summed per group
+    const bool grouped = H_kv != H;
+    float* dkh = grouped ? reinterpret_cast<float*>(ws + L.dkh) : nullptr;
+    float* dvh = grouped ? reinterpret_cast<float*>(ws + L.dvh) : nullptr;
+    cudaError_t e = launch_bwd_tc(qb, kb, vb, dob, nlse2p, dvecp, dqacc, a, r, lz, hl, rw, B, H, H_kv, T,
+                                  grouped ? dkh : dk, grouped ? dvh : dv, grouped ? 1 : grad_dtype,
+                                  reinterpret_cast<unsigned int*>(ws), s);
     if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return SAF_ERR_CUDA;
     if (launch_dq_convert(dqacc, dq, (int64_t)B * H * T, grad_dtype, s) != cudaSuccess) return SAF_ERR_CUDA;
+    if (grouped) {
+        if (launch_group_sum(dkh, dk, B, H, H_kv, T, grad_dtype, s) != cudaSuccess) return SAF_ERR_CUDA;
+        if (launch_group_sum(dvh, dv, B, H, H_kv, T, grad_dtype, s) != cudaSuccess) return SAF_ERR_CUDA;
+    }
     return SAF_OK;
+}
+
+saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, const float* a, const float* r,
+                              const float* logz, const uint8_t* replaced_mask, int B, int H, int T,
+                              int d_h, void* dq, void* dk, void* dv, int grad_dtype,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    return saf_mixed_attn_bwd_gqa(q, k, v, o, dout, lse, a, r, logz, replaced_mask, B, H, H, T, d_h, dq, dk, dv,
+                                  grad_dtype, workspace, workspace_bytes, stream);
 }
 
 saf_status saf_device_status(void* workspace, size_t workspace_bytes, void* stream) {

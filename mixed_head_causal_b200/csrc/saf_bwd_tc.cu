@@ -69,7 +69,7 @@ struct BwdTcParams {
     void* dv;
     unsigned int* err;
     int16_t slot_of_head[kMaxHeads];
-    int H, BH, T, Tp, nqb, grad_fp32;
+    int H, Hkv, BH, T, Tp, nqb, grad_fp32;  // Hkv: K/V heads (H / Hkv query heads share one)
     float scale, scale_log2;
 };
 
@@ -193,6 +193,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     int bh, J;
     grouped_order(blockIdx.x, p.BH, p.nqb, bh, J);
     const int h = bh % p.H;
+    const int bhkv = (bh / p.H) * p.Hkv + h / (p.H / p.Hkv);  // the K/V slice this query head reads
     const int slot = p.slot_of_head[h];
     const bool rep = slot >= 0;
     // a replaced head whose factors would leave fp32 range takes P^T itself
@@ -240,8 +241,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 prefetch_tmap(&tmK);
                 prefetch_tmap(&tmV);
                 mbar_expect_tx(bar_kv, 2 * TILE);
-                tma_load_3d(sb + SM_K, &tmK, bar_kv, 0, J * BN, bh);
-                tma_load_3d(sb + SM_V, &tmV, bar_kv, 0, J * BN, bh);
+                tma_load_3d(sb + SM_K, &tmK, bar_kv, 0, J * BN, bhkv);
+                tma_load_3d(sb + SM_V, &tmV, bar_kv, 0, J * BN, bhkv);
             }
             prefetch_tmap(&tmDO);
             for (int t = 0; t < ntiles; ++t) {
@@ -556,6 +557,38 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
 }
 
+// Shared K/V (Hkv < H): dK[b, g] = sum over the H / Hkv query heads h of group
+// g of the per-query-head fp32 rows, written in the output dtype (the
+// gradient of a shared input is the sum of its uses).  Four floats a thread.
+__global__ void __launch_bounds__(256) group_sum_kernel(const float* __restrict__ src, void* __restrict__ dst,
+                                                        int B, int H, int Hkv, int64_t rows_T, int grad_fp32) {
+    const int G = H / Hkv;
+    const int64_t per_head = rows_T * (kHeadDim / 4);  // float4s of one [T, 64] slice
+    const int64_t n = (int64_t)B * Hkv * per_head;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t bg = idx / per_head, off = idx - bg * per_head;
+        const int64_t b = bg / Hkv, g = bg - b * Hkv;
+        const float4* s0 = reinterpret_cast<const float4*>(src) + ((b * H + g * G) * per_head + off);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < G; ++u) {
+            const float4 x = s0[(int64_t)u * per_head];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        if (grad_fp32) {
+            reinterpret_cast<float4*>(dst)[idx] = acc;
+        } else {
+            uint2 o;
+            o.x = pack_bf16x2(acc.x, acc.y);
+            o.y = pack_bf16x2(acc.z, acc.w);
+            reinterpret_cast<uint2*>(dst)[idx] = o;
+        }
+    }
+}
+
 // rows of [BH, Tp]: -lse2 = -lse*log2(e) (-inf past T), D = rowsum(dO o O) (0
 // past T); zero the dQ accumulator rows.  8 threads per row.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
@@ -658,14 +691,27 @@ cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int gr
     return cudaGetLastError();
 }
 
+cudaError_t launch_group_sum(const float* src, void* dst, int B, int H, int Hkv, int T, int grad_fp32,
+                             cudaStream_t stream) {
+    const int64_t n4 = (int64_t)B * Hkv * T * (kHeadDim / 4);
+    if (n4 == 0) return cudaSuccess;
+    const int64_t blocks = (n4 + 255) / 256;
+    launch_begin(KID_GROUP_SUM, stream);
+    group_sum_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, stream>>>(src, dst, B, H, Hkv,
+                                                                                          (int64_t)T, grad_fp32);
+    launch_end(KID_GROUP_SUM, stream);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           const __nv_bfloat16* dout, const float* nlse2p, const float* dvecp, float* dqacc,
                           const float* a, const float* r, const float* logz, const HeadList& hl,
-                          const ReplacedWs& w, int B, int H, int T, void* dk, void* dv, int grad_fp32,
+                          const ReplacedWs& w, int B, int H, int Hkv, int T, void* dk, void* dv, int grad_fp32,
                           unsigned int* err, cudaStream_t stream) {
     const int BH = B * H;
     CUtensorMap mq, mk, mv, mdo, mdq;
-    if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, BH, T, &mk) || !make_tmap_bhtd(v, BH, T, &mv) ||
+    if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, B * Hkv, T, &mk) ||
+        !make_tmap_bhtd(v, B * Hkv, T, &mv) ||
         !make_tmap_bhtd(dout, BH, T, &mdo) || !make_tmap_bhtd_f32(dqacc, BH, T, &mdq))
         return cudaErrorNotSupported;
     BwdTcParams p;
@@ -683,6 +729,7 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     for (int hh = 0; hh < H; ++hh)
         if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
     p.H = H;
+    p.Hkv = Hkv;
     p.BH = BH;
     p.T = T;
     p.Tp = round_up128(T);

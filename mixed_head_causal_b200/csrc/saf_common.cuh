@@ -69,12 +69,14 @@ struct WsLayout {
     size_t nlse2p;    // [B*H, Tp] fp32 -lse * log2(e), -inf past T  (backward)
     size_t dvecp;    // [B*H, Tp] fp32 rowsum(dO o O), 0 past T      (backward)
     size_t dqacc;    // [B*H, T, 64] fp32 dQ accumulator              (backward)
+    size_t dkh, dvh; // [B*H, T, 64] fp32 per-query-head dK, dV (backward, shared K/V only)
     size_t total;
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline WsLayout ws_layout(int B, int H, int T, int is_bwd) {
+// Hkv < H: K/V shared by groups of H / Hkv query heads.
+inline WsLayout ws_layout(int B, int H, int T, int is_bwd, int Hkv = -1) {
     WsLayout L{};
     size_t off = 0;
     L.header = off; off += 256;
@@ -92,6 +94,10 @@ inline WsLayout ws_layout(int B, int H, int T, int is_bwd) {
         L.nlse2p = off; off = align256(off + 4 * BH * Tp);
         L.dvecp = off; off = align256(off + 4 * BH * Tp);
         L.dqacc = off; off = align256(off + 4 * BH * (size_t)T * kHeadDim);
+        if (Hkv > 0 && Hkv != H) {
+            L.dkh = off; off = align256(off + 4 * BH * (size_t)T * kHeadDim);
+            L.dvh = off; off = align256(off + 4 * BH * (size_t)T * kHeadDim);
+        }
     }
     L.total = off;
     return L;
@@ -128,7 +134,8 @@ int sm_count();
 // Kernel ids of the launch accounting (names in saf_profile.cu).
 enum KernelId {
     KID_LOGNORM = 1, KID_FWD_MMA = 2, KID_DOT = 3, KID_DKDV_MMA = 4, KID_DQ_MMA = 5,
-    KID_FWD_TC = 6, KID_BWD_TC = 7, KID_PREP_REPLACED = 8, KID_DQ_CONVERT = 9, KID_BWD_PRE = 10
+    KID_FWD_TC = 6, KID_BWD_TC = 7, KID_PREP_REPLACED = 8, KID_DQ_CONVERT = 9, KID_BWD_PRE = 10,
+    KID_GROUP_SUM = 11
 };
 // Every kernel launch of the library is bracketed by these two calls.
 void launch_begin(int kid, cudaStream_t s);
@@ -143,9 +150,10 @@ cudaError_t launch_prep_replaced(const float* a, const float* r, const float* lo
 // Tensor-core forward of every head (replaced heads whose factored form would
 // leave fp32 range, flag 1, take per-element exps of a + r - log Z); returns
 // cudaErrorNotSupported when the tensor maps cannot be built.
+// k, v hold Hkv heads; query head h reads K/V head h / (H / Hkv).
 cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
-                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, unsigned int* err,
+                          const HeadList& hl, const ReplacedWs& w, int B, int H, int Hkv, int T, unsigned int* err,
                           cudaStream_t stream);
 // Backward preprocessing for the tensor-core backward: padded lse*log2(e) and
 // rowsum(dO o O), and a zeroed dQ accumulator.
@@ -153,11 +161,16 @@ cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, co
                            float* nlse2p, float* dvecp, float* dqacc, cudaStream_t stream);
 // Tensor-core backward (dK, dV written; dQ reduced into dqacc); replaced
 // heads with flag 1 take per-element exps of a + r - log Z.
+// (dk, dv per query head: [B, H, T, 64]; with shared K/V the caller sums them
+// over each group with launch_group_sum)
 cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           const __nv_bfloat16* dout, const float* nlse2p, const float* dvecp, float* dqacc,
                           const float* a, const float* r, const float* logz, const HeadList& hl,
-                          const ReplacedWs& w, int B, int H, int T, void* dk, void* dv, int grad_fp32,
+                          const ReplacedWs& w, int B, int H, int Hkv, int T, void* dk, void* dv, int grad_fp32,
                           unsigned int* err, cudaStream_t stream);
+// dst[b, g] = sum of the H / Hkv fp32 rows src[b, h] of group g, [B, Hkv, T, 64] in the output dtype.
+cudaError_t launch_group_sum(const float* src, void* dst, int B, int H, int Hkv, int T, int grad_fp32,
+                             cudaStream_t stream);
 // dq = dqacc / sqrt(d_h) in the requested dtype.
 cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream);
 bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out);

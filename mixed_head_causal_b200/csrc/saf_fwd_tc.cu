@@ -62,7 +62,7 @@ struct FwdTcParams {
     ReplacedWs w;
     unsigned int* err;
     int16_t slot_of_head[kMaxHeads];
-    int H, BH, T, nqb;
+    int H, Hkv, BH, T, nqb;  // query heads, K/V heads (H / Hkv query heads share one)
     float scale_log2;
 };
 
@@ -236,7 +236,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // (b, h) slice and query block of an item, grouped longest-first order
     // (query block I visits I + 1 key blocks)
     struct Item {
-        int bh, I, h, slot;
+        int bh, bhkv, I, h, slot;  // query slice, its K/V slice, query block, head, replaced slot
         bool rep, direct;
     };
     auto decode = [&](int item) {
@@ -245,6 +245,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         grouped_order((unsigned)item, p.BH, p.nqb, it.bh, rank);
         it.I = p.nqb - 1 - rank;
         it.h = it.bh % p.H;
+        it.bhkv = (it.bh / p.H) * p.Hkv + it.h / (p.H / p.Hkv);
         it.slot = p.slot_of_head[it.h];
         it.rep = it.slot >= 0;
         it.direct = it.rep && p.w.flag[it.h] != 0;  // per-element exps instead of the factored form
@@ -281,7 +282,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const int g = gk + j, s = g % NSK, u = g / NSK;
                     if (!mbar_wait(bar_ke + 8 * s, (u & 1) ^ 1, kWaitLimit)) return false;
                     mbar_expect_tx(bar_kf + 8 * s, TILE_BYTES);
-                    tma_load_3d(sbase + SM_K + s * TILE_BYTES, &tmK, bar_kf + 8 * s, 0, j * BN, it.bh);
+                    tma_load_3d(sbase + SM_K + s * TILE_BYTES, &tmK, bar_kf + 8 * s, 0, j * BN, it.bhkv);
                     return true;
                 };
                 if (!it.rep && !load_k(0)) { ok = false; break; }
@@ -290,7 +291,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const int g = gv + j, s = g % NSV, u = g / NSV;
                     if (!mbar_wait(bar_ve + 8 * s, (u & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                     mbar_expect_tx(bar_vf + 8 * s, TILE_BYTES);
-                    tma_load_3d(sbase + SM_V + s * TILE_BYTES, &tmV, bar_vf + 8 * s, 0, j * BN, it.bh);
+                    tma_load_3d(sbase + SM_V + s * TILE_BYTES, &tmV, bar_vf + 8 * s, 0, j * BN, it.bhkv);
                 }
                 if (!it.rep) gk += nkb;
                 gv += nkb;
@@ -597,11 +598,12 @@ bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out) {
 
 cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
-                          const HeadList& hl, const ReplacedWs& w, int B, int H, int T, unsigned int* err,
+                          const HeadList& hl, const ReplacedWs& w, int B, int H, int Hkv, int T, unsigned int* err,
                           cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     const int BH = B * H;
-    if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, BH, T, &mk) || !make_tmap_bhtd(v, BH, T, &mv))
+    if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, B * Hkv, T, &mk) ||
+        !make_tmap_bhtd(v, B * Hkv, T, &mv))
         return cudaErrorNotSupported;
     FwdTcParams p;
     p.o = o;
@@ -616,6 +618,7 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     for (int hh = 0; hh < H; ++hh)
         if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
     p.H = H;
+    p.Hkv = Hkv;
     p.BH = BH;
     p.T = T;
     p.nqb = (T + BM - 1) / BM;

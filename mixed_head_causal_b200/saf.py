@@ -25,10 +25,15 @@ SIGNATURES = {
     "saf_status_string": ([_i], ctypes.c_char_p),
     "saf_version": ([], _i),
     "saf_workspace_size": ([_i, _i, _i, _i, _i], _sz),
+    "saf_workspace_size_gqa": ([_i, _i, _i, _i, _i, _i], _sz),
     "saf_replaced_lognorm": ([_vp, _vp, _vp, _i, _i, _vp, _vp], _i),
     "saf_mixed_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp], _i),
     "saf_mixed_attn_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                             _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
+    "saf_mixed_attn_fwd_gqa": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp],
+                               _i),
+    "saf_mixed_attn_bwd_gqa": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "saf_device_status": ([_vp, _sz, _vp], _i),
     "saf_mixed_attn_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                     _vp, _vp, _vp, _i, _vp], _i),
@@ -90,16 +95,21 @@ def _mask_buffer(mask) -> Tuple[ctypes.Array, int]:
     return buf, m.numel()
 
 
-def workspace_size(B: int, H: int, T: int, d_h: int = HEAD_DIM, backward: bool = False) -> int:
-    n = load().saf_workspace_size(B, H, T, d_h, 1 if backward else 0)
+def workspace_size(B: int, H: int, T: int, d_h: int = HEAD_DIM, backward: bool = False,
+                   h_kv: Optional[int] = None) -> int:
+    """Workspace bytes; h_kv (default H) K/V heads shared by groups of H / h_kv query heads."""
+    if h_kv is None or h_kv == H:
+        n = load().saf_workspace_size(B, H, T, d_h, 1 if backward else 0)
+    else:
+        n = load().saf_workspace_size_gqa(B, H, h_kv, T, d_h, 1 if backward else 0)
     if n == ctypes.c_size_t(-1).value:
         raise SafError(SAF_ERR_INVALID_ARG, "saf_workspace_size")
     return int(n)
 
 
-def new_workspace(B: int, H: int, T: int, device, backward: bool = False) -> torch.Tensor:
-    """A zero-initialised uint8 workspace (the error word must start at 0)."""
-    n = max(256, workspace_size(B, H, T, HEAD_DIM, backward))
+def new_workspace(B: int, H: int, T: int, device, backward: bool = False, h_kv: Optional[int] = None) -> torch.Tensor:
+    """A zero-initialised uint8 workspace (its 256-byte header must start at 0)."""
+    n = max(256, workspace_size(B, H, T, HEAD_DIM, backward, h_kv))
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
@@ -127,48 +137,71 @@ def mixed_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: tor
                    rho: torch.Tensor, mask, logz: Optional[torch.Tensor] = None,
                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None, stream=None):
-    """Forward of one mixed-head layer.  Returns (O [B,H,T,64] bf16, lse [B,H,T] fp32)."""
-    B, H, T, d = v.shape
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _check_layer_tensor(n, t, (B, H, T, d))
+    """Forward of one mixed-head layer.  Returns (O [B,H,T,64] bf16, lse [B,H,T] fp32).
+
+    k, v may hold fewer heads than q (H_kv dividing H): query head h then reads
+    K/V head h // (H // H_kv) (grouped-query attention)."""
+    B, H, T, d = q.shape
+    Hkv = k.shape[1]
+    _check_layer_tensor("q", q, (B, H, T, d))
+    for n, t in (("k", k), ("v", v)):
+        _check_layer_tensor(n, t, (B, Hkv, T, d))
     if out is None:
-        out = torch.empty_like(v)
+        out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty(B, H, T, dtype=torch.float32, device=v.device)
+        lse = torch.empty(B, H, T, dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = new_workspace(B, H, T, v.device, backward=False)
+        workspace = new_workspace(B, H, T, q.device, backward=False, h_kv=Hkv)
     mbuf, mh = _mask_buffer(mask)
     if mh != H:
         raise ValueError("mask length != H")
-    _check(load().saf_mixed_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(alpha), _ptr(rho),
-                                     _ptr(logz), ctypes.addressof(mbuf), B, H, T, d, _ptr(workspace),
-                                     workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
-           "saf_mixed_attn_fwd")
+    wsb = workspace.numel() * workspace.element_size()
+    if Hkv == H:
+        st = load().saf_mixed_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(alpha), _ptr(rho),
+                                       _ptr(logz), ctypes.addressof(mbuf), B, H, T, d, _ptr(workspace), wsb,
+                                       _stream_ptr(stream))
+    else:
+        st = load().saf_mixed_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(alpha),
+                                           _ptr(rho), _ptr(logz), ctypes.addressof(mbuf), B, H, Hkv, T, d,
+                                           _ptr(workspace), wsb, _stream_ptr(stream))
+    _check(st, "saf_mixed_attn_fwd")
     return out, lse
 
 
 def mixed_attn_bwd(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtype=torch.bfloat16,
                    dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """Backward of one mixed-head layer.  Returns (dQ, dK, dV) in grad_dtype (bf16 or fp32)."""
-    B, H, T, d = v.shape
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+    """Backward of one mixed-head layer.  Returns (dQ, dK, dV) in grad_dtype (bf16 or fp32).
+
+    With shared K/V (k, v holding H_kv < H heads) dK and dV have H_kv heads, each
+    the sum over the query heads of its group."""
+    B, H, T, d = q.shape
+    Hkv = k.shape[1]
+    for n, t in (("q", q), ("o", o), ("dout", dout)):
         _check_layer_tensor(n, t, (B, H, T, d))
+    for n, t in (("k", k), ("v", v)):
+        _check_layer_tensor(n, t, (B, Hkv, T, d))
     if grad_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("grad_dtype must be bf16 or fp32")
     gd = 1 if grad_dtype == torch.float32 else 0
-    dq = torch.empty(B, H, T, d, dtype=grad_dtype, device=v.device) if dq is None else dq
-    dk = torch.empty(B, H, T, d, dtype=grad_dtype, device=v.device) if dk is None else dk
-    dv = torch.empty(B, H, T, d, dtype=grad_dtype, device=v.device) if dv is None else dv
+    dq = torch.empty(B, H, T, d, dtype=grad_dtype, device=q.device) if dq is None else dq
+    dk = torch.empty(B, Hkv, T, d, dtype=grad_dtype, device=q.device) if dk is None else dk
+    dv = torch.empty(B, Hkv, T, d, dtype=grad_dtype, device=q.device) if dv is None else dv
     if workspace is None:
-        workspace = new_workspace(B, H, T, v.device, backward=True)
+        workspace = new_workspace(B, H, T, q.device, backward=True, h_kv=Hkv)
     mbuf, mh = _mask_buffer(mask)
     if mh != H:
         raise ValueError("mask length != H")
-    _check(load().saf_mixed_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(alpha),
-                                     _ptr(rho), _ptr(logz), ctypes.addressof(mbuf), B, H, T, d,
-                                     _ptr(dq), _ptr(dk), _ptr(dv), gd, _ptr(workspace),
-                                     workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
-           "saf_mixed_attn_bwd")
+    wsb = workspace.numel() * workspace.element_size()
+    if Hkv == H:
+        st = load().saf_mixed_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(alpha),
+                                       _ptr(rho), _ptr(logz), ctypes.addressof(mbuf), B, H, T, d,
+                                       _ptr(dq), _ptr(dk), _ptr(dv), gd, _ptr(workspace), wsb, _stream_ptr(stream))
+    else:
+        st = load().saf_mixed_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                           _ptr(alpha), _ptr(rho), _ptr(logz), ctypes.addressof(mbuf), B, H, Hkv,
+                                           T, d, _ptr(dq), _ptr(dk), _ptr(dv), gd, _ptr(workspace), wsb,
+                                           _stream_ptr(stream))
+    _check(st, "saf_mixed_attn_bwd")
     return dq, dk, dv
 
 

@@ -156,6 +156,32 @@ class Oracle:
                                      _f64(dout).reshape(sh), ar, rr, rep, n_threads)
         return dq.reshape(v.shape), dk.reshape(v.shape), dv.reshape(v.shape)
 
+    # ---- shared K/V (grouped-query attention): the plain layer with K and V
+    # repeated over each group of H / H_kv consecutive query heads; the
+    # gradient of a shared head is the sum over its group (each use of an
+    # input adds to its gradient).
+    @staticmethod
+    def _repeat_kv(x, H):
+        x64 = _f64(x)
+        B, Hkv, T, d = x64.shape
+        if H % Hkv:
+            raise ValueError("H_kv must divide H")
+        return np.ascontiguousarray(np.repeat(x64, H // Hkv, axis=1))
+
+    def fwd_gqa(self, q, k, v, a, r, mask, n_threads: Optional[int] = None):
+        """Forward with k, v [B,H_kv,T,d] shared by groups of H / H_kv query heads."""
+        H = _f64(q).shape[1]
+        return self.fwd(q, self._repeat_kv(k, H), self._repeat_kv(v, H), a, r, mask, n_threads)
+
+    def bwd_gqa(self, q, k, v, dout, a, r, mask, n_threads: Optional[int] = None):
+        """Backward with shared K/V.  Returns (dQ [B,H,T,d], dK, dV [B,H_kv,T,d])."""
+        q64 = _f64(q)
+        B, H, T, d = q64.shape
+        Hkv = _f64(k).shape[1]
+        dq, dk, dv = self.bwd(q64, self._repeat_kv(k, H), self._repeat_kv(v, H), dout, a, r, mask, n_threads)
+        G = H // Hkv
+        return dq, dk.reshape(B, Hkv, G, T, d).sum(axis=2), dv.reshape(B, Hkv, G, T, d).sum(axis=2)
+
 
 _default: Optional[Oracle] = None
 
@@ -177,6 +203,14 @@ def fwd(q, k, v, a, r, mask, n_threads=None):
 
 def bwd(q, k, v, dout, a, r, mask, n_threads=None):
     return default().bwd(q, k, v, dout, a, r, mask, n_threads)
+
+
+def fwd_gqa(q, k, v, a, r, mask, n_threads=None):
+    return default().fwd_gqa(q, k, v, a, r, mask, n_threads)
+
+
+def bwd_gqa(q, k, v, dout, a, r, mask, n_threads=None):
+    return default().bwd_gqa(q, k, v, dout, a, r, mask, n_threads)
 
 
 def fwd_slices(q, k, v, a_rows, r_rows, replaced, n_threads=None):

@@ -302,6 +302,46 @@ def check_layer_mixes_head_kinds(orc):
             assert np.all(dq[b, h] == 0) and np.all(dk[b, h] == 0)
 
 
+def check_grouped_kv_matches_autograd(orc):
+    """Shared K/V (H_kv = 2 heads, groups of 2 query heads, one replaced head in
+    each group): forward and backward against fp64 torch autograd of a dense
+    layer that indexes the shared K/V per query head (autograd sums the
+    gradient of each shared head over its uses by itself)."""
+    g = torch.Generator().manual_seed(14)
+    B, H, Hkv, T, d = 2, 4, 2, 20, 8
+    G = H // Hkv
+    q, do = (torch.randn(B, H, T, d, generator=g, dtype=torch.float64) for _ in range(2))
+    k, v = (torch.randn(B, Hkv, T, d, generator=g, dtype=torch.float64) for _ in range(2))
+    rng = _rng(14)
+    a = np.full((H, T), np.nan)
+    r = np.full((H, T), np.nan)
+    mask = np.array([0, 1, 0, 1], dtype=np.uint8)
+    for h in (1, 3):
+        a[h], r[h] = _pattern(T, rng)
+        r[h] *= 0.5 * h
+    o, lse = orc.fwd_gqa(q, k, v, a, r, mask)
+    dq, dk, dv = orc.bwd_gqa(q, k, v, do, a, r, mask)
+    assert dk.shape == (B, Hkv, T, d) and dv.shape == (B, Hkv, T, d)
+    qq, kk, vv = (x.clone().requires_grad_(True) for x in (q, k, v))
+    outs = []
+    for b in range(B):
+        for h in range(H):
+            kv = h // G
+            if mask[h]:
+                P, _ = _dense_pattern(a[h], r[h])
+                outs.append(torch.from_numpy(P) @ vv[b, kv])
+            else:
+                outs.append(_sdpa(qq[b, h][None, None], kk[b, kv][None, None], vv[b, kv][None, None])[0, 0])
+    ref = torch.stack(outs).reshape(B, H, T, d)
+    (ref * do).sum().backward()
+    np.testing.assert_allclose(o, ref.detach().numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dq, qq.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, kk.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, vv.grad.numpy(), rtol=0, atol=1e-11)
+    for h in (1, 3):
+        assert np.all(dq[:, h] == 0)
+
+
 def check_all_masked_row(orc):
     """Every logit -inf (a = -inf): output 0 and lse = -inf, no NaN."""
     T, d = 5, 4
@@ -329,5 +369,6 @@ ALL_CHECKS = [
     check_ordinary_finite_differences,
     check_zero_query_is_running_mean,
     check_layer_mixes_head_kinds,
+    check_grouped_kv_matches_autograd,
     check_all_masked_row,
 ]

@@ -96,6 +96,32 @@ def test_planted_mistake_is_caught(desc, old, new, nth):
         shutil.rmtree(tmp, ignore_errors=True)
 
 
+@pytest.mark.parametrize("mistake", ["groups interleaved", "first head of the group only"])
+def test_planted_grouped_kv_mistake_is_caught(mistake, monkeypatch):
+    """Plausible mistakes in the shared-K/V marshalling (query head h reading
+    K/V head h % H_kv, or a shared head's gradient taken from one query head
+    instead of the group sum) are rejected by the grouped-K/V pin."""
+    orc = oracle.Oracle()
+    if mistake == "groups interleaved":
+        def bad_repeat(x, H):
+            x64 = np.asarray(x, dtype=np.float64)
+            return np.ascontiguousarray(np.tile(x64, (1, H // x64.shape[1], 1, 1)))
+        monkeypatch.setattr(oracle.Oracle, "_repeat_kv", staticmethod(bad_repeat))
+    else:
+        good_bwd = oracle.Oracle.bwd_gqa
+
+        def bad_bwd(self, q, k, v, dout, a, r, mask, n_threads=None):
+            dq, dk, dv = good_bwd(self, q, k, v, dout, a, r, mask, n_threads)
+            B, H, T, d = np.asarray(q).shape
+            Hkv = np.asarray(k).shape[1]
+            full = self.bwd(q, self._repeat_kv(k, H), self._repeat_kv(v, H), dout, a, r, mask, n_threads)
+            G = H // Hkv
+            return dq, full[1][:, ::G], full[2][:, ::G]
+        monkeypatch.setattr(oracle.Oracle, "bwd_gqa", bad_bwd)
+    with pytest.raises(AssertionError):
+        pins.check_grouped_kv_matches_autograd(orc)
+
+
 def test_golden_regression(orc):
     """Frozen oracle outputs on a tiny mixed case (tests/golden/make_golden.py)."""
     path = os.path.join(HERE, "golden", "tiny_mixed_layer.json")

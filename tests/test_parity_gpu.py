@@ -211,3 +211,42 @@ def test_guarded_and_factored_heads_in_one_call():
     x["rho"][0] = -0.02 * torch.arange(650, dtype=torch.float32) + torch.randn(650, generator=gen) * 30.0
     got = P.run_layer(w, x)
     P.check_slices(w, x, got, _all_slices(w))
+
+
+@pytest.mark.parametrize("B,H,Hkv,T,replaced", [(2, 8, 2, 650, [1, 5]), (1, 4, 1, 300, [0, 3]),
+                                                (2, 6, 3, 1000, [2]), (1, 4, 2, 129, [])],
+                         ids=["gqa4_t650", "mqa_t300", "gqa2_t1000", "gqa2_t129_no_replaced"])
+@pytest.mark.parametrize("grad_dtype", [torch.float32, torch.bfloat16], ids=["grad_fp32", "grad_bf16"])
+def test_grouped_kv_layer(B, H, Hkv, T, replaced, grad_dtype):
+    """Shared K/V heads (H / Hkv query heads per K/V head, replaced heads mixed
+    in): O, lse, dQ and the group-summed dK, dV against the oracle."""
+    w = I.custom(B, H, T, replaced)
+    x = I.make_inputs(w, 21)
+    k = x["k"][:, :Hkv].contiguous()
+    v = x["v"][:, :Hkv].contiguous()
+    g = P.to_gpu(x)
+    kg, vg = k.cuda(), v.cuda()
+    o, lse = saf.mixed_attn_fwd(g["q"], kg, vg, g["alpha"], g["rho"], x["mask"])
+    dq, dk, dv = saf.mixed_attn_bwd(g["q"], kg, vg, o, g["do"], lse, g["alpha"], g["rho"], x["mask"],
+                                    grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    assert tuple(dk.shape) == (B, Hkv, T, 64) and tuple(dv.shape) == (B, Hkv, T, 64)
+    o_ref, lse_ref = oracle.fwd_gqa(x["q"], k, v, x["alpha"], x["rho"], x["mask"])
+    dq_ref, dk_ref, dv_ref = oracle.bwd_gqa(x["q"], k, v, x["do"], x["alpha"], x["rho"], x["mask"])
+    P.compare("O", o.cpu(), o_ref, stored_bf16=True)
+    lse_fin = np.isfinite(lse_ref)
+    assert np.abs(lse.cpu().double().numpy()[lse_fin] - lse_ref[lse_fin]).max() <= P.TOL_LSE
+    bf = grad_dtype == torch.bfloat16
+    P.compare("dQ", dq.cpu(), dq_ref, bf)
+    P.compare("dK", dk.cpu(), dk_ref, bf)
+    P.compare("dV", dv.cpu(), dv_ref, bf)
+
+
+def test_grouped_kv_argument_errors():
+    """H_kv must divide H; the warp-level path has no shared K/V."""
+    w = I.custom(1, 4, 64, [1])
+    x = I.make_inputs(w, 3)
+    g = P.to_gpu(x)
+    k3 = g["k"][:, :3].contiguous()
+    with pytest.raises(saf.SafError):
+        saf.mixed_attn_fwd(g["q"], k3, k3, g["alpha"], g["rho"], x["mask"])
