@@ -81,6 +81,8 @@ class Oracle:
         lib.oracle_fwd_slices.restype = i
         lib.oracle_bwd_slices.argtypes = [i, i, i, u8p, dp, dp, dp, dp, dp, dp, dp, dp, dp, i]
         lib.oracle_bwd_slices.restype = i
+        lib.oracle_pattern_grad_slice.argtypes = [i, i, dp, dp, dp, dp, dp, dp]
+        lib.oracle_pattern_grad_slice.restype = i
         self.lib = lib
 
     def lognorm(self, a, r) -> np.ndarray:
@@ -156,6 +158,29 @@ class Oracle:
                                      _f64(dout).reshape(sh), ar, rr, rep, n_threads)
         return dq.reshape(v.shape), dk.reshape(v.shape), dv.reshape(v.shape)
 
+    def pattern_grad(self, v, dout, a, r, mask):
+        """Trainable pattern: (dalpha, drho) [H,T] of a loss with output
+        gradient dout through the replaced heads (rows of ordinary heads 0).
+        v, dout [B,H,T,d]; sums over the batch (alpha, rho are per head)."""
+        v64, do64 = _f64(v), _f64(dout)
+        B, H, T, d = v64.shape
+        a64, r64 = _f64(a), _f64(r)
+        m = _f64(mask) != 0
+        da = np.zeros((H, T))
+        dr = np.zeros((H, T))
+        for h in range(H):
+            if not m[h]:
+                continue
+            ah, rh = np.ascontiguousarray(a64[h]), np.ascontiguousarray(r64[h])
+            for b in range(B):
+                vb, db = np.ascontiguousarray(v64[b, h]), np.ascontiguousarray(do64[b, h])
+                dah, drh = np.zeros(T), np.zeros(T)
+                if self.lib.oracle_pattern_grad_slice(T, d, _p(ah), _p(rh), _p(vb), _p(db), _p(dah), _p(drh)):
+                    raise MemoryError("oracle pattern gradient failed")
+                da[h] += dah
+                dr[h] += drh
+        return da, dr
+
     # ---- shared K/V (grouped-query attention): the plain layer with K and V
     # repeated over each group of H / H_kv consecutive query heads; the
     # gradient of a shared head is the sum over its group (each use of an
@@ -203,6 +228,10 @@ def fwd(q, k, v, a, r, mask, n_threads=None):
 
 def bwd(q, k, v, dout, a, r, mask, n_threads=None):
     return default().bwd(q, k, v, dout, a, r, mask, n_threads)
+
+
+def pattern_grad(v, dout, a, r, mask):
+    return default().pattern_grad(v, dout, a, r, mask)
 
 
 def fwd_gqa(q, k, v, a, r, mask, n_threads=None):

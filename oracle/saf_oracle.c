@@ -24,6 +24,13 @@
  *    gradients dV = P^T dO, dP = dO V^T, dS = P o (dP - rowsum(P o dP)),
  *    dQ = s dS K, dK = s dS^T Q with s = 1/sqrt(d_h).
  *
+ *  - Trainable pattern (the variant of Table 14 of the same page, where alpha
+ *    and rho receive gradients): the derivative of a loss through Eq. (3).
+ *    P is the row softmax of the logits alpha(j) + rho(i-j), so with
+ *    dP = dO V^T and D(i) = sum_j P(i,j) dP(i,j) the logit gradient is
+ *    dS(i,j) = P(i,j) (dP(i,j) - D(i)), and each logit's two terms collect
+ *    it: dalpha(j) = sum_i dS(i,j), drho(d) = sum_{i-j=d} dS(i,j).
+ *
  * Max-shifts (subtracting the row maximum before exp) are the only numerical
  * device used; they leave every result unchanged mathematically.  A row
  * whose every term is -inf (possible only with -inf alpha/rho) yields an all
@@ -101,6 +108,46 @@ static void fwd_ordinary(int T, int d, const double *q, const double *k,
         }
         lse[i] = m + log(l);
     }
+}
+
+/* ------------------------------------------------------ trainable pattern */
+
+/*
+ * One slice of a replaced head: adds its contributions to da[T] and dr[T]
+ * (the caller sums slices of the same head).  v, dout [T,d].  Returns 0, or
+ * -1 on allocation failure.
+ */
+int oracle_pattern_grad_slice(int T, int d, const double *a, const double *r,
+                              const double *v, const double *dout, double *da, double *dr)
+{
+    double *logz = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    double *prow = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    double *dprow = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!logz || !prow || !dprow) {
+        free(logz); free(prow); free(dprow);
+        return -1;
+    }
+    oracle_lognorm(T, a, r, logz);
+    for (int i = 0; i < T; ++i) {
+        if (logz[i] == -INFINITY) continue;
+        const double *doi = dout + (size_t)i * d;
+        double Di = 0.0;
+        for (int j = 0; j <= i; ++j) {
+            prow[j] = exp(a[j] + r[i - j] - logz[i]);
+            const double *vj = v + (size_t)j * d;
+            double dp = 0.0;
+            for (int c = 0; c < d; ++c) dp += doi[c] * vj[c];
+            dprow[j] = dp;
+            Di += prow[j] * dp;
+        }
+        for (int j = 0; j <= i; ++j) {
+            const double ds = prow[j] * (dprow[j] - Di);
+            da[j] += ds;
+            dr[i - j] += ds;
+        }
+    }
+    free(logz); free(prow); free(dprow);
+    return 0;
 }
 
 /* --------------------------------------------------------------- backward */

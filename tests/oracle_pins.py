@@ -342,6 +342,78 @@ def check_grouped_kv_matches_autograd(orc):
         assert np.all(dq[:, h] == 0)
 
 
+def _dense_pattern_torch_grads(a, r, v, do):
+    """fp64 torch autograd of L = sum(O o dO), O = P V, P the row softmax of the
+    masked logits a[j] + r[i-j] (a library routine differentiates Eq. (3))."""
+    T = a.shape[0]
+    at = torch.tensor(a, dtype=torch.float64, requires_grad=True)
+    rt = torch.tensor(r, dtype=torch.float64, requires_grad=True)
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    logits = at[j.expand(T, T)] + rt[(i - j).clamp(min=0)]
+    logits = logits.masked_fill(j > i, float("-inf"))
+    P = torch.softmax(logits, dim=1)
+    loss = sum(((P @ torch.as_tensor(vb)) * torch.as_tensor(db)).sum() for vb, db in zip(v, do))
+    loss.backward()
+    return at.grad.numpy(), rt.grad.numpy()
+
+
+def check_pattern_grad_matches_autograd(orc):
+    """Trainable pattern: dalpha, drho summed over the batch, per head, against
+    torch autograd of the dense definition; ordinary heads' rows stay 0."""
+    rng = _rng(15)
+    B, H, T, d = 2, 3, 21, 6
+    v, do = rng.normal(size=(B, H, T, d)), rng.normal(size=(B, H, T, d))
+    a = np.full((H, T), np.nan)
+    r = np.full((H, T), np.nan)
+    mask = np.array([1, 0, 1], dtype=np.uint8)
+    for h in (0, 2):
+        a[h], r[h] = _pattern(T, rng)
+        r[h] *= 1 + h
+    da, dr = orc.pattern_grad(v, do, a, r, mask)
+    assert np.all(da[1] == 0) and np.all(dr[1] == 0)
+    for h in (0, 2):
+        ga, gr = _dense_pattern_torch_grads(a[h], r[h], v[:, h], do[:, h])
+        np.testing.assert_allclose(da[h], ga, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dr[h], gr, rtol=0, atol=1e-12)
+
+
+def check_pattern_grad_finite_differences(orc):
+    """Central differences of L = sum(O o dO) through the oracle's own forward."""
+    rng = _rng(16)
+    T, d = 7, 3
+    a, r = _pattern(T, rng)
+    v, do = rng.normal(size=(1, 1, T, d)), rng.normal(size=(1, 1, T, d))
+    da, dr = orc.pattern_grad(v, do, a[None], r[None], np.array([1], dtype=np.uint8))
+    z = np.zeros((1, T, d))
+
+    def loss(aa, rr):
+        o, _ = orc.fwd_slices(z, z, v[0], aa[None], rr[None], [1])
+        return float((o[0] * do[0, 0]).sum())
+    eps = 1e-6
+    for idx in range(T):
+        e = np.zeros(T)
+        e[idx] = eps
+        np.testing.assert_allclose(da[0, idx], (loss(a + e, r) - loss(a - e, r)) / (2 * eps), rtol=0, atol=1e-7)
+        np.testing.assert_allclose(dr[0, idx], (loss(a, r + e) - loss(a, r - e)) / (2 * eps), rtol=0, atol=1e-7)
+
+
+def check_pattern_grad_sums_vanish(orc):
+    """Each row of dS sums to zero (softmax rows are normalised), so the
+    dalpha and drho vectors of every head sum to zero; a constant shift of
+    a or r leaves both gradients unchanged."""
+    rng = _rng(17)
+    B, T, d = 2, 33, 5
+    a, r = _pattern(T, rng)
+    v, do = rng.normal(size=(B, 1, T, d)), rng.normal(size=(B, 1, T, d))
+    m = np.array([1], dtype=np.uint8)
+    da, dr = orc.pattern_grad(v, do, a[None], r[None], m)
+    assert abs(da.sum()) < 1e-11 and abs(dr.sum()) < 1e-11
+    da2, dr2 = orc.pattern_grad(v, do, a[None] + 7.0, r[None] - 3.0, m)
+    np.testing.assert_allclose(da2, da, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dr2, dr, rtol=0, atol=1e-11)
+
+
 def check_all_masked_row(orc):
     """Every logit -inf (a = -inf): output 0 and lse = -inf, no NaN."""
     T, d = 5, 4
@@ -370,5 +442,8 @@ ALL_CHECKS = [
     check_zero_query_is_running_mean,
     check_layer_mixes_head_kinds,
     check_grouped_kv_matches_autograd,
+    check_pattern_grad_matches_autograd,
+    check_pattern_grad_finite_differences,
+    check_pattern_grad_sums_vanish,
     check_all_masked_row,
 ]

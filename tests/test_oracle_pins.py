@@ -60,6 +60,13 @@ MUTANTS = [
     ("replaced bwd: normaliser of the wrong row",
      "double p = exp(a[j] + r[i - j] - logz[i]);\n            double *dvj",
      "double p = exp(a[j] + r[i - j] - logz[j]);\n            double *dvj", 0),
+    ("pattern grad: distance bin of the key",
+     "dr[i - j] += ds;", "dr[j] += ds;", 0),
+    ("pattern grad: row term D dropped",
+     "const double ds = prow[j] * (dprow[j] - Di);", "const double ds = prow[j] * dprow[j];", 0),
+    ("pattern grad: dP from the wrong row of V",
+     "const double *vj = v + (size_t)j * d;\n            double dp = 0.0;",
+     "const double *vj = v + (size_t)i * d;\n            double dp = 0.0;", 0),
     ("replaced bwd: dQ not cleared",
      "memset(dq, 0, sizeof(double) * (size_t)T * d);\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz",
      "for (int c = 0; c < T * d; ++c) dq[c] = 1e-3 * c;\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz", 0),
