@@ -53,6 +53,12 @@ def parse():
     ap.add_argument("--head-cost", action="store_true",
                     help="instead of the headline line, time the workload's shape with 0, 25, 50 and 100%% of "
                          "the heads replaced and fit t = t0 + c_o n_o + c_r n_r per pass")
+    ap.add_argument("--pattern-grad", action="store_true",
+                    help="instead of the headline line, time the trainable-pattern gradient (dalpha, drho) of "
+                         "the workload's replaced heads")
+    ap.add_argument("--gqa", type=int, default=0, metavar="H_KV",
+                    help="instead of the headline line, time fwd and bwd with K/V shared by groups of "
+                         "H / H_KV query heads")
     return ap.parse_args()
 
 
@@ -464,6 +470,76 @@ def head_cost(args, local):
     print(json.dumps(out), flush=True)
 
 
+def _time(fn, steps):
+    for _ in range(3):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def pattern_grad_cost(args, local):
+    """Trainable-pattern gradient of the workload's replaced heads: time per
+    call (log Z given), and the dP contraction's algorithmic TFLOP/s (one
+    causal T x T x d unit per replaced (b, h); the kernel runs it twice)
+    against the measured bf16 peak."""
+    from mixed_head_causal_b200 import saf
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS[args.workload]
+    x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
+    mask = x["mask"]
+    n_r = int(mask.sum())
+    lz = saf.replaced_lognorm(x["alpha"], x["rho"], mask)
+    da = torch.empty(w.H, w.T, dtype=torch.float32, device=dev)
+    dr = torch.empty_like(da)
+    ms = _time(lambda: saf.replaced_pattern_grad(x["v"], x["do"], x["alpha"], x["rho"], mask, logz=lz, da=da,
+                                                 dr=dr), args.steps)
+    flops = w.B * n_r * w.d * float(w.T) ** 2
+    pk = peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({"metric": "trainable-pattern gradient (dalpha, drho) ms per call", "value": ms, "unit": "ms",
+                      "higher_is_better": False,
+                      "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "n_replaced": n_r},
+                      "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                   "frac": tf / pk["bf16_tflops"], "path": "warp-level mma.sync, two passes"}}),
+          flush=True)
+
+
+def gqa_cost(args, local):
+    """Forward and backward with K/V shared by groups of H / H_kv query heads
+    (the workload's shape and head mix): ms and tokens/s per pass."""
+    from mixed_head_causal_b200 import saf
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS[args.workload]
+    hkv = args.gqa
+    if w.H % hkv:
+        raise SystemExit("--gqa must divide H")
+    x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
+    mask = x["mask"]
+    k, v = x["k"][:, :hkv].contiguous(), x["v"][:, :hkv].contiguous()
+    lz = saf.replaced_lognorm(x["alpha"], x["rho"], mask)
+    o = torch.empty_like(x["q"])
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
+    wsf = saf.new_workspace(w.B, w.H, w.T, dev, backward=False, h_kv=hkv)
+    wsb = saf.new_workspace(w.B, w.H, w.T, dev, backward=True, h_kv=hkv)
+    dq = torch.empty_like(x["q"])
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    fwd = lambda: saf.mixed_attn_fwd(x["q"], k, v, x["alpha"], x["rho"], mask, logz=lz, out=o, lse=lse,  # noqa: E731
+                                     workspace=wsf)
+    bwd = lambda: saf.mixed_attn_bwd(x["q"], k, v, o, x["do"], lse, x["alpha"], x["rho"], mask, logz=lz,  # noqa: E731
+                                     dq=dq, dk=dk, dv=dv, workspace=wsb)
+    tf, tb = _time(fwd, args.steps), _time(bwd, args.steps)
+    tokens = w.B * w.T
+    print(json.dumps({"metric": "mixed-head causal attn with shared K/V heads, ms per pass", "unit": "ms",
+                      "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": hkv, "T": w.T},
+                      "fwd_ms": tf, "bwd_ms": tb, "tokens_per_s": tokens / ((tf + tb) * 1e-3)}), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -471,6 +547,12 @@ def main():
         if args.head_cost:
             if rank == 0:
                 head_cost(args, local)
+        elif args.pattern_grad:
+            if rank == 0:
+                pattern_grad_cost(args, local)
+        elif args.gqa:
+            if rank == 0:
+                gqa_cost(args, local)
         elif args.impl == "reference":
             reference_arm(args, world, rank)
         else:

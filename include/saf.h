@@ -196,6 +196,29 @@ SAF_API saf_status saf_mixed_attn_bwd_noalloc(const void *q, const void *k, cons
                                               void *stream);
 
 /*
+ * Trainable pattern (the variant of Table 14 of "When Can Attention Heads Be
+ * Statically Defined?", where the pattern vectors are trained): the gradients
+ * of a loss with output gradient `dout` with respect to a and r, through
+ * Eq. (3).  With P the pattern, dP = dout V^T and D(i) = sum_j P(i,j) dP(i,j):
+ *   dS(i,j) = P(i,j) (dP(i,j) - D(i)),
+ *   da[h,j] = sum over b, i of dS(i,j),   dr[h,d] = sum over b, i - j = d of dS(i,j).
+ *   v, dout  [B,H,T,d_h] bf16 in (rows of ordinary heads are not read).
+ *   a, r     [H,T] fp32; logz [H,T] from saf_replaced_lognorm, or NULL to
+ *            compute it into `workspace` (saf_workspace_size(B,H,T,d_h,0)
+ *            bytes, 256-byte aligned; unused when logz is given).
+ *   da, dr   [H,T] fp32 out, overwritten; rows of ordinary heads are zero.
+ * Sums are accumulated with fp32 atomics (the summation order, and so the
+ * last bits, vary from run to run).
+ */
+SAF_API saf_status saf_replaced_pattern_grad(const void *v, const void *dout,
+                                             const float *a, const float *r, const float *logz,
+                                             const uint8_t *replaced_mask,
+                                             int B, int H, int T, int d_h,
+                                             float *da, float *dr,
+                                             void *workspace, size_t workspace_bytes,
+                                             void *stream);
+
+/*
  * Reads (synchronously: waits for `stream`) and clears the device error word
  * that the kernels keep in the first 256 bytes of `workspace` (zero before
  * first use, see Workspace above); the kernels only ever set the word, and

@@ -236,6 +236,38 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
                                   grad_dtype, workspace, workspace_bytes, stream);
 }
 
+saf_status saf_replaced_pattern_grad(const void* v, const void* dout, const float* a, const float* r,
+                                     const float* logz, const uint8_t* replaced_mask, int B, int H, int T,
+                                     int d_h, float* da, float* dr, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+    saf_status st = check_shape(B, H, T, d_h);
+    if (st != SAF_OK) return st;
+    if ((int64_t)H * T == 0) return SAF_OK;
+    HeadList hl;
+    st = build_headlist(replaced_mask, H, &hl);
+    if (st != SAF_OK) return st;
+    if (!da || !dr || !aligned16(da) || !aligned16(dr)) return SAF_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(da, 0, sizeof(float) * (size_t)H * T, s) != cudaSuccess) return SAF_ERR_CUDA;
+    if (cudaMemsetAsync(dr, 0, sizeof(float) * (size_t)H * T, s) != cudaSuccess) return SAF_ERR_CUDA;
+    if (hl.n == 0 || B == 0) return SAF_OK;
+    if (!v || !dout || !a || !r) return SAF_ERR_INVALID_ARG;
+    if (!aligned16(v) || !aligned16(dout) || !aligned16(a) || !aligned16(r) || (logz && !aligned16(logz)))
+        return SAF_ERR_INVALID_ARG;
+    const float* lz = logz;
+    if (lz == nullptr) {
+        const WsLayout L = ws_layout(B, H, T, 0);
+        if (!workspace || workspace_bytes < L.total) return SAF_ERR_WORKSPACE;
+        if (!aligned256(workspace)) return SAF_ERR_INVALID_ARG;
+        float* lzw = reinterpret_cast<float*>(static_cast<char*>(workspace) + L.logz);
+        if (launch_lognorm(a, r, hl, T, lzw, s) != cudaSuccess) return SAF_ERR_CUDA;
+        lz = lzw;
+    }
+    return cuda_status(launch_pattern_grad(static_cast<const __nv_bfloat16*>(v),
+                                           static_cast<const __nv_bfloat16*>(dout), a, r, lz, hl, B, H, T, da, dr,
+                                           s));
+}
+
 saf_status saf_device_status(void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace || workspace_bytes < sizeof(WsHeader)) return SAF_ERR_WORKSPACE;
     WsHeader hdr;

@@ -135,7 +135,7 @@ int sm_count();
 enum KernelId {
     KID_LOGNORM = 1, KID_FWD_MMA = 2, KID_DOT = 3, KID_DKDV_MMA = 4, KID_DQ_MMA = 5,
     KID_FWD_TC = 6, KID_BWD_TC = 7, KID_PREP_REPLACED = 8, KID_DQ_CONVERT = 9, KID_BWD_PRE = 10,
-    KID_GROUP_SUM = 11
+    KID_GROUP_SUM = 11, KID_PATTERN_GRAD = 12
 };
 // Every kernel launch of the library is bracketed by these two calls.
 void launch_begin(int kid, cudaStream_t s);
@@ -168,6 +168,10 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
                           const float* a, const float* r, const float* logz, const HeadList& hl,
                           const ReplacedWs& w, int B, int H, int Hkv, int T, void* dk, void* dv, int grad_fp32,
                           unsigned int* err, cudaStream_t stream);
+// Trainable pattern: adds dalpha, drho [H, T] of the replaced heads (zeroed by the caller).
+cudaError_t launch_pattern_grad(const __nv_bfloat16* v, const __nv_bfloat16* dout, const float* a, const float* r,
+                                const float* logz, const HeadList& hl, int B, int H, int T, float* da, float* dr,
+                                cudaStream_t stream);
 // dst[b, g] = sum of the H / Hkv fp32 rows src[b, h] of group g, [B, Hkv, T, 64] in the output dtype.
 cudaError_t launch_group_sum(const float* src, void* dst, int B, int H, int Hkv, int T, int grad_fp32,
                              cudaStream_t stream);

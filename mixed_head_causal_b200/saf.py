@@ -35,6 +35,7 @@ SIGNATURES = {
     "saf_mixed_attn_bwd_gqa": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                 _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "saf_device_status": ([_vp, _sz, _vp], _i),
+    "saf_replaced_pattern_grad": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
     "saf_mixed_attn_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                     _vp, _vp, _vp, _i, _vp], _i),
     "saf_launch_count": ([], ctypes.c_uint64),
@@ -203,6 +204,27 @@ def mixed_attn_bwd(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtyp
                                            _stream_ptr(stream))
     _check(st, "saf_mixed_attn_bwd")
     return dq, dk, dv
+
+
+def replaced_pattern_grad(v, dout, alpha, rho, mask, logz=None, da=None, dr=None, workspace=None, stream=None):
+    """Trainable pattern: (dalpha, drho) [H, T] fp32 of the replaced heads
+    (rows of ordinary heads zero) for the output gradient dout."""
+    B, H, T, d = v.shape
+    for n, t in (("v", v), ("dout", dout)):
+        _check_layer_tensor(n, t, (B, H, T, d))
+    da = torch.empty(H, T, dtype=torch.float32, device=v.device) if da is None else da
+    dr = torch.empty(H, T, dtype=torch.float32, device=v.device) if dr is None else dr
+    if workspace is None and logz is None:
+        workspace = new_workspace(B, H, T, v.device, backward=False)
+    mbuf, mh = _mask_buffer(mask)
+    if mh != H:
+        raise ValueError("mask length != H")
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().saf_replaced_pattern_grad(_ptr(v), _ptr(dout), _ptr(alpha), _ptr(rho), _ptr(logz),
+                                            ctypes.addressof(mbuf), B, H, T, d, _ptr(da), _ptr(dr),
+                                            _ptr(workspace), wsb, _stream_ptr(stream)),
+           "saf_replaced_pattern_grad")
+    return da, dr
 
 
 def mixed_attn_bwd_noalloc(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtype=torch.bfloat16,

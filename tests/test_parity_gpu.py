@@ -250,3 +250,41 @@ def test_grouped_kv_argument_errors():
     k3 = g["k"][:, :3].contiguous()
     with pytest.raises(saf.SafError):
         saf.mixed_attn_fwd(g["q"], k3, k3, g["alpha"], g["rho"], x["mask"])
+
+
+@pytest.mark.parametrize("B,H,T,replaced", [(2, 3, 300, [0, 2]), (1, 2, 1000, [1]), (3, 4, 129, [0, 1, 2, 3]),
+                                            (1, 2, 64, [0])],
+                         ids=["b2_t300", "b1_t1000", "b3_t129_all_replaced", "b1_t64"])
+def test_pattern_grad(B, H, T, replaced):
+    """Trainable pattern: dalpha, drho against the oracle.  The kernel works in
+    fp32 (exact bf16 products, fp32 sums and exps); its error relative to the
+    largest gradient entry of a head stays far below 2e-4 (the fp32 rounding
+    of sums over about B*T terms), which is the bound used here; rows of
+    ordinary heads must be exactly zero."""
+    w = I.custom(B, H, T, replaced)
+    x = I.make_inputs(w, 31)
+    g = P.to_gpu(x)
+    da, dr = saf.replaced_pattern_grad(g["v"], g["do"], g["alpha"], g["rho"], x["mask"])
+    torch.cuda.synchronize()
+    da_ref, dr_ref = oracle.pattern_grad(x["v"], x["do"], x["alpha"], x["rho"], x["mask"])
+    da, dr = da.cpu().double().numpy(), dr.cpu().double().numpy()
+    for h in range(H):
+        if h not in replaced:
+            assert np.all(da[h] == 0) and np.all(dr[h] == 0)
+            continue
+        for got, ref in ((da[h], da_ref[h]), (dr[h], dr_ref[h])):
+            scale = max(1.0, np.abs(ref).max())
+            assert np.abs(got - ref).max() <= 2e-4 * scale, (h, np.abs(got - ref).max(), scale)
+
+
+def test_pattern_grad_extreme_range_and_explicit_logz():
+    """Pattern vectors far beyond the factored form's range (per-element exps
+    in every path) and a log Z passed in: same results as the oracle."""
+    w, x = _special(500, lambda T: torch.randn(T) * 40.0, lambda T: -0.05 * torch.arange(T, dtype=torch.float32))
+    g = P.to_gpu(x)
+    lz = saf.replaced_lognorm(g["alpha"], g["rho"], x["mask"])
+    da, dr = saf.replaced_pattern_grad(g["v"], g["do"], g["alpha"], g["rho"], x["mask"], logz=lz)
+    torch.cuda.synchronize()
+    da_ref, dr_ref = oracle.pattern_grad(x["v"], x["do"], x["alpha"], x["rho"], x["mask"])
+    for got, ref in ((da[1].cpu().double().numpy(), da_ref[1]), (dr[1].cpu().double().numpy(), dr_ref[1])):
+        assert np.abs(got - ref).max() <= 2e-4 * max(1.0, np.abs(ref).max())
