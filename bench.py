@@ -174,8 +174,9 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_sample(w, seed=0):
-    """A bounded sample of (b, h) slices with the workload's head-kind mix."""
+def oracle_sample(w, seed=0, groups=1):
+    """A bounded sample of (b, h) slices with the workload's head-kind mix,
+    `groups` copies of the smallest such group, on batches 0, 1, ..."""
     mask = I.replaced_mask(w, seed).numpy()
     rep = [h for h in range(w.H) if mask[h]]
     ordn = [h for h in range(w.H) if not mask[h]]
@@ -183,7 +184,11 @@ def oracle_sample(w, seed=0):
     from math import gcd
     g = gcd(len(ordn), len(rep)) if rep and ordn else 1
     n_o, n_r = (len(ordn) // g, len(rep) // g) if rep and ordn else (min(4, len(ordn)), min(4, len(rep)))
-    slices = [(0, ordn[i % len(ordn)]) for i in range(n_o)] + [(0, rep[i % len(rep)]) for i in range(n_r)]
+    slices = []
+    for gi in range(groups):
+        b = gi % w.B
+        slices += [(b, ordn[(gi * n_o + i) % len(ordn)]) for i in range(n_o)]
+        slices += [(b, rep[(gi * n_r + i) % len(rep)]) for i in range(n_r)]
     return slices
 
 
@@ -210,35 +215,48 @@ def run_oracle_sample(w, slices, seed=0, threads=None):
 
 
 def cpu_baseline(w):
-    slices = oracle_sample(w)
+    # four groups of the head-kind mix: 16 slices, about ten seconds of CPU
+    # work at the 124M shape on the machine's host cores
+    slices = oracle_sample(w, groups=4)
     dt, frac, cores = run_oracle_sample(w, slices)
     return {"value": w.tokens * frac / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{len(slices)} of {w.B * w.H} (batch, head) slices of {w.name} (same head-kind mix), "
                       f"fwd{'+bwd' if w.backward else ''}, {dt:.1f} s, scaled by slice count"}
 
 
+def arm_config(w, world, grad_dtype):
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_h": w.d, "n_replaced": len(I.replaced_heads(w)),
+            "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+            "passes": "fwd+bwd" if w.backward else "fwd", "grad_dtype": grad_dtype,
+            "l2": "inputs larger than L2 (no flush)", "flops_per_step": I.flops(w)["total"] * world}
+
+
 def reference_arm(args, world, rank):
     w = I.WORKLOADS[args.workload]
     if rank != 0:
         return
-    slices = oracle_sample(w)
-    for _ in range(args.warmup):
-        run_oracle_sample(w, slices)
-    times = []
-    for _ in range(args.steps):
-        dt, frac, cores = run_oracle_sample(w, slices)
-        times.append(dt)
-    total = sum(times)
-    value = w.tokens * frac * args.steps / total
+    # one slice per step, cycling through one group of the head-kind mix, so
+    # that any --steps K --warmup W run stays within a few minutes; the rate is
+    # the slices' share of the workload's tokens over their total time
+    group = oracle_sample(w)
+    for s in range(args.warmup):
+        run_oracle_sample(w, [group[s % len(group)]])
+    total, done, cores = 0.0, 0.0, 1
+    for s in range(args.steps):
+        dt, frac, cores = run_oracle_sample(w, [group[s % len(group)]])
+        total += dt
+        done += frac
+    value = w.tokens * done / total
+    slices = group
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_h": w.d,
-                       "n_replaced": len(I.replaced_heads(w))},
+            "config": arm_config(w, args.gpus, args.grad_dtype),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{len(slices)} of {w.B * w.H} (batch, head) slices per step, "
-                                       "scaled by slice count"},
+                             "sample": f"one of {w.B * w.H} (batch, head) slices per step, cycling through "
+                                       f"{len(slices)} with the layer's head-kind mix, scaled by slice count"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -401,11 +419,7 @@ def our_arm(args, world, rank, local):
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "tflops": tflops, "tflops_frac_of_peak": tflops / pk["bf16_tflops"],
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_h": w.d, "n_replaced": n_r,
-                       "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
-                       "passes": "fwd+bwd" if w.backward else "fwd", "grad_dtype": args.grad_dtype,
-                       "l2": "inputs larger than L2 (no flush)",
-                       "flops_per_step": fl["total"] * world},
+            "config": arm_config(w, world, args.grad_dtype),
             "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
             "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
         }
