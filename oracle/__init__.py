@@ -83,6 +83,8 @@ class Oracle:
         lib.oracle_bwd_slices.restype = i
         lib.oracle_pattern_grad_slice.argtypes = [i, i, dp, dp, dp, dp, dp, dp]
         lib.oracle_pattern_grad_slice.restype = i
+        lib.oracle_calibration_head.argtypes = [i, i, i, dp, dp, dp, dp]
+        lib.oracle_calibration_head.restype = i
         self.lib = lib
 
     def lognorm(self, a, r) -> np.ndarray:
@@ -158,6 +160,25 @@ class Oracle:
                                      _f64(dout).reshape(sh), ar, rr, rep, n_threads)
         return dq.reshape(v.shape), dk.reshape(v.shape), dv.reshape(v.shape)
 
+    def calibration(self, q, k):
+        """Calibration statistics of every head over the N samples of q, k
+        [N,H,T,d]: (A_hat [H,T,T], s_var [H]) per Eq. (1); N >= 2."""
+        q64, k64 = _f64(q), _f64(k)
+        N, H, T, d = q64.shape
+        if N < 2:
+            raise ValueError("Eq. (1) needs N >= 2 samples")
+        a_hat = np.zeros((H, T, T))
+        svar = np.zeros(H)
+        for h in range(H):
+            qh, kh = np.ascontiguousarray(q64[:, h]), np.ascontiguousarray(k64[:, h])
+            ah = np.zeros((T, T))
+            sv = ctypes.c_double(0.0)
+            if self.lib.oracle_calibration_head(N, T, d, _p(qh), _p(kh), _p(ah), ctypes.byref(sv)):
+                raise MemoryError("oracle calibration failed")
+            a_hat[h] = ah
+            svar[h] = sv.value
+        return a_hat, svar
+
     def pattern_grad(self, v, dout, a, r, mask):
         """Trainable pattern: (dalpha, drho) [H,T] of a loss with output
         gradient dout through the replaced heads (rows of ordinary heads 0).
@@ -232,6 +253,10 @@ def bwd(q, k, v, dout, a, r, mask, n_threads=None):
 
 def pattern_grad(v, dout, a, r, mask):
     return default().pattern_grad(v, dout, a, r, mask)
+
+
+def calibration(q, k):
+    return default().calibration(q, k)
 
 
 def fwd_gqa(q, k, v, a, r, mask, n_threads=None):

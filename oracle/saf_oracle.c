@@ -31,6 +31,11 @@
  *    dS(i,j) = P(i,j) (dP(i,j) - D(i)), and each logit's two terms collect
  *    it: dalpha(j) = sum_i dS(i,j), drho(d) = sum_{i-j=d} dS(i,j).
  *
+ *  - Calibration (section 二.1 of the reading notes): over N calibration
+ *    sequences, the sample mean of each head's causal softmax attention
+ *    matrix, A_hat = (1/N) sum_n A^(n), and its reconstruction error
+ *    s_var = sum_n ||A^(n) - A_hat||_F^2 / ((N - 1) T^2)   (Eq. (1)).
+ *
  * Max-shifts (subtracting the row maximum before exp) are the only numerical
  * device used; they leave every result unchanged mathematically.  A row
  * whose every term is -inf (possible only with -inf alpha/rho) yields an all
@@ -108,6 +113,55 @@ static void fwd_ordinary(int T, int d, const double *q, const double *k,
         }
         lse[i] = m + log(l);
     }
+}
+
+/* ------------------------------------------------------------ calibration */
+
+/*
+ * One head over N samples: q, k [N,T,d] (sample n at offset n*T*d).  Writes
+ * the mean attention matrix a_hat [T,T] (zero above the diagonal) and returns
+ * s_var through *svar (N >= 2).  Returns 0, or -1 on allocation failure.
+ */
+int oracle_calibration_head(int N, int T, int d, const double *q, const double *k, double *a_hat, double *svar)
+{
+    const size_t TT = (size_t)T * T;
+    double *a = malloc(sizeof(double) * (TT > 0 ? TT : 1) * (size_t)(N > 0 ? N : 1));
+    double *srow = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!a || !srow) {
+        free(a); free(srow);
+        return -1;
+    }
+    const double scale = 1.0 / sqrt((double)d);
+    for (int n = 0; n < N; ++n) {
+        const double *qn = q + (size_t)n * T * d, *kn = k + (size_t)n * T * d;
+        double *an = a + (size_t)n * TT;
+        for (int i = 0; i < T; ++i) {
+            double m = -INFINITY;
+            for (int j = 0; j <= i; ++j) {
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += qn[(size_t)i * d + c] * kn[(size_t)j * d + c];
+                srow[j] = scale * dot;
+                if (srow[j] > m) m = srow[j];
+            }
+            double l = 0.0;
+            for (int j = 0; j <= i; ++j) l += exp(srow[j] - m);
+            for (int j = 0; j < T; ++j) an[(size_t)i * T + j] = j <= i ? exp(srow[j] - m) / l : 0.0;
+        }
+    }
+    for (size_t e = 0; e < TT; ++e) {
+        double sum = 0.0;
+        for (int n = 0; n < N; ++n) sum += a[(size_t)n * TT + e];
+        a_hat[e] = sum / N;
+    }
+    double err = 0.0;
+    for (int n = 0; n < N; ++n)
+        for (size_t e = 0; e < TT; ++e) {
+            const double x = a[(size_t)n * TT + e] - a_hat[e];
+            err += x * x;
+        }
+    *svar = err / ((double)(N - 1) * (double)T * (double)T);
+    free(a); free(srow);
+    return 0;
 }
 
 /* ------------------------------------------------------ trainable pattern */

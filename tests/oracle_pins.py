@@ -414,6 +414,58 @@ def check_pattern_grad_sums_vanish(orc):
     np.testing.assert_allclose(dr2, dr, rtol=0, atol=1e-11)
 
 
+def _read_attention(orc, q, k):
+    """A = softmax_causal(q k^T / sqrt(d)) of one slice, read off the oracle's
+    forward with V = identity (an independent code path)."""
+    T, d = q.shape
+    # the forward takes one width for q, k and v: pad q, k to width T, with q
+    # scaled so that the forward's 1/sqrt(T) becomes 1/sqrt(d)
+    qp, kp = np.zeros((T, T)), np.zeros((T, T))
+    qp[:, :d] = np.asarray(q) * np.sqrt(T / d)
+    kp[:, :d] = np.asarray(k)
+    nan = np.full((1, T), np.nan)
+    o, _ = orc.fwd_slices(qp[None], kp[None], np.eye(T)[None], nan, nan, [0])
+    return o[0]
+
+
+def check_calibration_closed_forms(orc):
+    """Eq. (1) and the sample mean: identical samples give s_var = 0 and the
+    mean equal to the (forward-read) attention matrix; two samples give
+    s_var = ||A1 - A2||_F^2 / (2 T^2); the mean is row-stochastic and causal."""
+    rng = _rng(18)
+    T, d = 17, 8
+    q, k = rng.normal(size=(T, d)) * 1.3, rng.normal(size=(T, d)) * 1.3
+    Q = np.stack([q, q, q])[:, None]
+    K = np.stack([k, k, k])[:, None]
+    a_hat, sv = orc.calibration(Q, K)
+    A = _read_attention(orc, q, k)
+    np.testing.assert_allclose(a_hat[0], A, rtol=0, atol=1e-13)
+    assert sv[0] < 1e-28
+    q2, k2 = rng.normal(size=(T, d)), rng.normal(size=(T, d))
+    a_hat, sv = orc.calibration(np.stack([q, q2])[:, None], np.stack([k, k2])[:, None])
+    A2 = _read_attention(orc, q2, k2)
+    np.testing.assert_allclose(a_hat[0], 0.5 * (A + A2), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(sv[0], ((A - A2) ** 2).sum() / (2 * T * T), rtol=1e-9, atol=0)
+    np.testing.assert_allclose(a_hat[0].sum(axis=1), np.ones(T), rtol=0, atol=1e-13)
+    assert np.all(np.triu(a_hat[0], 1) == 0)
+
+
+def check_calibration_mean_is_linear(orc):
+    """A_hat V equals the mean of the oracle's forward outputs A_n V (same V
+    for every sample), head by head; s_var does not depend on sample order."""
+    rng = _rng(19)
+    N, H, T, d = 4, 2, 12, 4
+    q, k = rng.normal(size=(N, H, T, d)), rng.normal(size=(N, H, T, d))
+    v = rng.normal(size=(T, d))
+    a_hat, sv = orc.calibration(q, k)
+    nan = np.full((1, T), np.nan)
+    for h in range(H):
+        outs = [orc.fwd_slices(q[n, h][None], k[n, h][None], v[None], nan, nan, [0])[0][0] for n in range(N)]
+        np.testing.assert_allclose(a_hat[h] @ v, np.mean(outs, axis=0), rtol=0, atol=1e-13)
+    _, sv2 = orc.calibration(q[::-1], k[::-1])
+    np.testing.assert_allclose(sv2, sv, rtol=1e-13, atol=0)
+
+
 def check_all_masked_row(orc):
     """Every logit -inf (a = -inf): output 0 and lse = -inf, no NaN."""
     T, d = 5, 4
@@ -445,5 +497,7 @@ ALL_CHECKS = [
     check_pattern_grad_matches_autograd,
     check_pattern_grad_finite_differences,
     check_pattern_grad_sums_vanish,
+    check_calibration_closed_forms,
+    check_calibration_mean_is_linear,
     check_all_masked_row,
 ]

@@ -67,6 +67,13 @@ MUTANTS = [
     ("pattern grad: dP from the wrong row of V",
      "const double *vj = v + (size_t)j * d;\n            double dp = 0.0;",
      "const double *vj = v + (size_t)i * d;\n            double dp = 0.0;", 0),
+    ("calibration: mean over N - 1",
+     "a_hat[e] = sum / N;", "a_hat[e] = sum / (N - 1);", 0),
+    ("calibration: Eq. (1) normalised by N",
+     "*svar = err / ((double)(N - 1) * (double)T * (double)T);", "*svar = err / ((double)N * (double)T * (double)T);", 0),
+    ("calibration: scores not scaled",
+     "srow[j] = scale * dot;\n                if (srow[j] > m) m = srow[j];\n            }\n            double l = 0.0;\n            for (int j = 0; j <= i; ++j) l += exp(srow[j] - m);\n            for (int j = 0; j < T; ++j) an",
+     "srow[j] = dot;\n                if (srow[j] > m) m = srow[j];\n            }\n            double l = 0.0;\n            for (int j = 0; j <= i; ++j) l += exp(srow[j] - m);\n            for (int j = 0; j < T; ++j) an", 0),
     ("replaced bwd: dQ not cleared",
      "memset(dq, 0, sizeof(double) * (size_t)T * d);\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz",
      "for (int c = 0; c < T * d; ++c) dq[c] = 1e-3 * c;\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz", 0),
