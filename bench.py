@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--pattern-grad", action="store_true",
                     help="instead of the headline line, time the trainable-pattern gradient (dalpha, drho) of "
                          "the workload's replaced heads")
+    ap.add_argument("--calibration", action="store_true",
+                    help="instead of the headline line, time the calibration statistics (A_hat, s_var) over "
+                         "the workload's batch as N samples, every head ordinary")
     ap.add_argument("--gqa", type=int, default=0, metavar="H_KV",
                     help="instead of the headline line, time fwd and bwd with K/V shared by groups of "
                          "H / H_KV query heads")
@@ -524,6 +527,29 @@ def pattern_grad_cost(args, local):
           flush=True)
 
 
+def calibration_cost(args, local):
+    """Calibration statistics over the workload's B sequences (every head
+    ordinary): ms per call and the score contraction's algorithmic TFLOP/s
+    (one causal T x T x d unit per (sample, head); the kernel runs it twice)."""
+    from mixed_head_causal_b200 import saf
+    dev = torch.device("cuda", local)
+    w = I.custom(I.WORKLOADS[args.workload].B, I.WORKLOADS[args.workload].H, I.WORKLOADS[args.workload].T, [])
+    x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
+    _, lse = saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], x["mask"])
+    a_hat = torch.empty(w.H, w.T, w.T, dtype=torch.float32, device=dev)
+    svar = torch.empty(w.H, dtype=torch.float32, device=dev)
+    ms = _time(lambda: saf.attn_calibration(x["q"], x["k"], lse, a_hat=a_hat, svar=svar), args.steps)
+    flops = w.B * w.H * w.d * float(w.T) ** 2
+    pk = peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({"metric": "calibration statistics (A_hat, s_var) ms per call", "value": ms, "unit": "ms",
+                      "higher_is_better": False,
+                      "config": {"workload": w.name, "N": w.B, "H": w.H, "T": w.T},
+                      "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                   "frac": tf / pk["bf16_tflops"], "path": "warp-level mma.sync, two passes",
+                                   "a_hat_bytes": 4 * w.H * w.T * w.T}}), flush=True)
+
+
 def gqa_cost(args, local):
     """Forward and backward with K/V shared by groups of H / H_kv query heads
     (the workload's shape and head mix): ms and tokens/s per pass."""
@@ -567,6 +593,9 @@ def main():
         elif args.gqa:
             if rank == 0:
                 gqa_cost(args, local)
+        elif args.calibration:
+            if rank == 0:
+                calibration_cost(args, local)
         elif args.impl == "reference":
             reference_arm(args, world, rank)
         else:

@@ -219,6 +219,28 @@ SAF_API saf_status saf_replaced_pattern_grad(const void *v, const void *dout,
                                              void *stream);
 
 /*
+ * Calibration statistics (section 二.1 of the reading notes for "When Can
+ * Attention Heads Be Statically Defined?"): over N >= 2 calibration sequences
+ * run through plain causal softmax attention (every head ordinary), the
+ * sample mean of each head's attention matrix and its reconstruction error,
+ *   a_hat[h] = (1/N) sum_n A_h^(n)                       [H,T,T] fp32 out
+ *   svar[h]  = sum_n ||A_h^(n) - a_hat[h]||_F^2 / ((N-1) T^2)   (Eq. (1)) [H] fp32 out
+ * with A^(n) = softmax_causal(q_n k_n^T / sqrt(d_h)); no per-sample T x T
+ * matrix is stored.
+ *   q, k   [N,H,T,d_h] bf16 in (the N samples as the batch dimension).
+ *   lse    [N,H,T] fp32: the row log-sum-exp the forward pass returns for
+ *          these inputs (saf_mixed_attn_fwd with no replaced head).
+ *   workspace: at least saf_calibration_workspace_size(H,T,d_h) bytes.
+ * N < 2 returns SAF_ERR_INVALID_ARG.  Deterministic (fixed-order sums).
+ */
+SAF_API size_t saf_calibration_workspace_size(int H, int T, int d_h);
+SAF_API saf_status saf_attn_calibration(const void *q, const void *k, const float *lse,
+                                        int N, int H, int T, int d_h,
+                                        float *a_hat, float *svar,
+                                        void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
+/*
  * Reads (synchronously: waits for `stream`) and clears the device error word
  * that the kernels keep in the first 256 bytes of `workspace` (zero before
  * first use, see Workspace above); the kernels only ever set the word, and

@@ -236,6 +236,29 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
                                   grad_dtype, workspace, workspace_bytes, stream);
 }
 
+size_t saf_calibration_workspace_size(int H, int T, int d_h) {
+    if (check_shape(1, H, T, d_h) != SAF_OK) return (size_t)-1;
+    return sizeof(float) * calibration_partial_floats(H, T);
+}
+
+saf_status saf_attn_calibration(const void* q, const void* k, const float* lse, int N, int H, int T, int d_h,
+                                float* a_hat, float* svar, void* workspace, size_t workspace_bytes, void* stream) {
+    saf_status st = check_shape(N, H, T, d_h);
+    if (st != SAF_OK) return st;
+    if (N < 2) return SAF_ERR_INVALID_ARG;  // Eq. (1) divides by N - 1
+    if ((int64_t)H * T == 0) return SAF_OK;
+    if ((double)H * T * T > 9.0e18 / sizeof(float)) return SAF_ERR_INVALID_ARG;
+    if (!q || !k || !lse || !a_hat || !svar) return SAF_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(lse) || !aligned16(a_hat) || !aligned16(svar))
+        return SAF_ERR_INVALID_ARG;
+    const size_t need = sizeof(float) * calibration_partial_floats(H, T);
+    if (!workspace || workspace_bytes < need) return SAF_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return SAF_ERR_INVALID_ARG;
+    return cuda_status(launch_calibration(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                          lse, N, H, T, a_hat, svar, static_cast<float*>(workspace),
+                                          (cudaStream_t)stream));
+}
+
 saf_status saf_replaced_pattern_grad(const void* v, const void* dout, const float* a, const float* r,
                                      const float* logz, const uint8_t* replaced_mask, int B, int H, int T,
                                      int d_h, float* da, float* dr, void* workspace, size_t workspace_bytes,

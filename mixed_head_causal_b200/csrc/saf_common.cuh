@@ -135,7 +135,7 @@ int sm_count();
 enum KernelId {
     KID_LOGNORM = 1, KID_FWD_MMA = 2, KID_DOT = 3, KID_DKDV_MMA = 4, KID_DQ_MMA = 5,
     KID_FWD_TC = 6, KID_BWD_TC = 7, KID_PREP_REPLACED = 8, KID_DQ_CONVERT = 9, KID_BWD_PRE = 10,
-    KID_GROUP_SUM = 11, KID_PATTERN_GRAD = 12
+    KID_GROUP_SUM = 11, KID_PATTERN_GRAD = 12, KID_CALIBRATION = 13
 };
 // Every kernel launch of the library is bracketed by these two calls.
 void launch_begin(int kid, cudaStream_t s);
@@ -168,6 +168,11 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
                           const float* a, const float* r, const float* logz, const HeadList& hl,
                           const ReplacedWs& w, int B, int H, int Hkv, int T, void* dk, void* dv, int grad_fp32,
                           unsigned int* err, cudaStream_t stream);
+// Calibration statistics over N samples (q, k [N, H, T, 64], lse [N, H, T]):
+// A_hat [H, T, T] and s_var [H]; `partial` holds calibration_partial_floats(H, T) floats.
+size_t calibration_partial_floats(int H, int T);
+cudaError_t launch_calibration(const __nv_bfloat16* q, const __nv_bfloat16* k, const float* lse, int N, int H,
+                               int T, float* a_hat, float* svar, float* partial, cudaStream_t stream);
 // Trainable pattern: adds dalpha, drho [H, T] of the replaced heads (zeroed by the caller).
 cudaError_t launch_pattern_grad(const __nv_bfloat16* v, const __nv_bfloat16* dout, const float* a, const float* r,
                                 const float* logz, const HeadList& hl, int B, int H, int T, float* da, float* dr,

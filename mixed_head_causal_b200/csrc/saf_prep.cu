@@ -50,12 +50,22 @@ __global__ void __launch_bounds__(kLnWarps * 32) lognorm_kernel(const float* __r
         // d = i - k this chunk can meet; out-of-range entries are -inf (no term)
         const int dbase = i0 - k0 - (n - 1);
         const int span = n + kLnRows - 1;
-#pragma unroll 4
-        for (int u = threadIdx.x; u < n; u += blockDim.x) sa[u] = ah[k0 + u] * kLog2e;
-#pragma unroll 4
-        for (int q = threadIdx.x; q < span; q += blockDim.x) {
-            const int d = dbase + q;
-            sr[q] = (d >= 0 && d < T) ? rh[d] * kLog2e : kNegInf;
+        // every load of the chunk in flight before the first store (one
+        // round trip to L2 instead of one per pass of the loop)
+        constexpr int kPer = (kLnChunk + kLnRows) / (kLnWarps * 32) + 1;
+        float va[kPer], vr[kPer];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const int u = (int)threadIdx.x + e * kLnWarps * 32;
+            const int d = dbase + u;
+            va[e] = u < n ? ah[k0 + u] : 0.f;
+            vr[e] = (u < span && d >= 0 && d < T) ? rh[d] : kNegInf;
+        }
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const int u = (int)threadIdx.x + e * kLnWarps * 32;
+            if (u < n) sa[u] = va[e] * kLog2e;
+            if (u < span) sr[u] = vr[e] * kLog2e;
         }
         __syncthreads();
         // warp w takes k in [w * per, (w + 1) * per) of the chunk, 8 at a time;

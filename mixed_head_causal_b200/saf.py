@@ -36,6 +36,8 @@ SIGNATURES = {
                                 _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "saf_device_status": ([_vp, _sz, _vp], _i),
     "saf_replaced_pattern_grad": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
+    "saf_calibration_workspace_size": ([_i, _i, _i], _sz),
+    "saf_attn_calibration": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
     "saf_mixed_attn_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                     _vp, _vp, _vp, _i, _vp], _i),
     "saf_launch_count": ([], ctypes.c_uint64),
@@ -225,6 +227,25 @@ def replaced_pattern_grad(v, dout, alpha, rho, mask, logz=None, da=None, dr=None
                                             _ptr(workspace), wsb, _stream_ptr(stream)),
            "saf_replaced_pattern_grad")
     return da, dr
+
+
+def attn_calibration(q, k, lse, a_hat=None, svar=None, workspace=None, stream=None):
+    """Calibration statistics over the N samples of q, k [N,H,T,64] (lse from
+    the forward of the same inputs): (A_hat [H,T,T] fp32, s_var [H] fp32), Eq. (1)."""
+    N, H, T, d = q.shape
+    for n, t in (("q", q), ("k", k)):
+        _check_layer_tensor(n, t, (N, H, T, d))
+    a_hat = torch.empty(H, T, T, dtype=torch.float32, device=q.device) if a_hat is None else a_hat
+    svar = torch.empty(H, dtype=torch.float32, device=q.device) if svar is None else svar
+    if workspace is None:
+        nbytes = load().saf_calibration_workspace_size(H, T, d)
+        if nbytes == ctypes.c_size_t(-1).value:
+            raise SafError(SAF_ERR_INVALID_ARG, "saf_calibration_workspace_size")
+        workspace = torch.empty(max(16, int(nbytes)), dtype=torch.uint8, device=q.device)
+    _check(load().saf_attn_calibration(_ptr(q), _ptr(k), _ptr(lse), N, H, T, d, _ptr(a_hat), _ptr(svar),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream_ptr(stream)), "saf_attn_calibration")
+    return a_hat, svar
 
 
 def mixed_attn_bwd_noalloc(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtype=torch.bfloat16,

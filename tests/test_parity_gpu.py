@@ -288,3 +288,31 @@ def test_pattern_grad_extreme_range_and_explicit_logz():
     da_ref, dr_ref = oracle.pattern_grad(x["v"], x["do"], x["alpha"], x["rho"], x["mask"])
     for got, ref in ((da[1].cpu().double().numpy(), da_ref[1]), (dr[1].cpu().double().numpy(), dr_ref[1])):
         assert np.abs(got - ref).max() <= 2e-4 * max(1.0, np.abs(ref).max())
+
+
+@pytest.mark.parametrize("N,H,T", [(3, 2, 300), (2, 3, 64), (4, 1, 650)], ids=["n3_t300", "n2_t64", "n4_t650"])
+def test_calibration(N, H, T):
+    """Calibration statistics (sample-mean attention, Eq. (1)) against the
+    oracle: every element of A_hat within 1e-4 (probabilities; the kernel's
+    fp32 exps and the forward's lse are good to ~1e-6), s_var within 1e-3
+    relative; A_hat zero above the diagonal."""
+    w = I.custom(N, H, T, [])
+    x = I.make_inputs(w, 41)
+    g = P.to_gpu(x)
+    _, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"])
+    a_hat, svar = saf.attn_calibration(g["q"], g["k"], lse)
+    torch.cuda.synchronize()
+    a_ref, sv_ref = oracle.calibration(x["q"], x["k"])
+    a_hat = a_hat.cpu().double().numpy()
+    assert np.abs(a_hat - a_ref).max() <= 1e-4
+    assert np.all(np.triu(a_hat, 1) == 0)
+    np.testing.assert_allclose(svar.cpu().double().numpy(), sv_ref, rtol=1e-3, atol=0)
+
+
+def test_calibration_needs_two_samples():
+    w = I.custom(1, 2, 64, [])
+    x = I.make_inputs(w, 42)
+    g = P.to_gpu(x)
+    _, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"])
+    with pytest.raises(saf.SafError):
+        saf.attn_calibration(g["q"], g["k"], lse)
