@@ -85,6 +85,8 @@ class Oracle:
         lib.oracle_pattern_grad_slice.restype = i
         lib.oracle_calibration_head.argtypes = [i, i, i, dp, dp, dp, dp]
         lib.oracle_calibration_head.restype = i
+        lib.oracle_fit_pattern.argtypes = [i, dp, i, ctypes.c_double, dp, dp, dp]
+        lib.oracle_fit_pattern.restype = i
         self.lib = lib
 
     def lognorm(self, a, r) -> np.ndarray:
@@ -159,6 +161,17 @@ class Oracle:
         dq, dk, dv = self.bwd_slices(_f64(q).reshape(sh), _f64(k).reshape(sh), _f64(v).reshape(sh),
                                      _f64(dout).reshape(sh), ar, rr, rep, n_threads)
         return dq.reshape(v.shape), dk.reshape(v.shape), dv.reshape(v.shape)
+
+    def fit_pattern(self, target, steps: int = 400, lr: float = 0.1):
+        """Fits (alpha, rho) of one head to a target pattern [T,T] by Adam on
+        the row-wise cross-entropy.  Returns (alpha [T], rho [T], mean row KL)."""
+        t64 = np.ascontiguousarray(_f64(target))
+        T = t64.shape[0]
+        a, r = np.zeros(T), np.zeros(T)
+        kl = ctypes.c_double(0.0)
+        if self.lib.oracle_fit_pattern(T, _p(t64), steps, lr, _p(a), _p(r), ctypes.byref(kl)):
+            raise MemoryError("oracle pattern fit failed")
+        return a, r, kl.value
 
     def calibration(self, q, k):
         """Calibration statistics of every head over the N samples of q, k
@@ -257,6 +270,10 @@ def pattern_grad(v, dout, a, r, mask):
 
 def calibration(q, k):
     return default().calibration(q, k)
+
+
+def fit_pattern(target, steps=400, lr=0.1):
+    return default().fit_pattern(target, steps, lr)
 
 
 def fwd_gqa(q, k, v, a, r, mask, n_threads=None):

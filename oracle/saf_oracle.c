@@ -36,6 +36,18 @@
  *    matrix, A_hat = (1/N) sum_n A^(n), and its reconstruction error
  *    s_var = sum_n ||A^(n) - A_hat||_F^2 / ((N - 1) T^2)   (Eq. (1)).
  *
+ *  - Pattern fitting (section 二.3 and Appendix A.2 as summarised there): a
+ *    replaced head's (alpha, rho) minimise the row-wise cross-entropy to a
+ *    target pattern A (e.g. the calibration mean),
+ *      L = -(1/T) sum_i sum_{j<=i} A(i,j) log P(i,j),
+ *    which depends on A only through its column sums m[j] = sum_i A(i,j)
+ *    and distance sums n[d] = sum_i A(i,i-d) (the sufficient statistics of
+ *    Eq. (4)): L = -(1/T) (sum_j alpha_j m_j + sum_d rho_d n_d - sum_i log Z(i))
+ *    for a target with unit row sums.  Its gradient is
+ *      dL/dalpha_j = -(m_j - sum_i P(i,j)) / T,  dL/drho_d = -(n_d - sum_i P(i,i-d)) / T,
+ *    minimised by Adam (beta1 0.9, beta2 0.999, eps 1e-8, bias-corrected)
+ *    from alpha = rho = 0; the mean row KL(A || P) = L + (1/T) sum A log A.
+ *
  * Max-shifts (subtracting the row maximum before exp) are the only numerical
  * device used; they leave every result unchanged mathematically.  A row
  * whose every term is -inf (possible only with -inf alpha/rho) yields an all
@@ -113,6 +125,64 @@ static void fwd_ordinary(int T, int d, const double *q, const double *k,
         }
         lse[i] = m + log(l);
     }
+}
+
+/* -------------------------------------------------------- pattern fitting */
+
+/*
+ * Fits one head: target a_t [T,T] (row-stochastic, causal), `steps` Adam
+ * steps of learning rate lr.  Writes alpha, rho [T] and returns the mean row
+ * KL(A || P) of the result through *kl.  Returns 0, or -1 on allocation
+ * failure.
+ */
+int oracle_fit_pattern(int T, const double *a_t, int steps, double lr, double *alpha, double *rho, double *kl)
+{
+    const size_t n = (size_t)(T > 0 ? T : 1);
+    double *m = calloc(n, sizeof(double)), *nd = calloc(n, sizeof(double));
+    double *logz = malloc(sizeof(double) * n), *cs = malloc(sizeof(double) * n), *ds = malloc(sizeof(double) * n);
+    double *m1 = calloc(2 * n, sizeof(double)), *m2 = calloc(2 * n, sizeof(double));
+    if (!m || !nd || !logz || !cs || !ds || !m1 || !m2) {
+        free(m); free(nd); free(logz); free(cs); free(ds); free(m1); free(m2);
+        return -1;
+    }
+    double ent = 0.0;  /* sum A log A */
+    for (int i = 0; i < T; ++i)
+        for (int j = 0; j <= i; ++j) {
+            const double x = a_t[(size_t)i * T + j];
+            m[j] += x;
+            nd[i - j] += x;
+            if (x > 0.0) ent += x * log(x);
+        }
+    for (int j = 0; j < T; ++j) alpha[j] = rho[j] = 0.0;
+    const double b1 = 0.9, b2 = 0.999, eps = 1e-8;
+    double p1 = 1.0, p2 = 1.0;
+    for (int it = 0; it < steps; ++it) {
+        oracle_lognorm(T, alpha, rho, logz);
+        for (int j = 0; j < T; ++j) cs[j] = ds[j] = 0.0;
+        for (int i = 0; i < T; ++i)
+            for (int j = 0; j <= i; ++j) {
+                const double p = exp(alpha[j] + rho[i - j] - logz[i]);
+                cs[j] += p;
+                ds[i - j] += p;
+            }
+        p1 *= b1;
+        p2 *= b2;
+        for (int e = 0; e < 2 * T; ++e) {
+            const double g = e < T ? -(m[e] - cs[e]) / T : -(nd[e - T] - ds[e - T]) / T;
+            m1[e] = b1 * m1[e] + (1.0 - b1) * g;
+            m2[e] = b2 * m2[e] + (1.0 - b2) * g * g;
+            const double step = lr * (m1[e] / (1.0 - p1)) / (sqrt(m2[e] / (1.0 - p2)) + eps);
+            if (e < T) alpha[e] -= step;
+            else rho[e - T] -= step;
+        }
+    }
+    oracle_lognorm(T, alpha, rho, logz);
+    double loss = 0.0;
+    for (int j = 0; j < T; ++j) loss += alpha[j] * m[j] + rho[j] * nd[j];
+    for (int i = 0; i < T; ++i) loss -= logz[i];
+    *kl = (-loss + ent) / T;
+    free(m); free(nd); free(logz); free(cs); free(ds); free(m1); free(m2);
+    return 0;
 }
 
 /* ------------------------------------------------------------ calibration */

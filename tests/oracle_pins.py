@@ -466,6 +466,44 @@ def check_calibration_mean_is_linear(orc):
     np.testing.assert_allclose(sv2, sv, rtol=1e-13, atol=0)
 
 
+def _pattern_of(orc, a, r):
+    return _pattern_matrix(orc, np.asarray(a, dtype=np.float64), np.asarray(r, dtype=np.float64))[0]
+
+
+def check_fit_recovers_a_pattern(orc):
+    """A target that is itself a compact pattern (Eq. (3)) is fitted back: the
+    fitted pattern equals it (a and r up to their shift freedom) and the KL is
+    zero."""
+    rng = _rng(20)
+    T = 40
+    a, r = _pattern(T, rng)
+    target = _pattern_of(orc, a, r)
+    fa, fr, kl = orc.fit_pattern(target, 400, 0.1)
+    np.testing.assert_allclose(_pattern_of(orc, fa, fr), target, rtol=0, atol=1e-6)
+    assert abs(kl) < 1e-9
+
+
+def check_fit_matches_moments_and_kl(orc):
+    """A target outside the family (a random row-stochastic causal matrix):
+    at the optimum of the cross-entropy the fitted pattern's column sums and
+    distance sums equal the target's (the sufficient statistics of Eq. (4));
+    the returned KL equals the mean row KL computed directly."""
+    rng = _rng(21)
+    T = 24
+    logits = rng.normal(size=(T, T)) * 1.5
+    logits[np.triu_indices(T, 1)] = NEG_INF
+    target = np.exp(logits - logsumexp(logits, axis=1)[:, None])
+    fa, fr, kl = orc.fit_pattern(target, 3000, 0.01)
+    P = _pattern_of(orc, fa, fr)
+    np.testing.assert_allclose(P.sum(axis=0), target.sum(axis=0), rtol=0, atol=2e-4)
+    diag = lambda M: np.array([np.trace(M, offset=-d) for d in range(T)])  # noqa: E731
+    np.testing.assert_allclose(diag(P), diag(target), rtol=0, atol=2e-4)
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    direct = np.sum(target[mask] * (np.log(target[mask]) - np.log(P[mask]))) / T
+    np.testing.assert_allclose(kl, direct, rtol=0, atol=1e-10)
+    assert kl > 0.05  # the random target is far from the family
+
+
 def check_all_masked_row(orc):
     """Every logit -inf (a = -inf): output 0 and lse = -inf, no NaN."""
     T, d = 5, 4
@@ -499,5 +537,7 @@ ALL_CHECKS = [
     check_pattern_grad_sums_vanish,
     check_calibration_closed_forms,
     check_calibration_mean_is_linear,
+    check_fit_recovers_a_pattern,
+    check_fit_matches_moments_and_kl,
     check_all_masked_row,
 ]

@@ -74,6 +74,13 @@ MUTANTS = [
     ("calibration: scores not scaled",
      "srow[j] = scale * dot;\n                if (srow[j] > m) m = srow[j];\n            }\n            double l = 0.0;\n            for (int j = 0; j <= i; ++j) l += exp(srow[j] - m);\n            for (int j = 0; j < T; ++j) an",
      "srow[j] = dot;\n                if (srow[j] > m) m = srow[j];\n            }\n            double l = 0.0;\n            for (int j = 0; j <= i; ++j) l += exp(srow[j] - m);\n            for (int j = 0; j < T; ++j) an", 0),
+    ("fit: distance statistic of the key",
+     "nd[i - j] += x;", "nd[j] += x;", 0),
+    ("fit: gradient sign flipped",
+     "const double g = e < T ? -(m[e] - cs[e]) / T : -(nd[e - T] - ds[e - T]) / T;",
+     "const double g = e < T ? (m[e] - cs[e]) / T : (nd[e - T] - ds[e - T]) / T;", 0),
+    ("fit: KL without the entropy term",
+     "*kl = (-loss + ent) / T;", "*kl = -loss / T;", 0),
     ("replaced bwd: dQ not cleared",
      "memset(dq, 0, sizeof(double) * (size_t)T * d);\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz",
      "for (int c = 0; c < T * d; ++c) dq[c] = 1e-3 * c;\n    memset(dk, 0, sizeof(double) * (size_t)T * d);\n    memset(dv, 0, sizeof(double) * (size_t)T * d);\n    for (int i = 0; i < T; ++i) {\n        if (logz", 0),
