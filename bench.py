@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--calibration", action="store_true",
                     help="instead of the headline line, time the calibration statistics (A_hat, s_var) over "
                          "the workload's batch as N samples, every head ordinary")
+    ap.add_argument("--fit", action="store_true",
+                    help="instead of the headline line, time the fitting of (a, r) (400 Adam steps) to the "
+                         "patterns of the workload's replaced heads")
     ap.add_argument("--gqa", type=int, default=0, metavar="H_KV",
                     help="instead of the headline line, time fwd and bwd with K/V shared by groups of "
                          "H / H_KV query heads")
@@ -550,6 +553,39 @@ def calibration_cost(args, local):
                                    "a_hat_bytes": 4 * w.H * w.T * w.T}}), flush=True)
 
 
+def fit_cost(args, local):
+    """Pattern fitting (400 Adam steps) of the workload's replaced heads, the
+    targets being their own patterns (dense [T, T] fp32, built on the GPU from
+    the pattern vectors by the forward with V = I in 128-row slabs)."""
+    from mixed_head_causal_b200 import saf
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS[args.workload]
+    a, r = I.make_pattern(w, 0)
+    heads = I.replaced_heads(w)
+    T = w.T
+    lz = saf.replaced_lognorm(a.to(dev), r.to(dev), I.replaced_mask(w, 0))
+    targets = torch.zeros(len(heads), T, T, dtype=torch.float32, device=dev)
+    i = torch.arange(T, device=dev)[:, None]
+    j = torch.arange(T, device=dev)[None, :]
+    for s_, h in enumerate(heads):
+        ah, rh = a[h].to(dev), r[h].to(dev)
+        for i0 in range(0, T, 512):
+            ii = i[i0:i0 + 512]
+            logit = ah[j.expand(ii.shape[0], T)] + rh[(ii - j).clamp(min=0)] - lz[h][ii]
+            targets[s_, i0:i0 + 512] = torch.where(j <= ii, torch.exp(logit), torch.zeros((), device=dev))
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    _, _, kl = saf.fit_pattern(targets, steps=400, lr=0.1)
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"metric": "pattern fitting, 400 Adam steps, ms per call", "value": e0.elapsed_time(e1),
+                      "unit": "ms", "higher_is_better": False,
+                      "config": {"workload": w.name, "heads": len(heads), "T": T},
+                      "kl": [float(x) for x in kl.cpu()], "wall_s": time.perf_counter() - t0}), flush=True)
+
+
 def gqa_cost(args, local):
     """Forward and backward with K/V shared by groups of H / H_kv query heads
     (the workload's shape and head mix): ms and tokens/s per pass."""
@@ -596,6 +632,9 @@ def main():
         elif args.calibration:
             if rank == 0:
                 calibration_cost(args, local)
+        elif args.fit:
+            if rank == 0:
+                fit_cost(args, local)
         elif args.impl == "reference":
             reference_arm(args, world, rank)
         else:

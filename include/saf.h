@@ -219,6 +219,27 @@ SAF_API saf_status saf_replaced_pattern_grad(const void *v, const void *dout,
                                              void *stream);
 
 /*
+ * Pattern fitting (section 二.3 of the reading notes for "When Can Attention
+ * Heads Be Statically Defined?", with Appendix A.2 as summarised there): for
+ * each of n_heads target patterns (e.g. a_hat rows of saf_attn_calibration),
+ * the a, r of Eq. (3) minimising the row-wise cross-entropy
+ *   L = -(1/T) sum_i sum_{j<=i} A(i,j) log P(i,j),
+ * which sees the target only through its column sums and distance sums
+ * (Eq. (4)), by `steps` bias-corrected Adam steps (beta1 0.9, beta2 0.999,
+ * eps 1e-8, learning rate lr) from a = r = 0; the pages use 400 steps and
+ * accept a head at a mean row KL of at most 0.2 nat.
+ *   target  [n_heads,T,T] fp32 in: causal, rows summing to 1.
+ *   a, r    [n_heads,T] fp32 out;  kl [n_heads] fp32 out: mean row KL(A || P).
+ *   workspace: at least saf_fit_workspace_size(n_heads,T) bytes, 256-byte aligned.
+ * n_heads <= 256 and T <= 16384 (SAF_ERR_UNSUPPORTED otherwise).  One Adam
+ * step is three kernel launches.
+ */
+SAF_API size_t saf_fit_workspace_size(int n_heads, int T);
+SAF_API saf_status saf_fit_pattern(const float *target, int n_heads, int T, int steps, float lr,
+                                   float *a, float *r, float *kl,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Calibration statistics (section 二.1 of the reading notes for "When Can
  * Attention Heads Be Statically Defined?"): over N >= 2 calibration sequences
  * run through plain causal softmax attention (every head ordinary), the

@@ -13,6 +13,8 @@ using namespace saf;
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
+// the fitting kernels stage a, r and log Z of a head in shared memory (3 T floats)
+constexpr int kFitMaxT = 16384;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
@@ -234,6 +236,23 @@ saf_status saf_mixed_attn_bwd(const void* q, const void* k, const void* v, const
                               void* workspace, size_t workspace_bytes, void* stream) {
     return saf_mixed_attn_bwd_gqa(q, k, v, o, dout, lse, a, r, logz, replaced_mask, B, H, H, T, d_h, dq, dk, dv,
                                   grad_dtype, workspace, workspace_bytes, stream);
+}
+
+size_t saf_fit_workspace_size(int n_heads, int T) {
+    if (n_heads < 0 || n_heads > kMaxHeads || T < 0 || T > kFitMaxT) return (size_t)-1;
+    return fit_workspace_bytes(n_heads, T);
+}
+
+saf_status saf_fit_pattern(const float* target, int n_heads, int T, int steps, float lr, float* a, float* r,
+                           float* kl, void* workspace, size_t workspace_bytes, void* stream) {
+    if (n_heads < 0 || T < 0 || steps < 0 || !(lr > 0.f)) return SAF_ERR_INVALID_ARG;
+    if (n_heads > kMaxHeads || T > kFitMaxT) return SAF_ERR_UNSUPPORTED;
+    if ((int64_t)n_heads * T == 0) return SAF_OK;
+    if (!target || !a || !r || !kl) return SAF_ERR_INVALID_ARG;
+    if (!aligned16(target) || !aligned16(a) || !aligned16(r) || !aligned16(kl)) return SAF_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < fit_workspace_bytes(n_heads, T)) return SAF_ERR_WORKSPACE;
+    if (!aligned256(workspace)) return SAF_ERR_INVALID_ARG;
+    return cuda_status(launch_fit(target, n_heads, T, steps, lr, a, r, kl, workspace, (cudaStream_t)stream));
 }
 
 size_t saf_calibration_workspace_size(int H, int T, int d_h) {

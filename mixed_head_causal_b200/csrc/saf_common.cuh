@@ -135,7 +135,7 @@ int sm_count();
 enum KernelId {
     KID_LOGNORM = 1, KID_FWD_MMA = 2, KID_DOT = 3, KID_DKDV_MMA = 4, KID_DQ_MMA = 5,
     KID_FWD_TC = 6, KID_BWD_TC = 7, KID_PREP_REPLACED = 8, KID_DQ_CONVERT = 9, KID_BWD_PRE = 10,
-    KID_GROUP_SUM = 11, KID_PATTERN_GRAD = 12, KID_CALIBRATION = 13
+    KID_GROUP_SUM = 11, KID_PATTERN_GRAD = 12, KID_CALIBRATION = 13, KID_FIT = 14
 };
 // Every kernel launch of the library is bracketed by these two calls.
 void launch_begin(int kid, cudaStream_t s);
@@ -168,6 +168,11 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
                           const float* a, const float* r, const float* logz, const HeadList& hl,
                           const ReplacedWs& w, int B, int H, int Hkv, int T, void* dk, void* dv, int grad_fp32,
                           unsigned int* err, cudaStream_t stream);
+// Pattern fitting of nslots targets [nslots, T, T]: alpha, rho [nslots, T], kl [nslots];
+// `ws` holds fit_workspace_bytes(nslots, T) bytes (256-byte aligned).
+size_t fit_workspace_bytes(int nslots, int T);
+cudaError_t launch_fit(const float* target, int nslots, int T, int steps, float lr, float* alpha, float* rho,
+                       float* kl, void* ws, cudaStream_t stream);
 // Calibration statistics over N samples (q, k [N, H, T, 64], lse [N, H, T]):
 // A_hat [H, T, T] and s_var [H]; `partial` holds calibration_partial_floats(H, T) floats.
 size_t calibration_partial_floats(int H, int T);

@@ -23,7 +23,7 @@ struct Profile {
 } g_prof;
 
 const char* kNames[] = {"?", "lognorm", "fwd_mma", "dot", "dkdv_mma", "dq_mma",
-                        "fwd_tc", "bwd_tc", "prep_replaced", "dq_convert", "bwd_pre", "group_sum", "pattern_grad", "calibration"};
+                        "fwd_tc", "bwd_tc", "prep_replaced", "dq_convert", "bwd_pre", "group_sum", "pattern_grad", "calibration", "fit"};
 
 void release_locked() {
     for (auto& r : g_prof.recs) {

@@ -37,6 +37,8 @@ SIGNATURES = {
     "saf_device_status": ([_vp, _sz, _vp], _i),
     "saf_replaced_pattern_grad": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
     "saf_calibration_workspace_size": ([_i, _i, _i], _sz),
+    "saf_fit_workspace_size": ([_i, _i], _sz),
+    "saf_fit_pattern": ([_vp, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp], _i),
     "saf_attn_calibration": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
     "saf_mixed_attn_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                     _vp, _vp, _vp, _i, _vp], _i),
@@ -227,6 +229,26 @@ def replaced_pattern_grad(v, dout, alpha, rho, mask, logz=None, da=None, dr=None
                                             _ptr(workspace), wsb, _stream_ptr(stream)),
            "saf_replaced_pattern_grad")
     return da, dr
+
+
+def fit_pattern(target, steps: int = 400, lr: float = 0.1, stream=None):
+    """Fits a, r of Eq. (3) to target patterns [n, T, T] (fp32, causal, unit
+    row sums).  Returns (a [n, T], r [n, T], mean row KL [n])."""
+    if target.dim() == 2:
+        target = target[None]
+    n, T, T2 = target.shape
+    if T != T2 or target.dtype != torch.float32 or not target.is_cuda or not target.is_contiguous():
+        raise ValueError("target: expected a contiguous CUDA fp32 [n, T, T] tensor")
+    a = torch.empty(n, T, dtype=torch.float32, device=target.device)
+    r = torch.empty_like(a)
+    kl = torch.empty(n, dtype=torch.float32, device=target.device)
+    nbytes = load().saf_fit_workspace_size(n, T)
+    if nbytes == ctypes.c_size_t(-1).value:
+        raise SafError(SAF_ERR_INVALID_ARG, "saf_fit_workspace_size")
+    ws = torch.zeros(max(256, int(nbytes)), dtype=torch.uint8, device=target.device)
+    _check(load().saf_fit_pattern(_ptr(target), n, T, steps, lr, _ptr(a), _ptr(r), _ptr(kl), _ptr(ws),
+                                  ws.numel(), _stream_ptr(stream)), "saf_fit_pattern")
+    return a, r, kl
 
 
 def attn_calibration(q, k, lse, a_hat=None, svar=None, workspace=None, stream=None):

@@ -316,3 +316,54 @@ def test_calibration_needs_two_samples():
     _, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"])
     with pytest.raises(saf.SafError):
         saf.attn_calibration(g["q"], g["k"], lse)
+
+
+def _oracle_pattern(a, r):
+    """P of Eq. (3) for one head, read off the oracle's forward with V = I."""
+    T = a.shape[0]
+    z = np.zeros((1, T, T))
+    p, _ = oracle.fwd_slices(z, z, np.eye(T)[None], np.asarray(a, np.float64)[None], np.asarray(r, np.float64)[None],
+                             [1])
+    return p[0]
+
+
+def test_fit_recovers_compact_targets():
+    """Targets that are compact patterns themselves are fitted back (fp32 Adam,
+    400 steps): the fitted pattern matches the target and the KL is ~0."""
+    T = 200
+    gen = torch.Generator().manual_seed(51)
+    targets = []
+    for h in range(2):
+        a = torch.randn(T, generator=gen) * 0.5
+        a[0] += 3.0
+        r = -0.05 * (h + 1) * torch.arange(T, dtype=torch.float32) + torch.randn(T, generator=gen) * 0.3
+        r[0] += 1.0
+        targets.append(_oracle_pattern(a.double().numpy(), r.double().numpy()))
+    tg = torch.tensor(np.stack(targets), dtype=torch.float32, device="cuda")
+    fa, fr, kl = saf.fit_pattern(tg, steps=400, lr=0.1)
+    torch.cuda.synchronize()
+    for h in range(2):
+        P = _oracle_pattern(fa[h].cpu().double().numpy(), fr[h].cpu().double().numpy())
+        assert np.abs(P - targets[h]).max() <= 2e-3
+        assert abs(float(kl[h])) <= 1e-3
+
+
+def test_fit_matches_the_oracle_on_a_calibration_target():
+    """A calibration-mean target (the mean of 4 causal softmax matrices): the
+    GPU fit and the oracle's fp64 fit (same Adam schedule) reach the same KL
+    and the same pattern."""
+    N, T = 4, 96
+    gen = torch.Generator().manual_seed(52)
+    q = torch.randn(N, 1, T, 64, generator=gen)
+    k = torch.randn(N, 1, T, 64, generator=gen)
+    a_hat, _ = oracle.calibration(q, k)
+    target = a_hat[0]
+    fa, fr, kl = saf.fit_pattern(torch.tensor(target, dtype=torch.float32, device="cuda")[None], steps=400, lr=0.1)
+    torch.cuda.synchronize()
+    oa, orr, okl = oracle.fit_pattern(target, 400, 0.1)
+    assert abs(float(kl[0]) - okl) <= 2e-3
+    P = _oracle_pattern(fa[0].cpu().double().numpy(), fr[0].cpu().double().numpy())
+    assert np.abs(P - _oracle_pattern(oa, orr)).max() <= 1e-2
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    direct = np.sum(target[mask] * (np.log(target[mask]) - np.log(P[mask]))) / T
+    assert abs(float(kl[0]) - direct) <= 2e-3
