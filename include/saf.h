@@ -271,6 +271,17 @@ SAF_API saf_status saf_attn_calibration(const void *q, const void *k, const floa
  */
 SAF_API saf_status saf_device_status(void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Failure-path self-test (the pages have no counterpart): enqueues a kernel
+ * whose single wait, on an mbarrier that nothing completes, gives up after
+ * limit_cycles SM cycles (1 .. 2^31) and records the time-out in the
+ * workspace's error word, exactly as a kernel wait that timed out would; no
+ * copy or MMA is in flight, so the device stays usable.  A following
+ * saf_device_status returns SAF_ERR_TIMEOUT (and clears the word).
+ */
+SAF_API saf_status saf_selftest_wait_timeout(void *workspace, size_t workspace_bytes, long long limit_cycles,
+                                             void *stream);
+
 /* ------------------------------------------------------------------------
  * Launch accounting and per-kernel timing (for benchmarks and tracing).
  * ------------------------------------------------------------------------ */

@@ -310,6 +310,14 @@ saf_status saf_replaced_pattern_grad(const void* v, const void* dout, const floa
                                            s));
 }
 
+saf_status saf_selftest_wait_timeout(void* workspace, size_t workspace_bytes, long long limit_cycles,
+                                     void* stream) {
+    if (!workspace || workspace_bytes < sizeof(WsHeader)) return SAF_ERR_WORKSPACE;
+    if (!aligned256(workspace) || limit_cycles < 1 || limit_cycles > (1ll << 31)) return SAF_ERR_INVALID_ARG;
+    return cuda_status(launch_selftest_wait(static_cast<unsigned int*>(workspace), limit_cycles,
+                                            (cudaStream_t)stream));
+}
+
 saf_status saf_device_status(void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace || workspace_bytes < sizeof(WsHeader)) return SAF_ERR_WORKSPACE;
     WsHeader hdr;

@@ -168,6 +168,8 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
                           const float* a, const float* r, const float* logz, const HeadList& hl,
                           const ReplacedWs& w, int B, int H, int Hkv, int T, void* dk, void* dv, int grad_fp32,
                           unsigned int* err, cudaStream_t stream);
+// Failure-path self-test: a bounded wait on an mbarrier nobody completes.
+cudaError_t launch_selftest_wait(unsigned int* err, long long limit, cudaStream_t stream);
 // Pattern fitting of nslots targets [nslots, T, T]: alpha, rho [nslots, T], kl [nslots];
 // `ws` holds fit_workspace_bytes(nslots, T) bytes (256-byte aligned).
 size_t fit_workspace_bytes(int nslots, int T);

@@ -35,6 +35,7 @@ SIGNATURES = {
     "saf_mixed_attn_bwd_gqa": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                 _vp, _vp, _vp, _i, _vp, _sz, _vp], _i),
     "saf_device_status": ([_vp, _sz, _vp], _i),
+    "saf_selftest_wait_timeout": ([_vp, _sz, ctypes.c_longlong, _vp], _i),
     "saf_replaced_pattern_grad": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
     "saf_calibration_workspace_size": ([_i, _i, _i], _sz),
     "saf_fit_workspace_size": ([_i, _i], _sz),
@@ -296,6 +297,13 @@ def device_status(workspace: torch.Tensor, stream=None) -> int:
     """Reads and clears the device error word of `workspace` (synchronous)."""
     return int(load().saf_device_status(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                         _stream_ptr(stream)))
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, limit_cycles: int = 1 << 20, stream=None) -> None:
+    """Enqueues a bounded device wait that nothing completes (it sets the
+    workspace's error word when it gives up; see device_status)."""
+    _check(load().saf_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                            int(limit_cycles), _stream_ptr(stream)), "saf_selftest_wait_timeout")
 
 
 def launch_count() -> int:

@@ -128,3 +128,10 @@ def test_device_status_argument_errors(lib):
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="no fallback"):
         saf.load(str(tmp_path / "missing.so"))
+
+
+def test_selftest_argument_errors(lib):
+    assert lib.saf_selftest_wait_timeout(None, 256, 1000, None) == saf.SAF_ERR_WORKSPACE
+    assert lib.saf_selftest_wait_timeout(FAKE, 16, 1000, None) == saf.SAF_ERR_WORKSPACE
+    assert lib.saf_selftest_wait_timeout(FAKE, 256, 0, None) == saf.SAF_ERR_INVALID_ARG
+    assert lib.saf_selftest_wait_timeout(FAKE, 256, 1 << 40, None) == saf.SAF_ERR_INVALID_ARG

@@ -62,10 +62,14 @@ def test_several_tiles_full(path):
 
 
 def _special(T, a_fn, r_fn):
+    """Head 1 of a (1, 2, T) layer replaced with pattern vectors a_fn(T),
+    r_fn(T); their draws are seeded by T (the global generator is restored)."""
     w = I.custom(1, 2, T, [1])
     x = I.make_inputs(w, 7)
-    x["alpha"][1] = a_fn(T)
-    x["rho"][1] = r_fn(T)
+    with torch.random.fork_rng(devices=[]):
+        torch.manual_seed(1000 + T)
+        x["alpha"][1] = a_fn(T)
+        x["rho"][1] = r_fn(T)
     return w, x
 
 
@@ -277,17 +281,55 @@ def test_pattern_grad(B, H, T, replaced):
             assert np.abs(got - ref).max() <= 2e-4 * scale, (h, np.abs(got - ref).max(), scale)
 
 
+def _pattern_grad_noise(x, h):
+    """Expected fp32 rounding noise of dalpha, drho of head h.
+
+    The kernel's log P(i,j) = a[j] + r[i-j] - log Z(i) carries an error of
+    about one unit of fp32 rounding of the largest logit magnitude L (log Z(i)
+    is itself an fp32 number of that size), shared by a row and by every
+    batch.  A relative error eps_i of row i moves dS(i,j) by eps_i (dS(i,j) -
+    P(i,j) D(i)), so dalpha[j] and drho[d] collect sums of such terms of
+    random sign: noise = 2^-23 L sqrt(sum_i (sum_b |dS| + P |D|)^2) over the
+    entries (i, j) that reach the output."""
+    a = x["alpha"][h].double().numpy()
+    r = x["rho"][h].double().numpy()
+    T = a.shape[0]
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    causal = j <= i
+    logit = np.where(causal, a[None, :] + r[np.clip(i - j, 0, T - 1)], -np.inf)
+    top = logit.max(1, keepdims=True)
+    lz = top + np.log(np.exp(logit - top).sum(1, keepdims=True))
+    p = np.exp(logit - lz)
+    wsum = np.zeros((T, T))
+    for b in range(x["v"].shape[0]):
+        dp = x["do"][b, h].double().numpy() @ x["v"][b, h].double().numpy().T
+        dvec = (p * dp).sum(1, keepdims=True)
+        wsum += np.abs(p * (dp - dvec)) + p * np.abs(dvec)
+    big = max(np.abs(a).max(), np.abs(r[np.isfinite(r)]).max(), np.abs(lz).max())
+    delta = 2.0 ** -23 * (big + 1.0)
+    w2 = wsum ** 2
+    noise_a = delta * np.sqrt(w2.sum(0))
+    noise_r = delta * np.sqrt(np.array([np.trace(w2, -d) for d in range(T)]))
+    return noise_a, noise_r
+
+
 def test_pattern_grad_extreme_range_and_explicit_logz():
-    """Pattern vectors far beyond the factored form's range (per-element exps
-    in every path) and a log Z passed in: same results as the oracle."""
+    """Pattern vectors far beyond the factored form's range (logits of size
+    ~150) and a log Z passed in: dalpha, drho against the oracle within 2e-4
+    of the largest entry plus four times the expected fp32 noise of logits
+    that large (_pattern_grad_noise)."""
     w, x = _special(500, lambda T: torch.randn(T) * 40.0, lambda T: -0.05 * torch.arange(T, dtype=torch.float32))
     g = P.to_gpu(x)
     lz = saf.replaced_lognorm(g["alpha"], g["rho"], x["mask"])
     da, dr = saf.replaced_pattern_grad(g["v"], g["do"], g["alpha"], g["rho"], x["mask"], logz=lz)
     torch.cuda.synchronize()
     da_ref, dr_ref = oracle.pattern_grad(x["v"], x["do"], x["alpha"], x["rho"], x["mask"])
-    for got, ref in ((da[1].cpu().double().numpy(), da_ref[1]), (dr[1].cpu().double().numpy(), dr_ref[1])):
-        assert np.abs(got - ref).max() <= 2e-4 * max(1.0, np.abs(ref).max())
+    noise_a, noise_r = _pattern_grad_noise(x, 1)
+    for got, ref, noise in ((da[1].cpu().double().numpy(), da_ref[1], noise_a),
+                            (dr[1].cpu().double().numpy(), dr_ref[1], noise_r)):
+        tol = 2e-4 * max(1.0, np.abs(ref).max()) + 4.0 * noise
+        assert np.all(np.abs(got - ref) <= tol), (np.abs(got - ref).max(), tol.max())
 
 
 @pytest.mark.parametrize("N,H,T", [(3, 2, 300), (2, 3, 64), (4, 1, 650)], ids=["n3_t300", "n2_t64", "n4_t650"])
@@ -367,3 +409,38 @@ def test_fit_matches_the_oracle_on_a_calibration_target():
     mask = np.tril(np.ones((T, T), dtype=bool))
     direct = np.sum(target[mask] * (np.log(target[mask]) - np.log(P[mask]))) / T
     assert abs(float(kl[0]) - direct) <= 2e-3
+
+
+def test_device_wait_timeout_is_reported_and_cleared():
+    """A bounded device wait that nothing completes (no copy or MMA in flight)
+    sets the workspace error word; saf_device_status reports the time-out once
+    and clears it, and the layer still runs on the same context."""
+    w = I.custom(1, 2, 200, [1])
+    x = I.make_inputs(w, 61)
+    g = P.to_gpu(x)
+    ws = saf.new_workspace(w.B, w.H, w.T, "cuda")
+    saf.selftest_wait_timeout(ws, 1 << 20)
+    assert saf.device_status(ws) == saf.SAF_ERR_TIMEOUT
+    assert saf.device_status(ws) == saf.SAF_OK
+    o, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"], workspace=ws)
+    assert saf.device_status(ws) == saf.SAF_OK
+    P.check_slices(w, x, {"o": o.cpu(), "lse": lse.cpu()}, _all_slices(w))
+
+
+def test_persistent_forward_leaves_its_counters_zero():
+    """The persistent forward's work counters in the workspace header are zero
+    after each call (the last CTA resets them), so the workspace can be reused
+    and calls repeat exactly."""
+    w = I.custom(2, 3, 520, [0])
+    x = I.make_inputs(w, 62)
+    g = P.to_gpu(x)
+    ws = saf.new_workspace(w.B, w.H, w.T, "cuda")
+    outs = []
+    for _ in range(3):
+        o, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"], workspace=ws)
+        torch.cuda.synchronize()
+        header = ws[:64].view(torch.int32).cpu()
+        assert int(header[2]) == 0 and int(header[3]) == 0
+        outs.append((o.clone(), lse.clone()))
+    for o, lse in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1])
