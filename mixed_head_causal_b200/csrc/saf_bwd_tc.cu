@@ -1,12 +1,16 @@
 // Mixed-head causal attention backward on the 5th-generation tensor cores.
 //
-// One CTA owns one 128-key block J of one (batch, head) slice and walks the
+// A work item is one 128-key block J of one (batch, head) slice; it walks the
 // query blocks I >= J (causal tile skipping; the diagonal block is masked).
 // dK and dV accumulate in TMEM for the whole walk; each tile's dQ
 // contribution is reduced into an fp32 accumulator in global memory with a
-// TMA reduce-add.  Warp roles:
-//   warp 0      TMA producer: K, V once; Q, dO and the per-query vectors of
-//               each query block through an NQS-stage ring
+// TMA reduce-add.  The kernel is persistent: one CTA per SM pulls items,
+// longest first, from a counter in the workspace header (reset by the last
+// CTA), so K/V of the next item load while this one runs and the next item's
+// first MMAs overlap this one's dK/dV read-out.  Warp roles:
+//   warp 0      TMA producer: work items; K (two stages), V per item; Q, dO
+//               and the per-query vectors of each query block through an
+//               NQS-stage ring that runs on across items
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2..9  key rows, two warps per row quarter (query columns 0..63 and
 //               64..127 of each tile): P^T, dS^T, and the dK/dV epilogue
@@ -42,18 +46,20 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ0 = 384, C_DQ1 = 448;
 constexpr long long kWaitLimit = 1ll << 31;
 
+// K in two stages (its last reader, dQ = dS K, closes an item); V in one,
+// free once the item's last dP^T MMA is done, about a tile before the item ends
 constexpr uint32_t SM_K = 0;
-constexpr uint32_t SM_V = SM_K + TILE;
+constexpr uint32_t SM_V = SM_K + 2 * TILE;
 // Q/dO ring depth: a TMA round trip from L2 takes several tiles' worth of
 // MMA time, so the ring keeps NQS query blocks in flight
 constexpr int NQS = 3;
 constexpr uint32_t SM_Q = SM_V + TILE;          // NQS stages
 constexpr uint32_t SM_DO = SM_Q + NQS * TILE;   // NQS stages
 constexpr uint32_t SM_DS = SM_DO + NQS * TILE;  // 32 KB: dS^T as two 64-query atoms
-// dQ staging, 32 KB: two [128][32] fp32 boxes (columns 0..31 and 32..63)
-// with the 128-byte swizzle of the reduce map
+// dQ staging, 32 KB: per dQ warp two [32][32] fp32 boxes (its 32 query rows,
+// columns 0..31 and 32..63) with the 128-byte swizzle of the reduce map
 constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;
-constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;     // NQS x 512 B: -lse2 (ordinary) / r (replaced)
+constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;        // NQS x 512 B: -lse2 (ordinary) / r (replaced)
 constexpr uint32_t SM_VEC2 = SM_VEC1 + 512 * NQS;  // NQS x 512 B: D
 constexpr uint32_t SM_BAR = SM_VEC2 + 512 * NQS;
 constexpr uint32_t SM_TOTAL = SM_BAR + 256;
@@ -172,56 +178,55 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_addr(smem);
-    const uint32_t bar_kv = sb + SM_BAR;
-    const uint32_t bar_qf = bar_kv + 8;         // [NQS]
+    const uint32_t bar_itf = sb + SM_BAR;       // [2] work item slot full
+    const uint32_t bar_ite = bar_itf + 16;      // [2] work item slot read (13 warp arrivals)
+    const uint32_t bar_kf = bar_ite + 16;       // [2] K stage full
+    const uint32_t bar_ke = bar_kf + 16;        // [2] K stage free (the MMAs of its item done)
+    const uint32_t bar_vf = bar_ke + 16;        // V full
+    const uint32_t bar_ve = bar_vf + 8;         // V free (the item's last dP^T MMA done)
+    const uint32_t bar_qf = bar_ve + 8;         // [NQS]
     const uint32_t bar_qe = bar_qf + 8 * NQS;   // [NQS]
     const uint32_t bar_s = bar_qe + 8 * NQS;
     const uint32_t bar_dp = bar_s + 8;
-    const uint32_t bar_p = bar_dp + 8;     // 256 arrivals
-    const uint32_t bar_ds = bar_p + 8;     // 256 arrivals
-    const uint32_t bar_dqf = bar_ds + 8;   // [2]
-    const uint32_t bar_dqe = bar_dqf + 16; // [2] 128 arrivals
-    const uint32_t bar_acc = bar_dqe + 16;
-    const uint32_t bar_wb = bar_acc + 8;   // [2] replaced head: W buffer b consumed
-    const uint32_t bar_pb = bar_wb + 16;   // [2] replaced head: W buffer b written (256 arrivals)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 248);
-    static_assert(8 + 16 * NQS + 104 <= 248, "barrier area");
+    const uint32_t bar_p = bar_dp + 8;      // 256 arrivals
+    const uint32_t bar_ds = bar_p + 8;      // 256 arrivals
+    const uint32_t bar_dqf = bar_ds + 8;    // [2]
+    const uint32_t bar_dqe = bar_dqf + 16;  // [2] 128 arrivals
+    const uint32_t bar_acc = bar_dqe + 16;  // an item's dK, dV complete in TMEM
+    const uint32_t bar_acr = bar_acc + 8;   // an item's dK, dV read out of TMEM (8 warp arrivals)
+    const uint32_t bar_wb = bar_acr + 8;    // [2] replaced head: W buffer b consumed
+    const uint32_t bar_pb = bar_wb + 16;    // [2] replaced head: W buffer b written (256 arrivals)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 240);
+    int* item_slot = reinterpret_cast<int*>(smem + SM_BAR + 248);  // [2]
+    static_assert(80 + 16 * NQS + 112 <= 240, "barrier area");
 
     const int T = p.T;
-    // grouped, longest-first order (key block J walks nqb - J query blocks);
-    // a group's Q/dO tiles and dQ accumulator rows stay in L2
-    int bh, J;
-    grouped_order(blockIdx.x, p.BH, p.nqb, bh, J);
-    const int h = bh % p.H;
-    const int bhkv = (bh / p.H) * p.Hkv + h / (p.H / p.Hkv);  // the K/V slice this query head reads
-    const int slot = p.slot_of_head[h];
-    const bool rep = slot >= 0;
-    // a replaced head whose factors would leave fp32 range takes P^T itself
-    // (one exp per element) in place of W^T, and its dV rows need no c_j
-    const bool direct = rep && p.w.flag[h] != 0;
-    const int ntiles = p.nqb - J;
-    const bool ragged_keys = (J + 1) * BN > T;  // the key block runs past T
+    const int total = p.BH * p.nqb;  // work items: one key block of one (b, h) slice
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_kv, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_itf + 8 * b, 1);
+            mbar_init(bar_ite + 8 * b, 13);
+            mbar_init(bar_kf + 8 * b, 1);
+            mbar_init(bar_ke + 8 * b, 1);
+            mbar_init(bar_dqf + 8 * b, 1);
+            mbar_init(bar_dqe + 8 * b, 128);
+            mbar_init(bar_wb + 8 * b, 1);
+            mbar_init(bar_pb + 8 * b, 256);
+        }
         for (int s = 0; s < NQS; ++s) {
             mbar_init(bar_qf + 8 * s, 1);
             mbar_init(bar_qe + 8 * s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar_dqf + 8 * b, 1);
-            mbar_init(bar_dqe + 8 * b, 128);
-        }
+        mbar_init(bar_vf, 1);
+        mbar_init(bar_ve, 1);
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
         mbar_init(bar_p, 256);
         mbar_init(bar_ds, 256);
-        mbar_init(bar_wb, 1);
-        mbar_init(bar_wb + 8, 1);
-        mbar_init(bar_pb, 256);
-        mbar_init(bar_pb + 8, 256);
         mbar_init(bar_acc, 1);
+        mbar_init(bar_acr, 8);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -233,131 +238,247 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    // Work item n of this CTA (-1: none left), published by the producer
+    // through a 2-slot ring; every consumer warp acknowledges it.
+    auto take_item = [&](int n, int& item) -> bool {
+        if (!mbar_wait(bar_itf + 8 * (n & 1), (n >> 1) & 1, kWaitLimit)) return false;
+        item = *reinterpret_cast<volatile int*>(item_slot + (n & 1));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ite + 8 * (n & 1));
+        return true;
+    };
+    // (b, h) slice and key block of an item, grouped longest-first order (key
+    // block J walks nqb - J query blocks; a group's Q/dO tiles and dQ
+    // accumulator rows stay in L2)
+    struct Item {
+        int bh, bhkv, J, h, slot, ntiles;  // query slice, its K/V slice, key block, head, replaced slot, tiles
+        bool rep, direct, ragged;
+    };
+    auto decode = [&](int item) {
+        Item it;
+        grouped_order((unsigned)item, p.BH, p.nqb, it.bh, it.J);
+        it.h = it.bh % p.H;
+        it.bhkv = (it.bh / p.H) * p.Hkv + it.h / (p.H / p.Hkv);  // the K/V slice this query head reads
+        it.slot = p.slot_of_head[it.h];
+        it.rep = it.slot >= 0;
+        // a replaced head whose factors would leave fp32 range takes P^T itself
+        // (one exp per element) in place of W^T, and its dV rows need no c_j
+        it.direct = it.rep && p.w.flag[it.h] != 0;
+        it.ntiles = p.nqb - it.J;
+        it.ragged = (it.J + 1) * BN > T;  // the key block runs past T
+        return it;
+    };
+
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            if (!rep) {
-                prefetch_tmap(&tmQ);
-                prefetch_tmap(&tmK);
-                prefetch_tmap(&tmV);
-                mbar_expect_tx(bar_kv, 2 * TILE);
-                tma_load_3d(sb + SM_K, &tmK, bar_kv, 0, J * BN, bhkv);
-                tma_load_3d(sb + SM_V, &tmV, bar_kv, 0, J * BN, bhkv);
-            }
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
             prefetch_tmap(&tmDO);
-            for (int t = 0; t < ntiles; ++t) {
-                const int I = J + t, s = t % NQS, n = t / NQS;
-                if (!mbar_wait(bar_qe + 8 * s, (n & 1) ^ 1, kWaitLimit)) { report(p.err, 0x1101); break; }
-                const uint32_t bq = bar_qf + 8 * s;
-                if (!rep) {
-                    mbar_expect_tx(bq, 2 * TILE + 1024);
-                    tma_load_3d(sb + SM_Q + s * TILE, &tmQ, bq, 0, I * BM, bh);
-                    tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, bh);
-                    bulk_load(sb + SM_VEC1 + 512 * s, p.nlse2p + (size_t)bh * p.Tp + I * BM, 512, bq);
-                    bulk_load(sb + SM_VEC2 + 512 * s, p.dvecp + (size_t)bh * p.Tp + I * BM, 512, bq);
-                } else {
-                    mbar_expect_tx(bq, TILE + 512);
-                    tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, bh);
-                    bulk_load(sb + SM_VEC1 + 512 * s, p.w.rsc + (size_t)slot * p.w.Tp + I * BM, 512, bq);
+            int s = 0, u = 0, nk = 0;  // ring stage and pass of the next query block; ordinary items so far
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
+                const int w = (int)atomicAdd(p.err + kCtrBwdNext, 1u);
+                const int item = w < total ? w : -1;
+                if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                *reinterpret_cast<volatile int*>(item_slot + (n & 1)) = item;
+                mbar_arrive(bar_itf + 8 * (n & 1));
+                if (item < 0) break;
+                const Item it = decode(item);
+                if (!it.rep) {
+                    // K of the key block into stage nk & 1, once the MMAs of the
+                    // ordinary item two before (the stage's last user) are done;
+                    // this overlaps the load with the current item's tiles.  V goes
+                    // to L2 now and to shared memory after the first query block
+                    // (its buffer frees up only late in the previous item).
+                    const int kb = nk & 1;
+                    if (!mbar_wait(bar_ke + 8 * kb, ((nk >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                    mbar_expect_tx(bar_kf + 8 * kb, TILE);
+                    tma_load_3d(sb + SM_K + kb * TILE, &tmK, bar_kf + 8 * kb, 0, it.J * BN, it.bhkv);
+                    tma_prefetch_l2_3d(&tmV, 0, it.J * BN, it.bhkv);
                 }
+                for (int t = 0; t < it.ntiles; ++t) {
+                    const int I = it.J + t;
+                    if (!mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                    const uint32_t bq = bar_qf + 8 * s;
+                    if (!it.rep) {
+                        mbar_expect_tx(bq, 2 * TILE + 1024);
+                        tma_load_3d(sb + SM_Q + s * TILE, &tmQ, bq, 0, I * BM, it.bh);
+                        tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, it.bh);
+                        bulk_load(sb + SM_VEC1 + 512 * s, p.nlse2p + (size_t)it.bh * p.Tp + I * BM, 512, bq);
+                        bulk_load(sb + SM_VEC2 + 512 * s, p.dvecp + (size_t)it.bh * p.Tp + I * BM, 512, bq);
+                        if (t == 0) {
+                            // V of ordinary item nk: the previous one's last dP^T read V
+                            if (!mbar_wait(bar_ve, (nk & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                            mbar_expect_tx(bar_vf, TILE);
+                            tma_load_3d(sb + SM_V, &tmV, bar_vf, 0, it.J * BN, it.bhkv);
+                        }
+                    } else {
+                        mbar_expect_tx(bq, TILE + 512);
+                        tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, it.bh);
+                        bulk_load(sb + SM_VEC1 + 512 * s, p.w.rsc + (size_t)it.slot * p.w.Tp + I * BM, 512, bq);
+                    }
+                    if (++s == NQS) {
+                        s = 0;
+                        ++u;
+                    }
+                }
+                if (!it.rep) ++nk;
             }
+            if (!ok) report(p.err, 0x1101);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // K-major x K-major, 128 x 128
-            const uint32_t idTS = idesc_bf16(128, 64, 0, 1);   // TMEM A x MN-major B, 128 x 64
-            const uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // MN-major A x MN-major B
-            // descriptors of the tiles: one base plus (byte offset / 16)
-            const uint64_t d0 = sw128_desc(sb);
-            const uint64_t dK = d0 + (SM_K >> 4), dVd = d0 + (SM_V >> 4);
-            const uint64_t dDS = sw128_desc(sb + SM_DS, 16384);
-            bool ok = rep || mbar_wait(bar_kv, 0, kWaitLimit);
-            if (!ok) report(p.err, 0x1201);
-            // Ordinary heads run one tile ahead: S^T of tile t+1 is issued right
-            // after dV_t (the last reader of the P^T columns it overwrites) and
-            // dP^T of tile t+1 right after dQ_t, so the tensor cores work on the
-            // next tile while the row threads finish this one.  The tensor pipe
-            // executes one thread's MMAs in order, which orders those reuses.
-            // The issuing thread keeps its scalar work small (the pipe stalls
-            // while it computes): ring stages and their descriptors advance
-            // incrementally (a stage is TILE bytes = TILE / 16 descriptor units).
-            constexpr uint64_t kStage = TILE >> 4;
-            const uint64_t dQ0 = d0 + (SM_Q >> 4), dDO0 = d0 + (SM_DO >> 4);
-            auto issue_s = [&](uint64_t dQn) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQn + 2 * k, idSS, k > 0);
-                mma_commit(bar_s);
-            };
-            auto issue_dp = [&](uint64_t dDOn) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOn + 2 * k, idSS, k > 0);
-                mma_commit(bar_dp);
-            };
-            if (ok && !rep) {
-                if (!mbar_wait(bar_qf, 0, kWaitLimit)) { report(p.err, 0x1202); ok = false; }
-                tc_fence_after();
-                if (ok) { issue_s(dQ0); issue_dp(dDO0); }
+        const uint32_t idSS = idesc_bf16(128, 128, 0, 0);  // K-major x K-major, 128 x 128
+        const uint32_t idTS = idesc_bf16(128, 64, 0, 1);   // TMEM A x MN-major B, 128 x 64
+        const uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // MN-major A x MN-major B
+        // descriptors of the tiles: one base plus (byte offset / 16); ring
+        // stages and their descriptors advance incrementally (the issuing
+        // thread keeps its scalar work small: the pipe stalls while it computes)
+        constexpr uint64_t kStage = TILE >> 4;
+        const uint64_t d0 = sw128_desc(sb);
+        const uint64_t dK0 = d0 + (SM_K >> 4), dVd = d0 + (SM_V >> 4);
+        const uint64_t dQ0 = d0 + (SM_Q >> 4), dDO0 = d0 + (SM_DO >> 4);
+        const uint64_t dDS = sw128_desc(sb + SM_DS, 16384);
+        int s = 0, ph = 0;           // ring stage of the next query block and its phase parity
+        int go = 0, gr = 0, nk = 0;  // ordinary tiles, replaced tiles, ordinary items so far
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            int item;
+            ok = __all_sync(0xffffffffu, take_item(n, item));
+            if (!ok) {
+                if (lane == 0) report(p.err, 0x1208);
+                break;
             }
-            int s = 0, ph = 0;  // ring stage of tile t and its phase parity
-            for (int t = 0; ok && t < ntiles; ++t) {
-                const bool wrap = (s + 1 == NQS);
-                const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;  // tile t + 1
-                const uint64_t dQs = dQ0 + (uint64_t)s * kStage, dDOs = dDO0 + (uint64_t)s * kStage;
-                const uint32_t acc = t > 0 ? 1u : 0u;
-                if (!rep) {
-                    if (!mbar_wait(bar_p, t & 1, kWaitLimit)) { report(p.err, 0x1203); ok = false; break; }
-                    tc_fence_after();
+            if (item < 0) break;
+            const Item it = decode(item);
+            int okl = 1;
+            if (lane == 0) {
+                if (!it.rep) {
+                    // Ordinary heads run one tile ahead: S^T of tile t+1 is issued
+                    // right after dV_t (the last reader of the P^T columns it
+                    // overwrites) and dP^T of tile t+1 right after dQ_t, so the tensor
+                    // cores work on the next tile while the row threads finish this
+                    // one; an item's first S^T and dP^T go in while the row threads
+                    // still read out the previous item's dK, dV.  The tensor pipe
+                    // executes one thread's MMAs in order, which orders those reuses.
+                    const int kb = nk & 1;
+                    const uint64_t dK = dK0 + (uint64_t)kb * kStage;
+                    auto issue_s = [&](uint64_t dQn) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DV, tmem + C_S + packed_kcol(k), dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
-                    const bool more = t + 1 < ntiles;
-                    if (more) {
-                        if (!mbar_wait(bar_qf + 8 * s1, ph1, kWaitLimit)) { report(p.err, 0x1207); ok = false; break; }
+                        for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQn + 2 * k, idSS, k > 0);
+                        mma_commit(bar_s);
+                    };
+                    // dP^T of the item's last tile is V's last reader: V's buffer is
+                    // released with it
+                    auto issue_dp = [&](uint64_t dDOn, bool last) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOn + 2 * k, idSS, k > 0);
+                        mma_commit(bar_dp);
+                        if (last) mma_commit(bar_ve);
+                    };
+                    if (!mbar_wait(bar_kf + 8 * kb, (nk >> 1) & 1, kWaitLimit) ||
+                        !mbar_wait(bar_qf + 8 * s, ph, kWaitLimit)) {
+                        report(p.err, 0x1201);
+                        okl = 0;
+                    } else {
                         tc_fence_after();
-                        issue_s(dQ0 + (uint64_t)s1 * kStage);
+                        issue_s(dQ0 + (uint64_t)s * kStage);
+                        if (!mbar_wait(bar_vf, nk & 1, kWaitLimit)) {
+                            report(p.err, 0x120a);
+                            okl = 0;
+                        } else {
+                            tc_fence_after();
+                            issue_dp(dDO0 + (uint64_t)s * kStage, it.ntiles == 1);
+                        }
                     }
-                    if (!mbar_wait(bar_ds, t & 1, kWaitLimit)) { report(p.err, 0x1204); ok = false; break; }
-                    tc_fence_after();
+                    for (int t = 0; okl && t < it.ntiles; ++t) {
+                        const bool wrap = (s + 1 == NQS);
+                        const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;  // tile t + 1
+                        const uint64_t dQs = dQ0 + (uint64_t)s * kStage, dDOs = dDO0 + (uint64_t)s * kStage;
+                        const uint32_t acc = t > 0 ? 1u : 0u;
+                        if (!mbar_wait(bar_p, go & 1, kWaitLimit)) { report(p.err, 0x1203); okl = 0; break; }
+                        // dV, dK start over: the previous item's must have been read out
+                        if (t == 0 && n > 0 && !mbar_wait(bar_acr, (n - 1) & 1, kWaitLimit)) {
+                            report(p.err, 0x1209);
+                            okl = 0;
+                            break;
+                        }
+                        tc_fence_after();
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DK, tmem + C_DP + packed_kcol(k), dQs + 128 * k, idTS, k > 0 ? 1u : acc);
-                    const int b = t & 1;
-                    if (!mbar_wait(bar_dqe + 8 * b, ((t >> 1) & 1) ^ 1, kWaitLimit)) {
-                        report(p.err, 0x1205);
-                        ok = false;
-                        break;
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tmem + C_DV, tmem + C_S + packed_kcol(k), dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
+                        const bool more = t + 1 < it.ntiles;
+                        if (more) {
+                            if (!mbar_wait(bar_qf + 8 * s1, ph1, kWaitLimit)) { report(p.err, 0x1207); okl = 0; break; }
+                            tc_fence_after();
+                            issue_s(dQ0 + (uint64_t)s1 * kStage);
+                        }
+                        if (!mbar_wait(bar_ds, go & 1, kWaitLimit)) { report(p.err, 0x1204); okl = 0; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tmem + C_DK, tmem + C_DP + packed_kcol(k), dQs + 128 * k, idTS, k > 0 ? 1u : acc);
+                        const int b = go & 1;
+                        if (!mbar_wait(bar_dqe + 8 * b, ((go >> 1) & 1) ^ 1, kWaitLimit)) {
+                            report(p.err, 0x1205);
+                            okl = 0;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t cdq = b ? C_DQ1 : C_DQ0;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) mma_ss(tmem + cdq, dDS + 128 * k, dK + 128 * k, idDQ, k > 0);
+                        mma_commit(bar_dqf + 8 * b);
+                        if (more) issue_dp(dDO0 + (uint64_t)s1 * kStage, t + 2 == it.ntiles);
+                        mma_commit(bar_qe + 8 * s);
+                        s = s1;
+                        ph = ph1;
+                        ++go;
                     }
-                    tc_fence_after();
-                    const uint32_t cdq = b ? C_DQ1 : C_DQ0;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) mma_ss(tmem + cdq, dDS + 128 * k, dK + 128 * k, idDQ, k > 0);
-                    mma_commit(bar_dqf + 8 * b);
-                    if (more) issue_dp(dDO0 + (uint64_t)s1 * kStage);
+                    if (okl) {
+                        mma_commit(bar_acc);
+                        mma_commit(bar_ke + 8 * kb);
+                    }
+                    ++nk;
                 } else {
-                    if (!mbar_wait(bar_qf + 8 * s, ph, kWaitLimit)) { report(p.err, 0x1202); ok = false; break; }
-                    tc_fence_after();
-                    if (!mbar_wait(bar_pb + 8 * (t & 1), (t >> 1) & 1, kWaitLimit)) {
-                        report(p.err, 0x1206);
-                        ok = false;
-                        break;
+                    for (int t = 0; okl && t < it.ntiles; ++t) {
+                        const bool wrap = (s + 1 == NQS);
+                        const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;
+                        const uint64_t dDOs = dDO0 + (uint64_t)s * kStage;
+                        const uint32_t acc = t > 0 ? 1u : 0u;
+                        if (!mbar_wait(bar_qf + 8 * s, ph, kWaitLimit)) { report(p.err, 0x1202); okl = 0; break; }
+                        if (!mbar_wait(bar_pb + 8 * (gr & 1), (gr >> 1) & 1, kWaitLimit)) {
+                            report(p.err, 0x1206);
+                            okl = 0;
+                            break;
+                        }
+                        if (t == 0 && n > 0 && !mbar_wait(bar_acr, (n - 1) & 1, kWaitLimit)) {
+                            report(p.err, 0x1209);
+                            okl = 0;
+                            break;
+                        }
+                        tc_fence_after();
+                        // W of this tile sits in buffer gr & 1 (the S^T or the dP^T
+                        // columns, both unused by a replaced head): hi, then lo
+                        const uint32_t wcol = C_S + 128 * (gr & 1);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tmem + C_DV, tmem + wcol + 8 * k, dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tmem + C_DV, tmem + wcol + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
+                        mma_commit(bar_wb + 8 * (gr & 1));
+                        mma_commit(bar_qe + 8 * s);
+                        s = s1;
+                        ph = ph1;
+                        ++gr;
                     }
-                    tc_fence_after();
-                    // W of tile t sits in buffer t & 1 (the S^T or the dP^T
-                    // columns, both unused by a replaced head): hi, then lo
-                    const uint32_t wcol = C_S + 128 * (t & 1);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_ts(tmem + C_DV, tmem + wcol + 8 * k, dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) mma_ts(tmem + C_DV, tmem + wcol + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
-                    mma_commit(bar_wb + 8 * (t & 1));
+                    if (okl) mma_commit(bar_acc);
                 }
-                mma_commit(bar_qe + 8 * s);
-                s = s1;
-                ph = ph1;
             }
-            if (ok) mma_commit(bar_acc);
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
         }
     } else if (warp < 10) {
         // ------------------------------------------------ key rows
@@ -366,128 +487,147 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int quarter = warp & 3;
         const int half = (warp - 2) >> 2;
         const int jl = quarter * 32 + lane;  // key within the block = TMEM lane
-        const int j = J * BN + jl;
         const uint32_t lo = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lo + C_S, tDP = tmem + lo + C_DP;
         const float* vec1 = reinterpret_cast<const float*>(smem + SM_VEC1);
         const float* vec2 = reinterpret_cast<const float*>(smem + SM_VEC2);
+        int s = 0, u = 0, go = 0, gr = 0;  // ring stage and pass; ordinary, replaced tiles so far
         bool ok = true;
-        for (int t = 0; t < ntiles; ++t) {
-            const int I = J + t, s = t % NQS, n = t / NQS;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * s, n & 1, kWaitLimit));
-            if (!ok) { report(p.err, 0x1301); break; }
-            const float* v1 = vec1 + 128 * s;
-            if (!rep) {
-                const float* v2 = vec2 + 128 * s;
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_s, t & 1, kWaitLimit));
-                if (!ok) { report(p.err, 0x1302); break; }
-                tc_fence_after();
-                // P^T, 32 queries at a time: bf16 pairs written over the S^T
-                // columns already read (chunk c -> columns [16c, 16c + 16)).
-                // Masks only on the diagonal tile and in a ragged last key
-                // block (a warp-uniform choice: the TMEM ops are collective).
-                // P^T stays in registers for dS^T: the S^T columns are reused by
-                // the next tile's S^T as soon as dV has read them.
-                uint32_t pw[2][16];
-                if (t == 0 || ragged_keys) {
+        for (int n = 0; ok; ++n) {
+            int item;
+            ok = __all_sync(0xffffffffu, take_item(n, item));
+            if (!ok) {
+                report(p.err, 0x1306);
+                break;
+            }
+            if (item < 0) break;
+            const Item it = decode(item);
+            const int j = it.J * BN + jl;
+            const float aj = (it.direct && j < T) ? p.a[(size_t)it.h * T + j] : kNegInf;
+            for (int t = 0; t < it.ntiles; ++t) {
+                const int I = it.J + t;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * s, u & 1, kWaitLimit));
+                if (!ok) { report(p.err, 0x1301); break; }
+                const float* v1 = vec1 + 128 * s;
+                if (!it.rep) {
+                    const float* v2 = vec2 + 128 * s;
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_s, go & 1, kWaitLimit));
+                    if (!ok) { report(p.err, 0x1302); break; }
+                    tc_fence_after();
+                    // P^T, 32 queries at a time: bf16 pairs written over the S^T
+                    // columns already read (chunk c -> columns [16c, 16c + 16)).
+                    // Masks only on the diagonal tile and in a ragged last key
+                    // block (a warp-uniform choice: the TMEM ops are collective).
+                    // P^T stays in registers for dS^T: the S^T columns are reused by
+                    // the next tile's S^T as soon as dV has read them.
+                    uint32_t pw[2][16];
+                    if (t == 0 || it.ragged) {
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
-                        p_chunk<true>(tS, 2 * half + cc, v1, p.scale_log2, jl, t == 0, j < T, pw[cc]);
-                } else {
+                        for (int cc = 0; cc < 2; ++cc)
+                            p_chunk<true>(tS, 2 * half + cc, v1, p.scale_log2, jl, t == 0, j < T, pw[cc]);
+                    } else {
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
-                        p_chunk<false>(tS, 2 * half + cc, v1, p.scale_log2, jl, false, true, pw[cc]);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar_p);
-                // dS^T = P^T o (dP^T - D), P^T from registers; dS^T goes over the
-                // dP^T columns this warp has read and, as row jl of the MN-major
-                // A operand of dQ = dS K, into shared memory
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, t & 1, kWaitLimit));
-                if (!ok) { report(p.err, 0x1303); break; }
-                tc_fence_after();
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * half + cc;
-                    uint32_t v[32], dsw[16];
-                    tmem_ld32(tDP + 32 * c, v);
-                    tmem_wait_ld();
-                    const uint64_t* d2 = reinterpret_cast<const uint64_t*>(v2 + 32 * c);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        // (dP - D) paired, times P (bf16, widened), one rounding
-                        const float2 pf = unpack_bf16x2(pw[cc][e / 2]);
-                        const uint64_t g = sub_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), d2[e / 2]);
-                        const float2 ds = split_f32x2(mul_f32x2(f32x2(pf.x, pf.y), g));
-                        dsw[e / 2] = pack_bf16x2(ds.x, ds.y);
+                        for (int cc = 0; cc < 2; ++cc)
+                            p_chunk<false>(tS, 2 * half + cc, v1, p.scale_log2, jl, false, true, pw[cc]);
                     }
-                    tmem_st16(tDP + packed_col(c), dsw);
-                    // queries [64 half, 64 half + 64) form the MN atom `half`
-                    const uint32_t blk = sb + SM_DS + half * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int ch = cc * 4 + u;
-                        st_shared_v4(blk + ((ch ^ (jl & 7)) << 4), dsw[4 * u], dsw[4 * u + 1], dsw[4 * u + 2],
-                                     dsw[4 * u + 3]);
-                    }
-                }
-                fence_proxy_async_smem();
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar_ds);
-            } else {
-                // W^T(j, i) = E[i-j] r_i, hi + lo bf16, into buffer t & 1; that
-                // buffer was last read by the MMAs of tile t - 2 (one barrier per
-                // buffer, so neither can run two phases ahead of this wait)
-                const uint32_t tW = tmem + lo + C_S + 128 * (t & 1);
-                if (t >= 2) {
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(bar_wb + 8 * (t & 1), ((t >> 1) & 1) ^ 1, kWaitLimit));
-                    if (!ok) { report(p.err, 0x1304); break; }
-                }
-                tc_fence_after();
-                const float* ef = p.w.ef + (size_t)slot * p.w.Lp + 128 + (I - J) * BM - jl;
-                const float aj = (direct && j < T) ? p.a[(size_t)h * T + j] : kNegInf;
-                if (!direct) {
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar_p);
+                    // dS^T = P^T o (dP^T - D), P^T from registers; dS^T goes over the
+                    // dP^T columns this warp has read and, as row jl of the MN-major
+                    // A operand of dQ = dS K, into shared memory
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, go & 1, kWaitLimit));
+                    if (!ok) { report(p.err, 0x1303); break; }
+                    tc_fence_after();
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int c = 2 * half + cc;
-                        uint32_t hw[16], lw[16];
+                        uint32_t v[32], dsw[16];
+                        tmem_ld32(tDP + 32 * c, v);
+                        tmem_wait_ld();
+                        const uint64_t* d2 = reinterpret_cast<const uint64_t*>(v2 + 32 * c);
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const int ql = 32 * c + e;
-                            const float w0 = __ldg(ef + ql) * v1[ql];
-                            const float w1 = __ldg(ef + ql + 1) * v1[ql + 1];
-                            const uint32_t hb = pack_bf16x2(w0, w1);
-                            const float2 hf = unpack_bf16x2(hb);
-                            hw[e / 2] = hb;
-                            lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                            // (dP - D) paired, times P (bf16, widened), one rounding
+                            const float2 pf = unpack_bf16x2(pw[cc][e / 2]);
+                            const uint64_t g =
+                                sub_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), d2[e / 2]);
+                            const float2 ds = split_f32x2(mul_f32x2(f32x2(pf.x, pf.y), g));
+                            dsw[e / 2] = pack_bf16x2(ds.x, ds.y);
                         }
-                        tmem_st16(tW + 16 * c, hw);
-                        tmem_st16(tW + 64 + 16 * c, lw);
+                        tmem_st16(tDP + packed_col(c), dsw);
+                        // queries [64 half, 64 half + 64) form the MN atom `half`
+                        const uint32_t blk = sb + SM_DS + half * 16384 + (jl >> 3) * 1024 + (jl & 7) * 128;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int ch = cc * 4 + q4;
+                            st_shared_v4(blk + ((ch ^ (jl & 7)) << 4), dsw[4 * q4], dsw[4 * q4 + 1],
+                                         dsw[4 * q4 + 2], dsw[4 * q4 + 3]);
+                        }
                     }
+                    fence_proxy_async_smem();
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar_ds);
+                    ++go;
                 } else {
-                    direct_pt_half(p, h, T, aj, j, I * BM, half, tW);
+                    // W^T(j, i) = E[i-j] r_i, hi + lo bf16, into buffer gr & 1; that
+                    // buffer was last read by the MMAs of replaced tile gr - 2 (one
+                    // barrier per buffer, so neither can run two phases ahead of this
+                    // wait); MMAs of any ordinary item in between finished before this
+                    // item started (its dK, dV read-out waited for them)
+                    const uint32_t tW = tmem + lo + C_S + 128 * (gr & 1);
+                    if (gr >= 2) {
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(bar_wb + 8 * (gr & 1), ((gr >> 1) & 1) ^ 1, kWaitLimit));
+                        if (!ok) { report(p.err, 0x1304); break; }
+                    }
+                    tc_fence_after();
+                    if (!it.direct) {
+                        const float* ef = p.w.ef + (size_t)it.slot * p.w.Lp + 128 + (I - it.J) * BM - jl;
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int c = 2 * half + cc;
+                            uint32_t hw[16], lw[16];
+#pragma unroll
+                            for (int e = 0; e < 32; e += 2) {
+                                const int ql = 32 * c + e;
+                                const float w0 = __ldg(ef + ql) * v1[ql];
+                                const float w1 = __ldg(ef + ql + 1) * v1[ql + 1];
+                                const uint32_t hb = pack_bf16x2(w0, w1);
+                                const float2 hf = unpack_bf16x2(hb);
+                                hw[e / 2] = hb;
+                                lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                            }
+                            tmem_st16(tW + 16 * c, hw);
+                            tmem_st16(tW + 64 + 16 * c, lw);
+                        }
+                    } else {
+                        direct_pt_half(p, it.h, T, aj, j, I * BM, half, tW);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar_pb + 8 * (gr & 1));
+                    ++gr;
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar_pb + 8 * (t & 1));
+                if (++s == NQS) {
+                    s = 0;
+                    ++u;
+                }
             }
-        }
-        // dK, dV epilogue
-        if (ok) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_acc, 0, kWaitLimit));
-            if (!ok) report(p.err, 0x1305);
-        }
-        tc_fence_after();
-        if (ok) {
-            // half 0 writes the dV row (times c_j for a replaced head), half 1
-            // the dK row (times 1/sqrt(d); zero for a replaced head)
+            if (!ok) break;
+            // the item's dK, dV: half 0 writes the dV row (times c_j for a replaced
+            // head), half 1 the dK row (times 1/sqrt(d); zero for a replaced head)
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_acc, n & 1, kWaitLimit));
+            if (!ok) {
+                report(p.err, 0x1305);
+                break;
+            }
+            tc_fence_after();
             float vals[64];
             float mul;
-            if (half == 0) mul = (rep && !direct && j < T) ? p.w.cf[(size_t)slot * p.w.Tp + j] : 1.f;
-            else mul = rep ? 0.f : p.scale;
+            if (half == 0) mul = (it.rep && !it.direct && j < T) ? p.w.cf[(size_t)it.slot * p.w.Tp + j] : 1.f;
+            else mul = it.rep ? 0.f : p.scale;
             const uint32_t col = half == 0 ? C_DV : C_DK;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -497,63 +637,79 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                 for (int e = 0; e < 32; ++e) vals[32 * c + e] = __uint_as_float(v[e]) * mul;
             }
-            if (j < T) store_row(half == 0 ? p.dv : p.dk, p.grad_fp32, (size_t)bh * T + j, vals);
+            tc_fence_before();
+            mbar_arrive_warp(bar_acr);
+            // per-thread row stores (fire and forget: the warps move on to the next
+            // item at once, which measured faster than staging for coalescing)
+            if (j < T) store_row(half == 0 ? p.dv : p.dk, p.grad_fp32, (size_t)it.bh * T + j, vals);
         }
-    } else if (!rep) {
+    } else {
         // ------------------------------------------------ dQ tiles -> global accumulator
+        // Each warp moves its own 32 query rows: TMEM -> two 4 KB swizzled boxes
+        // of its own (columns 0..31, 32..63) -> TMA reduce-add (no cross-warp sync).
         const int quarter = warp & 3;
         const int ql = quarter * 32 + lane;
         const uint32_t lo = (uint32_t)(quarter * 32) << 16;
-        const bool leader = (warp == 10 && lane == 0);
+        const uint32_t box = sb + SM_DQ + quarter * 8192;
+        const uint32_t stg = box + lane * 128;
+        int go = 0;
         bool ok = true;
-        // every thread passes both named barriers of every tile, even after a
-        // timed-out wait (then it only skips the work), so none is left behind
-        for (int t = 0; t < ntiles; ++t) {
-            const int I = J + t, b = t & 1, nb = t >> 1;
-            if (ok) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_dqf + 8 * b, nb & 1, kWaitLimit));
-                if (!ok) report(p.err, 0x1401);
-            }
+        for (int n = 0; ok; ++n) {
+            int item;
+            ok = __all_sync(0xffffffffu, take_item(n, item));
             if (!ok) {
-                named_sync(1, 128);
-                named_sync(1, 128);
-                continue;
+                report(p.err, 0x1402);
+                break;
             }
-            tc_fence_after();
-            uint32_t v0[32], v1[32];
-            tmem_ld32(tmem + lo + (b ? C_DQ1 : C_DQ0), v0);
-            tmem_ld32(tmem + lo + (b ? C_DQ1 : C_DQ0) + 32, v1);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar_dqe + 8 * b);
-            // the staging buffer must have been read by the previous reduce
-            if (leader) bulk_wait_read0();
-            named_sync(1, 128);
-            // row ql of the two [128][32] fp32 boxes, 16-byte chunks XOR-swizzled
-            // by row (the reduce map's 128-byte swizzle; conflict-free stores)
-            const uint32_t stg = sb + SM_DQ + ql * 128;
+            if (item < 0) break;
+            const Item it = decode(item);
+            if (it.rep) continue;  // a replaced head adds nothing to dQ
+            for (int t = 0; t < it.ntiles; ++t, ++go) {
+                const int I = it.J + t, b = go & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_dqf + 8 * b, (go >> 1) & 1, kWaitLimit));
+                if (!ok) { report(p.err, 0x1401); break; }
+                tc_fence_after();
+                uint32_t v0[32], v1[32];
+                tmem_ld32(tmem + lo + (b ? C_DQ1 : C_DQ0), v0);
+                tmem_ld32(tmem + lo + (b ? C_DQ1 : C_DQ0) + 32, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar_dqe + 8 * b);
+                // the boxes must have been read by the previous tile's reduces
+                if (lane == 0) bulk_wait_read0();
+                __syncwarp();
+                // row `lane` of each [32][32] fp32 box, 16-byte chunks XOR-swizzled
+                // by row (the reduce map's 128-byte swizzle; conflict-free stores)
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const uint32_t off = (uint32_t)((u ^ (ql & 7)) << 4);
-                st_shared_v4(stg + off, v0[4 * u], v0[4 * u + 1], v0[4 * u + 2], v0[4 * u + 3]);
-                st_shared_v4(stg + 16384 + off, v1[4 * u], v1[4 * u + 1], v1[4 * u + 2], v1[4 * u + 3]);
-            }
-            fence_proxy_async_smem();
-            named_sync(1, 128);
-            if (leader) {
-                const uint32_t box = sb + SM_DQ;
-                tma_reduce_add_3d(&tmDQ, box, 0, I * BM, bh);
-                tma_reduce_add_3d(&tmDQ, box + 16384, 32, I * BM, bh);
-                bulk_commit();
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const uint32_t off = (uint32_t)((c4 ^ (ql & 7)) << 4);
+                    st_shared_v4(stg + off, v0[4 * c4], v0[4 * c4 + 1], v0[4 * c4 + 2], v0[4 * c4 + 3]);
+                    st_shared_v4(stg + 4096 + off, v1[4 * c4], v1[4 * c4 + 1], v1[4 * c4 + 2], v1[4 * c4 + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_reduce_add_3d(&tmDQ, box, 0, I * BM + quarter * 32, it.bh);
+                    tma_reduce_add_3d(&tmDQ, box + 4096, 32, I * BM + quarter * 32, it.bh);
+                    bulk_commit();
+                }
             }
         }
-        if (leader) bulk_wait0();
+        if (lane == 0) bulk_wait0();
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
+    }
+    // the last CTA to finish resets the work counters for the next launch
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.err + kCtrBwdDone, 1u) == gridDim.x - 1) {
+            atomicExch(p.err + kCtrBwdNext, 0u);
+            atomicExch(p.err + kCtrBwdDone, 0u);
+        }
     }
 }
 
@@ -646,8 +802,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 }  // namespace
 
-// [BH, T, 64] fp32 as a 3-D tensor (d, t, bh); 128 x 32 boxes (128-byte rows)
-// with the 128-byte swizzle.
+// [BH, T, 64] fp32 as a 3-D tensor (d, t, bh); 32 x 32 boxes (32 rows of 128
+// bytes) with the 128-byte swizzle.
 bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out) {
     static EncodeTiledFn fn = nullptr;
     static bool tried = false;
@@ -662,7 +818,7 @@ bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out) {
     if (!fn) return false;
     cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)BH};
     cuuint64_t strides[2] = {64 * 4, (cuuint64_t)T * 64 * 4};
-    cuuint32_t box[3] = {32, 128, 1};
+    cuuint32_t box[3] = {32, 32, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -740,8 +896,11 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     const int smem = SM_TOTAL + 1024;
     cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // persistent: one CTA per SM (TMEM and shared memory allow one), at most one per item
+    const int items = BH * p.nqb;
+    const int grid = items < sm_count() ? items : sm_count();
     launch_begin(KID_BWD_TC, stream);
-    bwd_tc_kernel<<<dim3((unsigned)BH * p.nqb), NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
+    bwd_tc_kernel<<<dim3((unsigned)grid), NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
     launch_end(KID_BWD_TC, stream);
     return cudaGetLastError();
 }

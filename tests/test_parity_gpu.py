@@ -444,3 +444,35 @@ def test_persistent_forward_leaves_its_counters_zero():
         outs.append((o.clone(), lse.clone()))
     for o, lse in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1])
+
+
+def test_persistent_backward_leaves_its_counters_zero():
+    """The persistent backward's work counters in the workspace header are zero
+    after each call, and repeated calls give the same dK, dV (one CTA owns a key
+    block) and dQ up to the order of its fp32 reduce-adds."""
+    w = I.custom(2, 3, 520, [0])
+    x = I.make_inputs(w, 63)
+    g = P.to_gpu(x)
+    o, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"])
+    ws = saf.new_workspace(w.B, w.H, w.T, "cuda", backward=True)
+    outs = []
+    for _ in range(3):
+        dq, dk, dv = saf.mixed_attn_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, g["alpha"], g["rho"], x["mask"],
+                                        grad_dtype=torch.float32, workspace=ws)
+        torch.cuda.synchronize()
+        header = ws[:64].view(torch.int32).cpu()
+        assert int(header[0]) == 0 and int(header[4]) == 0 and int(header[5]) == 0
+        outs.append((dq.clone(), dk.clone(), dv.clone()))
+    for dq, dk, dv in outs[1:]:
+        assert torch.equal(dk, outs[0][1]) and torch.equal(dv, outs[0][2])
+        assert (dq - outs[0][0]).abs().max().item() <= 1e-5 * max(1.0, outs[0][0].abs().max().item())
+
+
+def test_persistent_backward_many_items_per_cta():
+    """More key-block items than SMs (512 items of 1 to 16 tiles, ordinary and
+    replaced heads interleaved in the longest-first order, a ragged T), so every
+    CTA runs several items back to back: every slice against the oracle."""
+    w = I.custom(4, 8, 2000, [1, 4, 6])
+    x = I.make_inputs(w, 64)
+    got = P.run_layer(w, x, torch.float32)
+    P.check_slices(w, x, got, _all_slices(w))
