@@ -8,6 +8,7 @@ exceptions.  It raises when the library is missing: there is no fallback.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from typing import Optional, Tuple
 
@@ -50,6 +51,22 @@ SIGNATURES = {
 }
 
 _lib = None
+
+
+def _annotated(fn):
+    """With SAF_NVTX=1 in the environment, each call is an NVTX range named
+    saf.<function> (a profiler can then select one call, e.g. ncu --nvtx
+    --nvtx-include); otherwise the call is unchanged."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        if os.environ.get("SAF_NVTX", "") in ("", "0"):
+            return fn(*args, **kwargs)
+        torch.cuda.nvtx.range_push("saf." + fn.__name__)
+        try:
+            return fn(*args, **kwargs)
+        finally:
+            torch.cuda.nvtx.range_pop()
+    return wrapper
 
 
 class SafError(RuntimeError):
@@ -125,6 +142,7 @@ def _check_layer_tensor(name: str, t: torch.Tensor, shape, dtype=torch.bfloat16)
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}")
 
 
+@_annotated
 def replaced_lognorm(alpha: torch.Tensor, rho: torch.Tensor, mask, out: Optional[torch.Tensor] = None,
                      stream=None) -> torch.Tensor:
     """log Z [H, T] of the replaced heads (other rows left as in `out`)."""
@@ -139,6 +157,7 @@ def replaced_lognorm(alpha: torch.Tensor, rho: torch.Tensor, mask, out: Optional
     return out
 
 
+@_annotated
 def mixed_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
                    rho: torch.Tensor, mask, logz: Optional[torch.Tensor] = None,
                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
@@ -174,6 +193,7 @@ def mixed_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: tor
     return out, lse
 
 
+@_annotated
 def mixed_attn_bwd(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtype=torch.bfloat16,
                    dq=None, dk=None, dv=None, workspace=None, stream=None):
     """Backward of one mixed-head layer.  Returns (dQ, dK, dV) in grad_dtype (bf16 or fp32).
@@ -211,6 +231,7 @@ def mixed_attn_bwd(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtyp
     return dq, dk, dv
 
 
+@_annotated
 def replaced_pattern_grad(v, dout, alpha, rho, mask, logz=None, da=None, dr=None, workspace=None, stream=None):
     """Trainable pattern: (dalpha, drho) [H, T] fp32 of the replaced heads
     (rows of ordinary heads zero) for the output gradient dout."""
@@ -232,6 +253,7 @@ def replaced_pattern_grad(v, dout, alpha, rho, mask, logz=None, da=None, dr=None
     return da, dr
 
 
+@_annotated
 def fit_pattern(target, steps: int = 400, lr: float = 0.1, stream=None):
     """Fits a, r of Eq. (3) to target patterns [n, T, T] (fp32, causal, unit
     row sums).  Returns (a [n, T], r [n, T], mean row KL [n])."""
@@ -252,6 +274,7 @@ def fit_pattern(target, steps: int = 400, lr: float = 0.1, stream=None):
     return a, r, kl
 
 
+@_annotated
 def attn_calibration(q, k, lse, a_hat=None, svar=None, workspace=None, stream=None):
     """Calibration statistics over the N samples of q, k [N,H,T,64] (lse from
     the forward of the same inputs): (A_hat [H,T,T] fp32, s_var [H] fp32), Eq. (1)."""
@@ -271,6 +294,7 @@ def attn_calibration(q, k, lse, a_hat=None, svar=None, workspace=None, stream=No
     return a_hat, svar
 
 
+@_annotated
 def mixed_attn_bwd_noalloc(q, k, v, o, dout, lse, alpha, rho, mask, logz=None, grad_dtype=torch.bfloat16,
                            dq=None, dk=None, dv=None, stream=None):
     """Backward without a workspace (the library's own fixed scratch, see

@@ -135,3 +135,24 @@ def test_selftest_argument_errors(lib):
     assert lib.saf_selftest_wait_timeout(FAKE, 16, 1000, None) == saf.SAF_ERR_WORKSPACE
     assert lib.saf_selftest_wait_timeout(FAKE, 256, 0, None) == saf.SAF_ERR_INVALID_ARG
     assert lib.saf_selftest_wait_timeout(FAKE, 256, 1 << 40, None) == saf.SAF_ERR_INVALID_ARG
+
+
+def test_nvtx_ranges_are_opt_in(monkeypatch):
+    """With SAF_NVTX=1 each binding call is one NVTX range (pushed and popped
+    even when the call raises); without it no NVTX call is made."""
+    import torch
+
+    calls = []
+    monkeypatch.setattr(torch.cuda.nvtx, "range_push", lambda name: calls.append(("push", name)))
+    monkeypatch.setattr(torch.cuda.nvtx, "range_pop", lambda: calls.append(("pop",)))
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    k_bad = torch.zeros(1, 2, 9, 64, dtype=torch.bfloat16)  # T mismatch: rejected before the library
+    a = torch.zeros(2, 8)
+    monkeypatch.delenv("SAF_NVTX", raising=False)
+    with pytest.raises(ValueError):
+        saf.mixed_attn_fwd(q, k_bad, k_bad, a, a, [0, 1])
+    assert calls == []
+    monkeypatch.setenv("SAF_NVTX", "1")
+    with pytest.raises(ValueError):
+        saf.mixed_attn_fwd(q, k_bad, k_bad, a, a, [0, 1])
+    assert calls == [("push", "saf.mixed_attn_fwd"), ("pop",)]
