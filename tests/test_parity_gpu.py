@@ -218,8 +218,10 @@ def test_guarded_and_factored_heads_in_one_call():
 
 
 @pytest.mark.parametrize("B,H,Hkv,T,replaced", [(2, 8, 2, 650, [1, 5]), (1, 4, 1, 300, [0, 3]),
-                                                (2, 6, 3, 1000, [2]), (1, 4, 2, 129, [])],
-                         ids=["gqa4_t650", "mqa_t300", "gqa2_t1000", "gqa2_t129_no_replaced"])
+                                                (2, 6, 3, 1000, [2]), (1, 4, 2, 129, []),
+                                                (2, 8, 2, 2000, [1, 5])],
+                         ids=["gqa4_t650", "mqa_t300", "gqa2_t1000", "gqa2_t129_no_replaced",
+                              "gqa4_t2000_several_items_per_cta"])
 @pytest.mark.parametrize("grad_dtype", [torch.float32, torch.bfloat16], ids=["grad_fp32", "grad_bf16"])
 def test_grouped_kv_layer(B, H, Hkv, T, replaced, grad_dtype):
     """Shared K/V heads (H / Hkv query heads per K/V head, replaced heads mixed
