@@ -629,13 +629,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (half == 0) mul = (it.rep && !it.direct && j < T) ? p.w.cf[(size_t)it.slot * p.w.Tp + j] : 1.f;
             else mul = it.rep ? 0.f : p.scale;
             const uint32_t col = half == 0 ? C_DV : C_DK;
+            // a replaced head's dK columns were never written by this item (TMEM
+            // holds whatever came before): its rows are zeros, not 0 x that
+            const bool zero = half == 1 && it.rep;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tmem + lo + col + 32 * c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) vals[32 * c + e] = __uint_as_float(v[e]) * mul;
+                for (int e = 0; e < 32; ++e) vals[32 * c + e] = zero ? 0.f : __uint_as_float(v[e]) * mul;
             }
             tc_fence_before();
             mbar_arrive_warp(bar_acr);
