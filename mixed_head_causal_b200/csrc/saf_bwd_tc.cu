@@ -400,6 +400,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         const uint32_t acc = t > 0 ? 1u : 0u;
                         if (!mbar_wait(bar_p, go & 1, kWaitLimit)) { report(p.err, 0x1203); okl = 0; break; }
                         // dV, dK start over: the previous item's must have been read out
+                        // (already implied: the row warps read them out before writing
+                        // this P^T; the wait is a cheap safeguard)
                         if (t == 0 && n > 0 && !mbar_wait(bar_acr, (n - 1) & 1, kWaitLimit)) {
                             report(p.err, 0x1209);
                             okl = 0;
