@@ -49,11 +49,12 @@ __host__ __device__ inline int round_up128(int x) { return (x + 127) & ~127; }
 // stay in L2, and inside a group the CTAs run longest first across all its
 // slices, so the last CTAs to start are the shortest and the tail is small.
 constexpr int kHeadGroup = 16;
-__device__ __forceinline__ void grouped_order(unsigned b, int BH, int nblk, int& bh, int& rank) {
+__host__ __device__ __forceinline__ void grouped_order(unsigned b, int BH, int nblk, int& bh, int& rank) {
     const unsigned per_group = (unsigned)kHeadGroup * (unsigned)nblk;
     const int g = (int)(b / per_group);
     const int r = (int)(b - (unsigned)g * per_group);
-    const int heads = min(kHeadGroup, BH - g * kHeadGroup);
+    const int left = BH - g * kHeadGroup;  // slices in this group (the last one may be partial)
+    const int heads = left < kHeadGroup ? left : kHeadGroup;
     rank = r / heads;
     bh = g * kHeadGroup + (r - rank * heads);
 }
