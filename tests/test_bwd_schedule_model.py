@@ -1,8 +1,9 @@
 """A model of the synchronization protocol of the persistent backward kernel
 (`csrc/saf_bwd_tc.cu`), checked under random schedules.
 
-Each role of the kernel (TMA producer, MMA issuer, key-row warps, dQ warps) is
-written here as a generator that performs the same barrier operations, in the
+Each role of the kernel (TMA producer, MMA issuer, each of the 8 key-row warps
+and each of the 4 dQ warps, with the kernel's arrival counts and their own
+slices of the TMEM regions) is written here as a generator that performs the same barrier operations, in the
 same order and with the same phase parities, as the CUDA code (the machinery
 is in tests/schedule_model.py).  For every run the model checks:
 
@@ -23,6 +24,17 @@ import pytest
 from tests.schedule_model import Machine, ModelError, W, mutate, publish, simulate, take
 
 NQS = 3  # Q/dO ring depth
+ROWS = 8  # key-row warps: each owns one slice (lane quarter x column half) of S^T, dP^T and dS^T
+DQW = 4   # dQ warps: each owns one lane quarter of the dQ tiles
+
+
+def parts(res, n):
+    """The per-warp slices of a region that the MMA reads or writes whole."""
+    return [f"{res}.{w}" for w in range(n)]
+
+
+def all_of(res, n, version):
+    return [(r, version) for r in parts(res, n)]
 
 
 def ring(g):
@@ -71,10 +83,10 @@ def mma_issuer(m):
             yield W(f"kf{kb}", nk >> 1, (nk >> 1) & 1)
             s0, p0, u0 = ring(G)
             yield W(f"qf{s0}", u0, p0)
-            m.mma([(f"K{kb}", ("K", nk)), (f"Q{s0}", ("Q", G))], [("C_S", ("S", go))], "S")
+            m.mma([(f"K{kb}", ("K", nk)), (f"Q{s0}", ("Q", G))], all_of("C_S", ROWS, ("S", go)), "S")
             m.commit("s")
             yield W("vf", nk, nk & 1)
-            m.mma([("V", ("V", nk)), (f"DO{s0}", ("DO", G))], [("C_DP", ("dP", go))], "dP")
+            m.mma([("V", ("V", nk)), (f"DO{s0}", ("DO", G))], all_of("C_DP", ROWS, ("dP", go)), "dP")
             m.commit("dp")
             if ntiles == 1:
                 m.commit("ve")
@@ -86,21 +98,21 @@ def mma_issuer(m):
                 if t == 0 and n > 0:
                     yield W("acr", n - 1, (n - 1) & 1)
                 acc_in = [("C_DV", ("dV", n, t - 1))] if t > 0 else []
-                m.mma([("C_S", ("P", go)), (f"DO{st}", ("DO", g))] + acc_in, [("C_DV", ("dV", n, t))], "dV")
+                m.mma(all_of("C_S", ROWS, ("P", go)) + [(f"DO{st}", ("DO", g))] + acc_in, [("C_DV", ("dV", n, t))], "dV")
                 more = t + 1 < ntiles
                 if more:
                     yield W(f"qf{s1}", u1, p1)
-                    m.mma([(f"K{kb}", ("K", nk)), (f"Q{s1}", ("Q", g + 1))], [("C_S", ("S", go + 1))], "S")
+                    m.mma([(f"K{kb}", ("K", nk)), (f"Q{s1}", ("Q", g + 1))], all_of("C_S", ROWS, ("S", go + 1)), "S")
                     m.commit("s")
                 yield W("ds", go, go & 1)
                 acc_in = [("C_DK", ("dK", n, t - 1))] if t > 0 else []
-                m.mma([("C_DP", ("dS", go)), (f"Q{st}", ("Q", g))] + acc_in, [("C_DK", ("dK", n, t))], "dK")
+                m.mma(all_of("C_DP", ROWS, ("dS", go)) + [(f"Q{st}", ("Q", g))] + acc_in, [("C_DK", ("dK", n, t))], "dK")
                 b = go & 1
                 yield W(f"dqe{b}", (go >> 1) - 1, ((go >> 1) & 1) ^ 1)
-                m.mma([("DS", ("dS", go)), (f"K{kb}", ("K", nk))], [(f"C_DQ{b}", ("dQ", go))], "dQ")
+                m.mma(all_of("DS", ROWS, ("dS", go)) + [(f"K{kb}", ("K", nk))], all_of(f"C_DQ{b}", DQW, ("dQ", go)), "dQ")
                 m.commit(f"dqf{b}")
                 if more:
-                    m.mma([("V", ("V", nk)), (f"DO{s1}", ("DO", g + 1))], [("C_DP", ("dP", go + 1))], "dP")
+                    m.mma([("V", ("V", nk)), (f"DO{s1}", ("DO", g + 1))], all_of("C_DP", ROWS, ("dP", go + 1)), "dP")
                     m.commit("dp")
                     if t + 2 == ntiles:
                         m.commit("ve")
@@ -119,7 +131,7 @@ def mma_issuer(m):
                     yield W("acr", n - 1, (n - 1) & 1)
                 wreg = "C_S" if gr % 2 == 0 else "C_DP"
                 acc_in = [("C_DV", ("dV", n, t - 1))] if t > 0 else []
-                m.mma([(wreg, ("W", gr)), (f"DO{st}", ("DO", g))] + acc_in, [("C_DV", ("dV", n, t))], "dV(W)")
+                m.mma(all_of(wreg, ROWS, ("W", gr)) + [(f"DO{st}", ("DO", g))] + acc_in, [("C_DV", ("dV", n, t))], "dV(W)")
                 m.commit(f"wb{gr & 1}")
                 m.commit(f"qe{st}")
                 gr += 1
@@ -128,7 +140,7 @@ def mma_issuer(m):
         n += 1
 
 
-def key_rows(m):
+def key_rows(m, w):
     go = gr = 0
     G = 0
     n = 0
@@ -143,22 +155,22 @@ def key_rows(m):
             yield W(f"qf{s}", u, p)
             if not rep:
                 yield W("s", go, go & 1)
-                m.read("C_S", ("S", go), "rows P")
+                m.read(f"C_S.{w}", ("S", go), "rows P")
                 m.read(f"VEC1_{s}", ("VEC", g), "rows P")
-                m.write("C_S", ("P", go), "rows P")
+                m.write(f"C_S.{w}", ("P", go), "rows P")
                 m.bars["p"].arrive()
                 yield W("dp", go, go & 1)
-                m.read("C_DP", ("dP", go), "rows dS")
+                m.read(f"C_DP.{w}", ("dP", go), "rows dS")
                 m.read(f"VEC2_{s}", ("VEC", g), "rows dS")
-                m.write("C_DP", ("dS", go), "rows dS")
-                m.write("DS", ("dS", go), "rows dS")
+                m.write(f"C_DP.{w}", ("dS", go), "rows dS")
+                m.write(f"DS.{w}", ("dS", go), "rows dS")
                 m.bars["ds"].arrive()
                 go += 1
             else:
                 if gr >= 2:
                     yield W(f"wb{gr & 1}", (gr >> 1) - 1, ((gr >> 1) & 1) ^ 1)
                 m.read(f"VEC1_{s}", ("VEC", g), "rows W")
-                m.write("C_S" if gr % 2 == 0 else "C_DP", ("W", gr), "rows W")
+                m.write(f"{'C_S' if gr % 2 == 0 else 'C_DP'}.{w}", ("W", gr), "rows W")
                 m.bars[f"pb{gr & 1}"].arrive()
                 gr += 1
         G += ntiles
@@ -171,7 +183,7 @@ def key_rows(m):
         n += 1
 
 
-def dq_warps(m):
+def dq_warp(m, w):
     go = 0
     n = 0
     while True:
@@ -185,7 +197,7 @@ def dq_warps(m):
         for _ in range(ntiles):
             b = go & 1
             yield W(f"dqf{b}", go >> 1, (go >> 1) & 1)
-            m.read(f"C_DQ{b}", ("dQ", go), "dQ warps")
+            m.read(f"C_DQ{b}.{w}", ("dQ", go), "dQ warps")
             m.bars[f"dqe{b}"].arrive()
             go += 1
 
@@ -194,15 +206,21 @@ def run(items, seed):
     m = Machine()
     for b in range(2):
         m.bar(f"itf{b}")
-        m.bar(f"ite{b}", 3)  # MMA issuer, key rows, dQ warps (one arrival per role here)
-        for name in ("kf", "ke", "dqf", "dqe", "wb", "pb"):
+        m.bar(f"ite{b}", 1 + ROWS + DQW)  # each consumer warp acknowledges an item
+        for name in ("kf", "ke", "dqf", "wb"):
             m.bar(f"{name}{b}")
+        m.bar(f"dqe{b}", DQW)
+        m.bar(f"pb{b}", ROWS)
     for st in range(NQS):
         m.bar(f"qf{st}")
         m.bar(f"qe{st}")
-    for name in ("vf", "ve", "s", "dp", "p", "ds", "acc", "acr"):
+    for name in ("vf", "ve", "s", "dp", "acc"):
         m.bar(name)
-    roles = {"producer": producer(m, items), "mma": mma_issuer(m), "rows": key_rows(m), "dq": dq_warps(m)}
+    for name in ("p", "ds", "acr"):
+        m.bar(name, ROWS)
+    roles = {"producer": producer(m, items), "mma": mma_issuer(m)}
+    roles.update({f"rows{w}": key_rows(m, w) for w in range(ROWS)})
+    roles.update({f"dq{w}": dq_warp(m, w) for w in range(DQW)})
     simulate(m, roles, random.Random(seed))
 
 
@@ -214,7 +232,7 @@ def random_items(rng, max_tiles=5):
 def test_random_item_sequences_and_schedules(seed):
     rng = random.Random(1000 + seed)
     items = random_items(rng)
-    for sched in range(25):
+    for sched in range(10):
         run(items, seed * 100 + sched)
 
 
@@ -230,7 +248,7 @@ def test_edge_sequences():
         [(True, 5), (True, 4), (False, 2), (True, 1)],
     ]
     for i, items in enumerate(cases):
-        for sched in range(40):
+        for sched in range(20):
             run(items, 7000 + 100 * i + sched)
 
 

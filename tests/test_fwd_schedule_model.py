@@ -1,7 +1,8 @@
 """A model of the synchronization protocol of the persistent forward kernel
 (`csrc/saf_fwd_tc.cu`), checked under random schedules.
 
-The roles (TMA producer, MMA issuer, query-row warps) perform the kernel's
+The roles (TMA producer, MMA issuer, each of the 4 query-row warps with the
+kernel's arrival counts and its own lane quarter of S, P and O) perform the kernel's
 barrier operations in its order and with its phase parities (machinery in
 tests/schedule_model.py).  Resources: Q in two buffers (this item, the next),
 K and V rings of two stages each (K loaded one block ahead of V), the S
@@ -17,6 +18,12 @@ import pytest
 from tests.schedule_model import Machine, ModelError, W, mutate, publish, simulate, take
 
 NSK = NSV = 2  # K, V ring stages
+ROWS = 4       # query-row warps: each owns one lane quarter of S, P and O
+
+
+def all_of(res, version):
+    """A region the MMA reads or writes whole: every warp's slice."""
+    return [(f"{res}.{w}", version) for w in range(ROWS)]
 
 
 def producer(m, items):
@@ -66,7 +73,8 @@ def mma_issuer(m):
             g = gk + j
             s, u = g % NSK, g // NSK
             yield W(f"kf{s}", u, u & 1)
-            m.mma([(f"Q{b}", ("Q", nq)), (f"K{s}", ("K", g))], [("S_lo", ("S", go + j)), ("S_hi", ("S", go + j))], "S")
+            m.mma([(f"Q{b}", ("Q", nq)), (f"K{s}", ("K", g))],
+                  all_of("S_lo", ("S", go + j)) + all_of("S_hi", ("S", go + j)), "S")
             m.commit("s")
             m.commit(f"ke{s}")
             if j == nkb - 1:
@@ -85,12 +93,12 @@ def mma_issuer(m):
             wb = (gr + j) & 1
             if rep:
                 yield W(f"pb{wb}", (gr + j) >> 1, ((gr + j) >> 1) & 1)
-                a = ("S_lo" if wb == 0 else "S_hi", ("W", gr + j))
+                a = all_of("S_lo" if wb == 0 else "S_hi", ("W", gr + j))
             else:
                 yield W("p", go + j, (go + j) & 1)
-                a = ("P", ("P", go + j))
-            acc_in = [("O", ("O", n, j - 1))] if j > 0 else []
-            m.mma([a, (f"V{s}", ("V", g))] + acc_in, [("O", ("O", n, j))], "P.V")
+                a = all_of("P", ("P", go + j))
+            acc_in = all_of("O", ("O", n, j - 1)) if j > 0 else []
+            m.mma(a + [(f"V{s}", ("V", g))] + acc_in, all_of("O", ("O", n, j)), "P.V")
             m.commit(f"ob{wb}" if rep else "o")
             m.commit(f"ve{s}")
         if rep:
@@ -103,7 +111,7 @@ def mma_issuer(m):
         n += 1
 
 
-def query_rows(m):
+def query_rows(m, w):
     go = gr = 0
     n = 0
     while True:
@@ -114,27 +122,27 @@ def query_rows(m):
         for j in range(nkb):
             if not rep:
                 yield W("s", go + j, (go + j) & 1)
-                m.read("S_lo", ("S", go + j), "rows")
-                m.read("S_hi", ("S", go + j), "rows")
+                m.read(f"S_lo.{w}", ("S", go + j), "rows")
+                m.read(f"S_hi.{w}", ("S", go + j), "rows")
                 m.bars["sf"].arrive()
                 if j > 0:
                     yield W("o", go + j - 1, (go + j - 1) & 1)
-                    m.read("O", ("O", n, j - 1), "rows rescale")
-                    m.write("O", ("O", n, j - 1), "rows rescale")
-                m.write("P", ("P", go + j), "rows")
+                    m.read(f"O.{w}", ("O", n, j - 1), "rows rescale")
+                    m.write(f"O.{w}", ("O", n, j - 1), "rows rescale")
+                m.write(f"P.{w}", ("P", go + j), "rows")
                 m.bars["p"].arrive()
             else:
                 g = gr + j
                 if g >= 2:
                     yield W(f"ob{g & 1}", (g >> 1) - 1, ((g >> 1) & 1) ^ 1)
-                m.write("S_lo" if g % 2 == 0 else "S_hi", ("W", g), "rows W")
+                m.write(f"{'S_lo' if g % 2 == 0 else 'S_hi'}.{w}", ("W", g), "rows W")
                 m.bars[f"pb{g & 1}"].arrive()
         gl = (gr if rep else go) + nkb - 1  # the item's last P.V
         if rep:
             yield W(f"ob{gl & 1}", gl >> 1, (gl >> 1) & 1)
         else:
             yield W("o", gl, gl & 1)
-        m.read("O", ("O", n, nkb - 1), "rows epilogue")
+        m.read(f"O.{w}", ("O", n, nkb - 1), "rows epilogue")
         if rep:
             gr += nkb
         else:
@@ -146,18 +154,22 @@ def run(items, seed):
     m = Machine()
     for b in range(2):
         m.bar(f"itf{b}")
-        m.bar(f"ite{b}", 2)  # MMA issuer and row warps (one arrival per role here)
-        for name in ("qf", "qe", "ob", "pb"):
+        m.bar(f"ite{b}", 1 + ROWS)  # the MMA warp and each row warp acknowledge an item
+        for name in ("qf", "qe", "ob"):
             m.bar(f"{name}{b}")
+        m.bar(f"pb{b}", ROWS)
     for s in range(NSK):
         m.bar(f"kf{s}")
         m.bar(f"ke{s}")
     for s in range(NSV):
         m.bar(f"vf{s}")
         m.bar(f"ve{s}")
-    for name in ("s", "sf", "p", "o"):
+    for name in ("s", "o"):
         m.bar(name)
-    roles = {"producer": producer(m, items), "mma": mma_issuer(m), "rows": query_rows(m)}
+    for name in ("sf", "p"):
+        m.bar(name, ROWS)
+    roles = {"producer": producer(m, items), "mma": mma_issuer(m)}
+    roles.update({f"rows{w}": query_rows(m, w) for w in range(ROWS)})
     simulate(m, roles, random.Random(seed))
 
 
@@ -169,7 +181,7 @@ def random_items(rng, max_blocks=5):
 def test_random_item_sequences_and_schedules(seed):
     rng = random.Random(2000 + seed)
     items = random_items(rng)
-    for sched in range(25):
+    for sched in range(15):
         run(items, seed * 100 + sched)
 
 
