@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--grad-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the extra keys (per_config, head_cost) after the headline timing")
     ap.add_argument("--head-cost", action="store_true",
                     help="instead of the headline line, time the workload's shape with 0, 25, 50 and 100%% of "
                          "the heads replaced and fit t = t0 + c_o n_o + c_r n_r per pass")
@@ -285,6 +287,137 @@ def algorithmic_flops_per_launch(kernel: str, w, n_r: int) -> float:
     return table.get(kernel, 0.0)
 
 
+def device_inputs(w, dev, seed=0):
+    """Inputs of workload w drawn on the GPU with the recipe's distributions
+    (Q, K, V, dO standard normal rounded to bf16; the pattern vectors and the
+    replaced heads exactly as in the seeded recipe).  Used only for timing the
+    extra shapes, where building the seeded CPU tensors would take minutes."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + seed)
+    x = {}
+    for name in ("q", "k", "v") + (("do",) if w.backward else ()):
+        x[name] = torch.randn(w.B, w.H, w.T, w.d, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    a, r = I.make_pattern(w, seed)
+    x["alpha"], x["rho"] = a.to(dev), r.to(dev)
+    x["mask"] = I.replaced_mask(w, seed)
+    return x
+
+
+def _event_ms(fn, reps, stream):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def time_passes(w, dev, x, reps, gd=torch.bfloat16):
+    """Device time of each pass of the layer on workload w (inputs resident):
+    log Z, forward, backward, and the whole step (log Z + forward + backward,
+    as the headline step), each the mean of `reps` back-to-back calls after
+    two warm-up calls."""
+    from mixed_head_causal_b200 import saf
+    stream = torch.cuda.current_stream(dev)
+    mask = x["mask"]
+    n_r = int(mask.sum())
+    o = torch.empty(w.B, w.H, w.T, w.d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
+    logz = torch.zeros(w.H, w.T, dtype=torch.float32, device=dev)
+    lz = logz if n_r else None
+    ws_f = saf.new_workspace(w.B, w.H, w.T, dev, backward=False)
+    grads = None
+    ws_b = None
+    if w.backward:
+        grads = [torch.empty(w.B, w.H, w.T, w.d, dtype=gd, device=dev) for _ in range(3)]
+        ws_b = saf.new_workspace(w.B, w.H, w.T, dev, backward=True)
+
+    def ln():
+        if n_r:
+            saf.replaced_lognorm(x["alpha"], x["rho"], mask, out=logz)
+
+    def fwd():
+        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, logz=lz, out=o, lse=lse,
+                           workspace=ws_f)
+
+    def bwd():
+        saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask, logz=lz,
+                           grad_dtype=gd, dq=grads[0], dk=grads[1], dv=grads[2], workspace=ws_b)
+
+    def step():
+        ln()
+        fwd()
+        if w.backward:
+            bwd()
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    out = {"lognorm_ms": _event_ms(ln, reps, stream) if n_r else 0.0, "fwd_ms": _event_ms(fwd, reps, stream)}
+    if w.backward:
+        out["bwd_ms"] = _event_ms(bwd, reps, stream)
+    out["step_ms"] = _event_ms(step, reps, stream)
+    del o, lse, logz, ws_f, grads, ws_b
+    return out
+
+
+def rates(w, t, pk):
+    """tokens/s, TFLOP/s and fraction of the peak of one timed shape."""
+    fl = I.flops(w)
+    res = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "n_replaced": len(I.replaced_heads(w)),
+           "passes": "fwd+bwd" if w.backward else "fwd"}
+    res.update({k: round(v, 5) for k, v in t.items()})
+    res["tokens_per_s"] = w.tokens / (t["step_ms"] * 1e-3)
+    res["tflops"] = fl["total"] / (t["step_ms"] * 1e-3) / 1e12
+    res["frac_of_peak"] = res["tflops"] / pk["bf16_tflops"]
+    res["fwd_tflops"] = fl["fwd"] / (t["fwd_ms"] * 1e-3) / 1e12
+    if w.backward:
+        res["bwd_tflops"] = fl["bwd"] / (t["bwd_ms"] * 1e-3) / 1e12
+    return res
+
+
+def per_config(dev, pk, reps=10):
+    """The other measured shapes of the layer: the 50%-replaced 124M shape at
+    8K, the 1B-scale shape, and the batch-64 / T=4096 prefill sweep (forward
+    only); each with its pass split."""
+    out = {}
+    names = ["124m_b4_t8192_r50", "1b_b4_h32_t8192_r25"] + list(I.PREFILL_SWEEP)
+    for name in names:
+        w = I.WORKLOADS[name]
+        x = device_inputs(w, dev)
+        t = time_passes(w, dev, x, reps if w.T * w.B <= 64 * 4096 else max(3, reps // 2))
+        out[name] = rates(w, t, pk)
+        del x
+        torch.cuda.empty_cache()
+    return out
+
+
+def head_cost_fit(base, dev, reps=10):
+    """Per-head cost of each head kind on the shape of `base`: n_r = 0, H/4,
+    H/2 and H replaced heads (the first n_r), forward and backward timed
+    separately, and the least-squares fit t = t0 + c_o n_o + c_r n_r."""
+    import numpy as np
+    rows = []
+    for n_r in sorted({0, base.H // 4, base.H // 2, base.H}):
+        w = I.custom(base.B, base.H, base.T, list(range(n_r)))
+        x = device_inputs(w, dev)
+        t = time_passes(w, dev, x, reps)
+        rows.append((w.H - n_r, n_r, t["fwd_ms"], t["bwd_ms"]))
+        del x
+        torch.cuda.empty_cache()
+    A = np.array([[1.0, r[0], r[1]] for r in rows])
+    out = {"config": {"workload": base.name, "B": base.B, "H": base.H, "T": base.T,
+                      "n_replaced_points": [r[1] for r in rows]},
+           "times_ms": [{"n_o": r[0], "n_r": r[1], "fwd": r[2], "bwd": r[3]} for r in rows]}
+    for name, col in (("fwd", 2), ("bwd", 3), ("fwd+bwd", None)):
+        y = np.array([r[2] + r[3] if col is None else r[col] for r in rows])
+        t0, c_o, c_r = np.linalg.lstsq(A, y, rcond=None)[0]
+        out[name] = {"t0_ms": float(t0), "c_o_ms": float(c_o), "c_r_ms": float(c_r),
+                     "c_r_over_c_o": float(c_r / c_o) if c_o else None}
+    return out
+
+
 def our_arm(args, world, rank, local):
     from mixed_head_causal_b200 import saf
     if not torch.cuda.is_available():
@@ -415,6 +548,15 @@ def our_arm(args, world, rank, local):
         e2e = {"value": tokens / (e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
+    # ---- the pass split of the headline shape, the other shapes and the
+    # per-head cost (separate timings after the headline; milliseconds each)
+    split = rates(w, time_passes(w, dev, x, 20, gd), pk)
+    extra, hc = None, None
+    if rank == 0 and not args.no_extra:
+        extra = per_config(dev, pk)
+        if w.backward and n_r:
+            hc = head_cost_fit(w, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
@@ -428,65 +570,17 @@ def our_arm(args, world, rank, local):
             "config": arm_config(w, world, args.grad_dtype),
             "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
             "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
+            "passes": split, "per_config": extra, "head_cost": hc,
         }
         print(json.dumps(line), flush=True)
 
 
 def head_cost(args, local):
-    """Per-head cost of each head kind: the workload's shape timed with
-    n_r = 0, H/4, H/2 and H replaced heads (the first n_r heads), forward and
-    backward separately, and a least-squares fit t = t0 + c_o n_o + c_r n_r."""
-    import numpy as np
-    from mixed_head_causal_b200 import saf
+    """Per-head cost of each head kind (the head_cost key of the headline
+    line, printed alone)."""
     dev = torch.device("cuda", local)
-    base = I.WORKLOADS[args.workload]
-    rows = []
-    for n_r in sorted({0, base.H // 4, base.H // 2, base.H}):
-        w = I.custom(base.B, base.H, base.T, list(range(n_r)))
-        x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
-        mask = x["mask"]
-        lz = torch.zeros(w.H, w.T, dtype=torch.float32, device=dev)
-        if n_r:
-            saf.replaced_lognorm(x["alpha"], x["rho"], mask, out=lz)
-        lzp = lz if n_r else None
-        o = torch.empty_like(x["v"])
-        lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
-        g = [torch.empty_like(x["v"]) for _ in range(3)]
-        wsf = saf.new_workspace(w.B, w.H, w.T, dev, backward=False)
-        wsb = saf.new_workspace(w.B, w.H, w.T, dev, backward=True)
-
-        def fwd():
-            saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, logz=lzp, out=o, lse=lse,
-                               workspace=wsf)
-
-        def bwd():
-            saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask, logz=lzp,
-                               dq=g[0], dk=g[1], dv=g[2], workspace=wsb)
-
-        times = {}
-        for name, fn in (("fwd", fwd), ("bwd", bwd)):
-            for _ in range(3):
-                fn()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize()
-            e0.record()
-            for _ in range(args.steps):
-                fn()
-            e1.record()
-            torch.cuda.synchronize()
-            times[name] = e0.elapsed_time(e1) / args.steps
-        rows.append((w.H - n_r, n_r, times["fwd"], times["bwd"]))
-        del x, o, lse, g, wsf, wsb
-        torch.cuda.empty_cache()
-    A = np.array([[1.0, r[0], r[1]] for r in rows])
-    out = {"metric": "per-head cost of ordinary vs replaced heads (ms per head per step)",
-           "config": {"workload": args.workload, "B": base.B, "H": base.H, "T": base.T, "d_h": base.d,
-                      "n_replaced_points": [r[1] for r in rows]},
-           "times_ms": [{"n_o": r[0], "n_r": r[1], "fwd": r[2], "bwd": r[3]} for r in rows]}
-    for name, col in (("fwd", 2), ("bwd", 3), ("fwd+bwd", None)):
-        y = np.array([r[2] + r[3] if col is None else r[col] for r in rows])
-        t0, c_o, c_r = np.linalg.lstsq(A, y, rcond=None)[0]
-        out[name] = {"t0_ms": t0, "c_o_ms": c_o, "c_r_ms": c_r, "c_r_over_c_o": c_r / c_o if c_o else None}
+    out = {"metric": "per-head cost of ordinary vs replaced heads (ms per head per step)"}
+    out.update(head_cost_fit(I.WORKLOADS[args.workload], dev, reps=args.steps))
     print(json.dumps(out), flush=True)
 
 
