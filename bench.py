@@ -5,9 +5,10 @@
                     [--impl ours|reference]
 
 One step is the whole hot path on one batch, all through the C ABI with the
-inputs resident in HBM: the replaced heads' log-normalisers (computed once
-per step and reused by both passes, like lse), the forward call and the
-backward call (row terms, fused backward, dQ conversion).
+inputs resident in HBM: the forward call (the replaced heads' pattern
+preparation -- log-normalisers and factored arrays -- in one launch, then the
+fused forward) and the backward call (row terms with the pattern preparation
+in one launch, the fused backward, the dQ conversion).
 Default workload: the 124M-shape layer B=8, H=12 (3 replaced), T=4096,
 d_h=64, forward + backward.
 
@@ -315,17 +316,14 @@ def _event_ms(fn, reps, stream):
 
 def time_passes(w, dev, x, reps, gd=torch.bfloat16):
     """Device time of each pass of the layer on workload w (inputs resident):
-    log Z, forward, backward, and the whole step (log Z + forward + backward,
-    as the headline step), each the mean of `reps` back-to-back calls after
-    two warm-up calls."""
+    forward, backward (each with its pattern preparation), and the whole step
+    (forward + backward, as the headline step), each the mean of `reps`
+    back-to-back calls after two warm-up calls."""
     from mixed_head_causal_b200 import saf
     stream = torch.cuda.current_stream(dev)
     mask = x["mask"]
-    n_r = int(mask.sum())
     o = torch.empty(w.B, w.H, w.T, w.d, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
-    logz = torch.zeros(w.H, w.T, dtype=torch.float32, device=dev)
-    lz = logz if n_r else None
     ws_f = saf.new_workspace(w.B, w.H, w.T, dev, backward=False)
     grads = None
     ws_b = None
@@ -333,20 +331,14 @@ def time_passes(w, dev, x, reps, gd=torch.bfloat16):
         grads = [torch.empty(w.B, w.H, w.T, w.d, dtype=gd, device=dev) for _ in range(3)]
         ws_b = saf.new_workspace(w.B, w.H, w.T, dev, backward=True)
 
-    def ln():
-        if n_r:
-            saf.replaced_lognorm(x["alpha"], x["rho"], mask, out=logz)
-
     def fwd():
-        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, logz=lz, out=o, lse=lse,
-                           workspace=ws_f)
+        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, out=o, lse=lse, workspace=ws_f)
 
     def bwd():
-        saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask, logz=lz,
+        saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask,
                            grad_dtype=gd, dq=grads[0], dk=grads[1], dv=grads[2], workspace=ws_b)
 
     def step():
-        ln()
         fwd()
         if w.backward:
             bwd()
@@ -354,11 +346,11 @@ def time_passes(w, dev, x, reps, gd=torch.bfloat16):
     for _ in range(2):
         step()
     torch.cuda.synchronize()
-    out = {"lognorm_ms": _event_ms(ln, reps, stream) if n_r else 0.0, "fwd_ms": _event_ms(fwd, reps, stream)}
+    out = {"fwd_ms": _event_ms(fwd, reps, stream)}
     if w.backward:
         out["bwd_ms"] = _event_ms(bwd, reps, stream)
     out["step_ms"] = _event_ms(step, reps, stream)
-    del o, lse, logz, ws_f, grads, ws_b
+    del o, lse, ws_f, grads, ws_b
     return out
 
 
@@ -440,18 +432,13 @@ def our_arm(args, world, rank, local):
     ws_b = saf.new_workspace(B, H, T, dev, backward=True) if w.backward else None
     stream = torch.cuda.current_stream(dev)
 
-    logz = torch.zeros(H, T, dtype=torch.float32, device=dev)
-
     def step():
-        # one training step of the layer: the replaced heads' log-normalisers
-        # once (the backward reuses them, like lse), then forward and backward
-        if n_r:
-            saf.replaced_lognorm(x["alpha"], x["rho"], mask, out=logz)
-        lz = logz if n_r else None
-        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, logz=lz, out=o, lse=lse,
-                           workspace=ws_f)
+        # one training step of the layer: forward and backward, each preparing
+        # the replaced heads' patterns (log Z and the factored arrays) in its
+        # first launch
+        saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask, out=o, lse=lse, workspace=ws_f)
         if w.backward:
-            saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask, logz=lz,
+            saf.mixed_attn_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, x["alpha"], x["rho"], mask,
                                grad_dtype=gd, dq=dq, dk=dk, dv=dv, workspace=ws_b)
 
     torch.cuda.synchronize()

@@ -128,23 +128,23 @@ saf_status saf_mixed_attn_fwd_gqa(const void* q, const void* k, const void* v, v
 
     cudaStream_t s = (cudaStream_t)stream;
     char* ws = static_cast<char*>(workspace);
-    const float* lz = logz;
-    if (hl.n > 0 && lz == nullptr) {
-        float* lzw = reinterpret_cast<float*>(ws + L.logz);
-        cudaError_t e = launch_lognorm(a, r, hl, T, lzw, s);
-        if (e != cudaSuccess) return SAF_ERR_CUDA;
-        lz = lzw;
-    }
+    // log Z: the caller's, or computed into the workspace
+    float* lzw = reinterpret_cast<float*>(ws + L.logz);
+    const float* lz = logz ? logz : lzw;
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
     const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
     __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
     if (force_mma_path()) {
         if (H_kv != H) return SAF_ERR_UNSUPPORTED;  // the warp-level path has no shared K/V
+        if (hl.n > 0 && !logz && launch_lognorm(a, r, hl, T, lzw, s) != cudaSuccess) return SAF_ERR_CUDA;
         return cuda_status(launch_fwd_mma(qb, kb, vb, ob, lse, a, r, lz, hl, B, H, T, s));
     }
+    // one launch prepares the replaced heads' patterns (log Z and the factored
+    // arrays), one runs the layer
     const ReplacedWs rw = replaced_ws(ws, L, T);
-    if (hl.n > 0 && launch_prep_replaced(a, r, lz, hl, T, rw, s) != cudaSuccess) return SAF_ERR_CUDA;
+    if (hl.n > 0 && launch_pattern(a, r, logz, logz ? nullptr : lzw, hl, T, &rw, s) != cudaSuccess)
+        return SAF_ERR_CUDA;
     cudaError_t e =
         launch_fwd_tc(qb, kb, vb, ob, lse, a, r, lz, hl, rw, B, H, H_kv, T, reinterpret_cast<unsigned int*>(ws), s);
     if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
@@ -188,12 +188,9 @@ saf_status saf_mixed_attn_bwd_gqa(const void* q, const void* k, const void* v, c
 
     cudaStream_t s = (cudaStream_t)stream;
     char* ws = static_cast<char*>(workspace);
-    const float* lz = logz;
-    if (hl.n > 0 && lz == nullptr) {
-        float* lzw = reinterpret_cast<float*>(ws + L.logz);
-        if (launch_lognorm(a, r, hl, T, lzw, s) != cudaSuccess) return SAF_ERR_CUDA;
-        lz = lzw;
-    }
+    // log Z: the caller's, or computed into the workspace
+    float* lzw = reinterpret_cast<float*>(ws + L.logz);
+    const float* lz = logz ? logz : lzw;
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
     const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
@@ -201,17 +198,21 @@ saf_status saf_mixed_attn_bwd_gqa(const void* q, const void* k, const void* v, c
     const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
     if (force_mma_path()) {
         if (H_kv != H) return SAF_ERR_UNSUPPORTED;  // the warp-level path has no shared K/V
+        if (hl.n > 0 && !logz && launch_lognorm(a, r, hl, T, lzw, s) != cudaSuccess) return SAF_ERR_CUDA;
         float* dvec = reinterpret_cast<float*>(ws + L.dvec);
         if (launch_bwd_dot(ob, dob, dvec, hl, B, H, T, s) != cudaSuccess) return SAF_ERR_CUDA;
         return cuda_status(launch_bwd_mma(qb, kb, vb, dob, lse, dvec, a, r, lz, hl, B, H, T, dq, dk, dv,
                                           grad_dtype, s));
     }
     const ReplacedWs rw = replaced_ws(ws, L, T);
-    if (hl.n > 0 && launch_prep_replaced(a, r, lz, hl, T, rw, s) != cudaSuccess) return SAF_ERR_CUDA;
     float* nlse2p = reinterpret_cast<float*>(ws + L.nlse2p);
     float* dvecp = reinterpret_cast<float*>(ws + L.dvecp);
     float* dqacc = reinterpret_cast<float*>(ws + L.dqacc);
-    if (launch_bwd_pre(ob, dob, lse, B * H, T, nlse2p, dvecp, dqacc, s) != cudaSuccess) return SAF_ERR_CUDA;
+    // one launch: the row terms, the zeroed dQ accumulator and counters, and
+    // the replaced heads' patterns
+    if (launch_bwd_pre(ob, dob, lse, B * H, T, nlse2p, dvecp, dqacc, a, r, logz, logz ? nullptr : lzw, hl, rw,
+                       s) != cudaSuccess)
+        return SAF_ERR_CUDA;
     // shared K/V: per-query-head fp32 dK, dV into the workspace, then summed per group
     const bool grouped = H_kv != H;
     float* dkh = grouped ? reinterpret_cast<float*>(ws + L.dkh) : nullptr;

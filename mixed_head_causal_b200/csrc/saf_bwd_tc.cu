@@ -62,7 +62,8 @@ constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;
 constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;        // NQS x 512 B: -lse2 (ordinary) / r (replaced)
 constexpr uint32_t SM_VEC2 = SM_VEC1 + 512 * NQS;  // NQS x 512 B: D
 constexpr uint32_t SM_BAR = SM_VEC2 + 512 * NQS;
-constexpr uint32_t SM_TOTAL = SM_BAR + 256;
+constexpr uint32_t SM_DFL = SM_BAR + 256;  // per replaced slot: 1 = per-element path
+constexpr uint32_t SM_TOTAL = SM_DFL + 256;
 
 struct BwdTcParams {
     const float* nlse2p;
@@ -76,6 +77,7 @@ struct BwdTcParams {
     unsigned int* err;
     int16_t slot_of_head[kMaxHeads];
     int H, Hkv, BH, T, Tp, nqb, grad_fp32;  // Hkv: K/V heads (H / Hkv query heads share one)
+    int nslots;  // replaced heads
     float scale, scale_log2;
 };
 
@@ -233,6 +235,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
         tmem_relinquish();
     }
+    uint8_t* dfl = smem + SM_DFL;
+    if (warp == 0) slot_flags(p.w, p.nslots, dfl);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -254,7 +258,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         int bh, bhkv, J, h, slot, ntiles;  // query slice, its K/V slice, key block, head, replaced slot, tiles
         bool rep, direct, ragged;
     };
-    auto decode = [&](int item) {
+    // the published item word carries the head's per-element flag in bit 30
+    // (set by the producer from the per-slot flags)
+    auto decode = [&](int word) {
+        const int item = word & 0x3fffffff;
         Item it;
         grouped_order((unsigned)item, p.BH, p.nqb, it.bh, it.J);
         it.h = it.bh % p.H;
@@ -263,7 +270,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         it.rep = it.slot >= 0;
         // a replaced head whose factors would leave fp32 range takes P^T itself
         // (one exp per element) in place of W^T, and its dV rows need no c_j
-        it.direct = it.rep && p.w.flag[it.h] != 0;
+        it.direct = it.rep && ((word >> 30) & 1) != 0;
         it.ntiles = p.nqb - it.J;
         it.ragged = (it.J + 1) * BN > T;  // the key block runs past T
         return it;
@@ -280,7 +287,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bool ok = true;
             for (int n = 0; ok; ++n) {
                 const int w = (int)atomicAdd(p.err + kCtrBwdNext, 1u);
-                const int item = w < total ? w : -1;
+                int item = w < total ? w : -1;
+                if (item >= 0) {
+                    const Item pre = decode(item);
+                    if (pre.rep && dfl[pre.slot]) item |= 1 << 30;
+                }
                 if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                 *reinterpret_cast<volatile int*>(item_slot + (n & 1)) = item;
                 mbar_arrive(bar_itf + 8 * (n & 1));
@@ -750,43 +761,6 @@ __global__ void __launch_bounds__(256) group_sum_kernel(const float* __restrict_
     }
 }
 
-// rows of [BH, Tp]: -lse2 = -lse*log2(e) (-inf past T), D = rowsum(dO o O) (0
-// past T); zero the dQ accumulator rows.  8 threads per row.
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
-                                                      const __nv_bfloat16* __restrict__ dout,
-                                                      const float* __restrict__ lse, int T, int Tp, int64_t rows,
-                                                      float* __restrict__ nlse2p, float* __restrict__ dvecp,
-                                                      float* __restrict__ dqacc) {
-    const int64_t r = (int64_t)blockIdx.x * 32 + (threadIdx.x >> 3);
-    const int part = threadIdx.x & 7;
-    if (r >= rows) return;
-    const int64_t bh = r / Tp;
-    const int i = (int)(r - bh * Tp);
-    float acc = 0.f;
-    if (i < T) {
-        const int64_t row = bh * T + i;
-        const uint4 ov = *reinterpret_cast<const uint4*>(o + row * kHeadDim + part * 8);
-        const uint4 dv = *reinterpret_cast<const uint4*>(dout + row * kHeadDim + part * 8);
-        const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 a = unpack_bf16x2(ow[e]), b = unpack_bf16x2(dw[e]);
-            acc = fmaf(a.x, b.x, acc);
-            acc = fmaf(a.y, b.y, acc);
-        }
-        float4* z = reinterpret_cast<float4*>(dqacc + row * kHeadDim + part * 8);
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-    if (part == 0) {
-        dvecp[r] = i < T ? acc : 0.f;
-        nlse2p[r] = i < T ? -lse[bh * T + i] * kLog2e : kNegInf;
-    }
-}
-
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc, void* __restrict__ dq,
                                                          int64_t n4, int grad_fp32, float scale) {
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n4;
@@ -828,17 +802,6 @@ bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out) {
     return fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int BH, int T,
-                           float* nlse2p, float* dvecp, float* dqacc, cudaStream_t stream) {
-    const int Tp = round_up128(T);
-    const int64_t rows = (int64_t)BH * Tp;
-    if (rows == 0) return cudaSuccess;
-    launch_begin(KID_BWD_PRE, stream);
-    bwd_pre_kernel<<<(unsigned)((rows + 31) / 32), 256, 0, stream>>>(o, dout, lse, T, Tp, rows, nlse2p, dvecp, dqacc);
-    launch_end(KID_BWD_PRE, stream);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream) {
@@ -889,12 +852,14 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     for (int hh = 0; hh < kMaxHeads; ++hh) p.slot_of_head[hh] = -1;
     for (int hh = 0; hh < H; ++hh)
         if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
+    p.nslots = slot;
     p.H = H;
     p.Hkv = Hkv;
     p.BH = BH;
     p.T = T;
     p.Tp = round_up128(T);
     p.nqb = (T + BM - 1) / BM;
+    if ((int64_t)BH * p.nqb >= (int64_t)1 << 30) return cudaErrorNotSupported;  // item words hold 30 bits
     p.grad_fp32 = grad_fp32;
     p.scale = 0.125f;
     p.scale_log2 = kLog2e * 0.125f;

@@ -33,15 +33,31 @@ struct Shape {
 // saf_prep.cu), one row per replaced-head slot s (slot order = head order).
 struct ReplacedWs {
     int Tp, Lp;          // T rounded up to 128; Tp + 256
+    int ntiles;          // 32-row tiles of a head: ceil(T / 32)
     uint32_t* epair;     // [slots][Lp]   bf16 pairs {E[x], E[x-1]} at x + 128
     float* ef;           // [slots][Lp]   fp32 E[x] at x + 128
     uint32_t* cpair;     // [slots][Tp/2] bf16 pairs {c[2m], c[2m+1]}
     float* cf;           // [slots][Tp]   fp32 c[j]
     float* rsc;          // [slots][Tp]   fp32 r_i
-    int* flag;           // [H] 1 = head needs the per-element exp path
+    int* tflag;          // [slots][ntiles] 1 = a row of the tile needs the per-element
+                         // exp path (a head takes it when any of its tiles does)
 };
 
 __host__ __device__ inline int round_up128(int x) { return (x + 127) & ~127; }
+
+// Per replaced slot, whether the head takes the per-element path: the OR of
+// its tiles' range flags (written by the pattern preparation), into dfl[slot]
+// in shared memory.  Called by one warp; a barrier of the block must follow
+// before dfl is read.
+__device__ __forceinline__ void slot_flags(const ReplacedWs& w, int nslots, uint8_t* dfl) {
+    const int lane = threadIdx.x & 31;
+    for (int s = 0; s < nslots; ++s) {
+        int any = 0;
+        for (int t = lane; t < w.ntiles; t += 32) any |= w.tflag[(size_t)s * w.ntiles + t];
+        any = __any_sync(0xffffffffu, any != 0);
+        if (lane == 0) dfl[s] = (uint8_t)any;
+    }
+}
 
 // CTA order of the tensor-core kernels.  A CTA does one block-row of one
 // (batch, head) slice; its work shrinks with its causal rank (rank 0 = the
@@ -66,7 +82,7 @@ struct WsLayout {
     size_t header;   // device error word + counters (256 B)
     size_t logz;     // [H, T] fp32 (used when the caller passes logz = NULL)
     size_t dvec;     // [B, H, T] fp32 row terms rowsum(dO o O) (backward only)
-    size_t epair, ef, cpair, cf, rsc, flag;  // factored replaced-head arrays (H slots)
+    size_t epair, ef, cpair, cf, rsc, tflag;  // factored replaced-head arrays (H slots)
     size_t nlse2p;    // [B*H, Tp] fp32 -lse * log2(e), -inf past T  (backward)
     size_t dvecp;    // [B*H, Tp] fp32 rowsum(dO o O), 0 past T      (backward)
     size_t dqacc;    // [B*H, T, 64] fp32 dQ accumulator              (backward)
@@ -89,7 +105,7 @@ inline WsLayout ws_layout(int B, int H, int T, int is_bwd, int Hkv = -1) {
     L.cpair = off; off = align256(off + 4 * (size_t)H * (Tp / 2));
     L.cf = off; off = align256(off + 4 * (size_t)H * Tp);
     L.rsc = off; off = align256(off + 4 * (size_t)H * Tp);
-    L.flag = off; off = align256(off + 4 * (size_t)H);
+    L.tflag = off; off = align256(off + 4 * (size_t)H * (Tp / 32));
     if (is_bwd) {
         const size_t BH = (size_t)B * H;
         L.nlse2p = off; off = align256(off + 4 * BH * Tp);
@@ -113,7 +129,8 @@ inline ReplacedWs replaced_ws(char* ws, const WsLayout& L, int T) {
     w.cpair = reinterpret_cast<uint32_t*>(ws + L.cpair);
     w.cf = reinterpret_cast<float*>(ws + L.cf);
     w.rsc = reinterpret_cast<float*>(ws + L.rsc);
-    w.flag = reinterpret_cast<int*>(ws + L.flag);
+    w.ntiles = (T + 31) / 32;
+    w.tflag = reinterpret_cast<int*>(ws + L.tflag);
     return w;
 }
 
@@ -134,8 +151,8 @@ int sm_count();
 // ---------------------------------------------------------------- accounting
 // Kernel ids of the launch accounting (names in saf_profile.cu).
 enum KernelId {
-    KID_LOGNORM = 1, KID_FWD_MMA = 2, KID_DOT = 3, KID_DKDV_MMA = 4, KID_DQ_MMA = 5,
-    KID_FWD_TC = 6, KID_BWD_TC = 7, KID_PREP_REPLACED = 8, KID_DQ_CONVERT = 9, KID_BWD_PRE = 10,
+    KID_PATTERN = 1, KID_FWD_MMA = 2, KID_DOT = 3, KID_DKDV_MMA = 4, KID_DQ_MMA = 5,
+    KID_FWD_TC = 6, KID_BWD_TC = 7, /* 8: retired */ KID_DQ_CONVERT = 9, KID_BWD_PRE = 10,
     KID_GROUP_SUM = 11, KID_PATTERN_GRAD = 12, KID_CALIBRATION = 13, KID_FIT = 14
 };
 // Every kernel launch of the library is bracketed by these two calls.
@@ -144,10 +161,15 @@ void launch_end(int kid, cudaStream_t s);
 
 // ---------------------------------------------------------------- launchers
 // (defined in the kernel translation units; all enqueue on `stream`)
+// log Z of the replaced heads into logz [H, T] (the pattern preparation with
+// no factored arrays).
 cudaError_t launch_lognorm(const float* a, const float* r, const HeadList& hl, int T,
                            float* logz, cudaStream_t stream);
-cudaError_t launch_prep_replaced(const float* a, const float* r, const float* logz, const HeadList& hl, int T,
-                                 const ReplacedWs& w, cudaStream_t stream);
+// Pattern preparation of the replaced heads, one launch: log Z (taken from
+// logz_in, or computed and written to logz_out) and, when w is non-null, the
+// factored arrays and their range flags.
+cudaError_t launch_pattern(const float* a, const float* r, const float* logz_in, float* logz_out, const HeadList& hl,
+                           int T, const ReplacedWs* w, cudaStream_t stream);
 // Tensor-core forward of every head (replaced heads whose factored form would
 // leave fp32 range, flag 1, take per-element exps of a + r - log Z); returns
 // cudaErrorNotSupported when the tensor maps cannot be built.
@@ -156,12 +178,16 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
                           __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
                           const HeadList& hl, const ReplacedWs& w, int B, int H, int Hkv, int T, unsigned int* err,
                           cudaStream_t stream);
-// Backward preprocessing for the tensor-core backward: padded lse*log2(e) and
-// rowsum(dO o O), and a zeroed dQ accumulator.
+// Backward preprocessing for the tensor-core backward, one launch: padded
+// -lse*log2(e) and rowsum(dO o O), a zeroed dQ accumulator, and (hl.n > 0)
+// the replaced heads' pattern preparation (what launch_pattern does: log Z
+// from logz_in or into logz_out, and the factored arrays).
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int BH, int T,
-                           float* nlse2p, float* dvecp, float* dqacc, cudaStream_t stream);
+                           float* nlse2p, float* dvecp, float* dqacc, const float* a, const float* r,
+                           const float* logz_in, float* logz_out, const HeadList& hl, const ReplacedWs& w,
+                           cudaStream_t stream);
 // Tensor-core backward (dK, dV written; dQ reduced into dqacc); replaced
-// heads with flag 1 take per-element exps of a + r - log Z.
+// heads with the per-element flag take exps of a + r - log Z.
 // (dk, dv per query head: [B, H, T, 64]; with shared K/V the caller sums them
 // over each group with launch_group_sum)
 cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
@@ -186,10 +212,10 @@ cudaError_t launch_pattern_grad(const __nv_bfloat16* v, const __nv_bfloat16* dou
                                 const float* logz, const HeadList& hl, int B, int H, int T, float* da, float* dr,
                                 cudaStream_t stream);
 // dst[b, g] = sum of the H / Hkv fp32 rows src[b, h] of group g, [B, Hkv, T, 64] in the output dtype.
-cudaError_t launch_group_sum(const float* src, void* dst, int B, int H, int Hkv, int T, int grad_fp32,
-                             cudaStream_t stream);
 // dq = dqacc / sqrt(d_h) in the requested dtype.
 cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream);
+cudaError_t launch_group_sum(const float* src, void* dst, int B, int H, int Hkv, int T, int grad_fp32,
+                             cudaStream_t stream);
 bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out);
 bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out);
 // Warp-level (mma.sync) forward and backward of every head, the reference

@@ -4,7 +4,7 @@
 // One CTA computes one 128-row query block of one (batch, head) slice; both
 // head kinds share the grid, which is ordered longest rows first.  Warp roles:
 //   warp 0      TMA producer: Q once, then K and V tiles of 128 keys through
-//               separate rings (3 K stages, 2 V stages), K one block ahead of
+//               separate rings (2 K stages, 2 V stages), K one block ahead of
 //               V (K is skipped for replaced heads)
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2..5  one query row per thread: softmax / pattern builder, epilogue
@@ -20,8 +20,14 @@
 // order is S_0, S_1, PV_0, S_2, PV_1, ...
 // Replaced head (Eq. (3), section 二.3, in factored form): the tile
 //   W(i,j) = E[i-j] c_j     (bf16 pairs multiplied in registers, no exp)
-// is written to TMEM and O += W V_j; the epilogue scales row i by r_i, giving
-//   O_i = sum_j exp(a[j] + r[i-j] - log Z(i)) V_j.
+// is written to TMEM and O += W V_j; a second MMA against a tile of ones
+// accumulates the row sums of the same bf16 W, and the epilogue divides row i
+// by its sum.  Eq. (3) gives W(i,j) / sum_j W(i,j) = exp(a[j] + r[i-j] - log Z(i))
+// (the factors E, c and r_i cancel), so
+//   O_i = sum_j exp(a[j] + r[i-j] - log Z(i)) V_j,
+// and normalising by the sum of the rounded weights, as an ordinary head
+// normalises by the sum of its probabilities, reproduces a dominant term's V
+// exactly instead of scaling it by the rounding of its weight.
 // A replaced head whose factors would leave fp32 range (flag set by the prep
 // kernel) takes the pattern itself, one exp per element, in the same slot.
 // Causal tile skipping: key blocks past the diagonal are never visited; the
@@ -44,14 +50,21 @@ constexpr int NTHREADS = 192;
 constexpr uint32_t TILE_BYTES = 128 * 64 * 2;  // one 128 x 64 bf16 tile
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t TS_COL = 0, TO_COL = 128, TP_COL = 192;  // S, O, P regions
+// replaced heads: row sums of W in the (then unused) P columns 192..207
+constexpr uint32_t TSUM_COL = TP_COL;
 constexpr long long kWaitLimit = 1ll << 31;                 // cycles
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr uint32_t SM_Q = 0;
 constexpr uint32_t SM_K = SM_Q + 2 * TILE_BYTES;  // Q: two buffers (this item, next item)
 constexpr uint32_t SM_V = SM_K + NSK * TILE_BYTES;
-constexpr uint32_t SM_BAR = SM_V + NSV * TILE_BYTES;
-constexpr uint32_t SM_TOTAL = SM_BAR + 256;
+// 16 rows x 128 bytes of bf16 ones: the B operand (N = 16, K-major) of the
+// row-sum MMA of replaced heads (every element is 1, so each 16-key step
+// reads the same atom)
+constexpr uint32_t SM_ONES = SM_V + NSV * TILE_BYTES;
+constexpr uint32_t SM_BAR = SM_ONES + 2048;
+constexpr uint32_t SM_DFL = SM_BAR + 256;  // per replaced slot: 1 = per-element path
+constexpr uint32_t SM_TOTAL = SM_DFL + 256;
 
 struct FwdTcParams {
     __nv_bfloat16* o;
@@ -63,6 +76,7 @@ struct FwdTcParams {
     unsigned int* err;
     int16_t slot_of_head[kMaxHeads];
     int H, Hkv, BH, T, nqb;  // query heads, K/V heads (H / Hkv query heads share one)
+    int nslots;  // replaced heads
     float scale_log2;
 };
 
@@ -219,6 +233,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
         tmem_relinquish();
     }
+    if (warp == 0) {  // the ones tile (2 KB), 64 bytes per lane of the producer warp
+        const uint32_t one2 = 0x3F803F80u;  // two bf16 1.0
+#pragma unroll
+        for (int u = 0; u < 4; ++u) st_shared_v4(sbase + SM_ONES + (u * 32 + lane) * 16, one2, one2, one2, one2);
+        fence_proxy_async_smem();
+    }
+    uint8_t* dfl = smem + SM_DFL;
+    if (warp == 0) slot_flags(p.w, p.nslots, dfl);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -239,7 +261,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         int bh, bhkv, I, h, slot;  // query slice, its K/V slice, query block, head, replaced slot
         bool rep, direct;
     };
-    auto decode = [&](int item) {
+    // the published item word carries the head's per-element flag in bit 30
+    // (set by the producer from the per-slot flags)
+    auto decode = [&](int word) {
+        const int item = word & 0x3fffffff;
         Item it;
         int rank;
         grouped_order((unsigned)item, p.BH, p.nqb, it.bh, rank);
@@ -248,7 +273,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         it.bhkv = (it.bh / p.H) * p.Hkv + it.h / (p.H / p.Hkv);
         it.slot = p.slot_of_head[it.h];
         it.rep = it.slot >= 0;
-        it.direct = it.rep && p.w.flag[it.h] != 0;  // per-element exps instead of the factored form
+        it.direct = it.rep && ((word >> 30) & 1) != 0;  // per-element exps instead of the factored form
         return it;
     };
 
@@ -262,7 +287,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bool ok = true;
             for (int n = 0; ok; ++n) {
                 const int w = (int)atomicAdd(p.err + kCtrFwdNext, 1u);
-                const int item = w < total ? w : -1;
+                int item = w < total ? w : -1;
+                if (item >= 0) {
+                    const Item pre = decode(item);
+                    if (pre.rep && dfl[pre.slot]) item |= 1 << 30;
+                }
                 if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                 *reinterpret_cast<volatile int*>(item_slot + (n & 1)) = item;
                 mbar_arrive(bar_itf + 8 * (n & 1));
@@ -302,6 +331,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // ------------------------------------------------ MMA issuer
         const uint32_t idS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
         const uint32_t idO = idesc_bf16(128, 64, 0, 1);   // P (TMEM) x V (MN-major)
+        const uint32_t idSum = idesc_bf16(128, 16, 0, 0); // W (TMEM) x ones (K-major)
+        const uint64_t dOnes = sw128_desc(sbase + SM_ONES);
         // descriptors advance by stage (TILE_BYTES = TILE_BYTES / 16 units):
         // the issuing thread keeps its scalar work small, the pipe waits on it
         constexpr uint64_t kStage = TILE_BYTES >> 4;
@@ -362,6 +393,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                     for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
                         mma_ts(tmem + TO_COL, tmem + acol + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
+                    if (it.rep) {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)  // row sums of the same W
+                            mma_ts(tmem + TSUM_COL, tmem + acol + 8 * k, dOnes + 2 * (k & 3), idSum,
+                                   (j > 0 || k > 0) ? 1u : 0u);
+                    }
                     mma_commit(it.rep ? bar_ob + 8 * wb : bar_o);
                     mma_commit(bar_ve + 8 * s);
                 }
@@ -500,9 +537,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         scale = l > 0.f ? 1.f / l : 0.f;
                         lse_v = (m == kNegInf || l <= 0.f) ? kNegInf : (m + log2f(l)) * kLn2;
                     } else {
-                        scale = direct ? 1.f : p.w.rsc[(size_t)slot * p.w.Tp + i];
                         lse_v = p.logz[(size_t)h * T + i];
                     }
+                }
+                if (rep) {  // every row reads its W sum (a warp-wide TMEM load)
+                    const float sum = __uint_as_float(tmem_ld1(tmem + lane_off + TSUM_COL));
+                    tmem_wait_ld();
+                    scale = (i < T && sum > 0.f) ? 1.f / sum : 0.f;
                 }
                 __nv_bfloat16* orow = p.o + ((size_t)bh * T + (i < T ? i : 0)) * kHeadDim;
 #pragma unroll
@@ -617,11 +658,13 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     for (int hh = 0; hh < kMaxHeads; ++hh) p.slot_of_head[hh] = -1;
     for (int hh = 0; hh < H; ++hh)
         if (hl.replaced[hh]) p.slot_of_head[hh] = (int16_t)(slot++);
+    p.nslots = slot;
     p.H = H;
     p.Hkv = Hkv;
     p.BH = BH;
     p.T = T;
     p.nqb = (T + BM - 1) / BM;
+    if ((int64_t)BH * p.nqb >= (int64_t)1 << 30) return cudaErrorNotSupported;  // item words hold 30 bits
     p.scale_log2 = kLog2e / 8.0f;
     const int smem = SM_TOTAL + 1024;
     cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -22,8 +22,8 @@ struct Profile {
     int open = -1;  // index of the record whose stop event is pending
 } g_prof;
 
-const char* kNames[] = {"?", "lognorm", "fwd_mma", "dot", "dkdv_mma", "dq_mma",
-                        "fwd_tc", "bwd_tc", "prep_replaced", "dq_convert", "bwd_pre", "group_sum", "pattern_grad", "calibration", "fit"};
+const char* kNames[] = {"?", "pattern", "fwd_mma", "dot", "dkdv_mma", "dq_mma",
+                        "fwd_tc", "bwd_tc", "(retired)", "dq_convert", "bwd_pre", "group_sum", "pattern_grad", "calibration", "fit"};
 
 void release_locked() {
     for (auto& r : g_prof.recs) {

@@ -1,11 +1,16 @@
 """Shared helpers of the GPU-vs-oracle parity tests.
 
 The bar (stated once, used by every parity test):
-  * mean |gpu - oracle| <= 2e-2 / 10 = 2e-3 over every element of a tensor;
-  * element-wise |gpu - oracle| <= 2e-2 for fp32-stored results, and
-    <= 2e-2 + 2^-8 |oracle| for bf16-stored results (2^-8 |x| bounds the
-    rounding of x to bfloat16's 8-bit significand, a floor no kernel can go
-    under once the result is stored in bf16);
+  * mean |gpu - oracle| <= 2e-3 over every element of a tensor;
+  * element-wise |gpu - oracle| <= 2e-2 on O (stored in bf16) and on every
+    fp32-stored gradient, with nothing added for the storage rounding;
+  * bf16-stored gradients: the same bare 2e-2 whenever the storage floor
+    max |bf16(oracle) - oracle| of the compared tensor is at most 1e-2.  Above
+    that (long sums near key 0 of dK, dV reach |x| >= 4, where one bf16
+    half-ulp is already 1.6e-2) the bound is 2e-2 plus each element's own
+    rounding |bf16(oracle) - oracle|, and the strict gate on that workload is
+    carried by its fp32-gradient run, which every such test has beside it;
+    the floor is printed either way;
   * bit-exact zeros where the method fixes them (dQ, dK of replaced heads);
   * lse within 2e-3 (natural-log units).
 """
@@ -21,7 +26,7 @@ from mixed_head_causal_b200 import saf
 TOL_MAX = 2e-2
 TOL_MEAN = 2e-3
 TOL_LSE = 2e-3
-BF16_REL = 2.0 ** -8
+BF16_FLOOR_GATE = 1e-2  # storage floor above which a bf16 gradient's bound adds its rounding
 
 
 def to_gpu(x):
@@ -41,12 +46,27 @@ def run_layer(w, x, grad_dtype=torch.float32, backward=True):
     return {k: v.cpu() for k, v in out.items()}
 
 
-def compare(name, got: torch.Tensor, ref: np.ndarray, stored_bf16: bool):
+def bf16_rounding(ref: np.ndarray) -> np.ndarray:
+    """|bf16(x) - x| element-wise: what storing the exact result in bf16 costs."""
+    r = torch.from_numpy(np.ascontiguousarray(ref))
+    return np.abs(r.to(torch.bfloat16).double().numpy() - ref)
+
+
+def compare(name, got: torch.Tensor, ref: np.ndarray, stored_bf16: bool = False, gradient: bool = True):
+    """Element-wise check of one tensor against the oracle.  `stored_bf16`
+    with `gradient` applies the storage-floor rule for bf16 gradients; O is
+    passed with gradient=False and always gets the bare bound."""
     g = got.double().numpy()
     err = np.abs(g - ref)
-    bound = TOL_MAX + (BF16_REL * np.abs(ref) if stored_bf16 else 0.0)
+    bound = np.full_like(err, TOL_MAX)
+    floor = 0.0
+    if stored_bf16 and err.size:
+        rnd = bf16_rounding(ref)
+        floor = float(rnd.max())
+        if gradient and floor > BF16_FLOOR_GATE:
+            bound = bound + rnd
     stats = {"max": float(err.max()) if err.size else 0.0, "mean": float(err.mean()) if err.size else 0.0,
-             "worst_over_bound": float((err / bound).max()) if err.size else 0.0}
+             "worst_over_bound": float((err / bound).max()) if err.size else 0.0, "bf16_floor": floor}
     assert np.isfinite(g).all(), f"{name}: non-finite values"
     assert stats["mean"] <= TOL_MEAN, f"{name}: mean |err| {stats['mean']:.3e} > {TOL_MEAN}"
     assert np.all(err <= bound), f"{name}: max |err| {stats['max']:.3e} over the bound ({stats})"
@@ -72,7 +92,7 @@ def check_slices(w, x, got, slices, seed=0, grad_dtype=torch.float32):
     o_ref, lse_ref = oracle.fwd_slices(q, k, v, arows, rrows, rep)
     stats = {}
     sel = lambda t: torch.stack([t[b, h] for b, h in slices])  # noqa: E731
-    stats["o"] = compare("O", sel(got["o"]), o_ref, stored_bf16=True)
+    stats["o"] = compare("O", sel(got["o"]), o_ref, stored_bf16=True, gradient=False)
     lse_err = np.abs(sel(got["lse"]).double().numpy() - lse_ref)
     assert lse_err.max() <= TOL_LSE, f"lse max err {lse_err.max():.3e}"
     stats["lse"] = {"max": float(lse_err.max())}

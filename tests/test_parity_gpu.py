@@ -54,11 +54,13 @@ def test_ragged_lengths(T, kind, path):
     P.check_slices(w, x, got, _all_slices(w))
 
 
-def test_several_tiles_full(path):
+@pytest.mark.parametrize("grad_dtype", [torch.float32, torch.bfloat16], ids=["grad_fp32", "grad_bf16"])
+def test_several_tiles_full(grad_dtype, path):
     w = I.custom(2, 4, 1000, [1, 2])
     x = I.make_inputs(w, 5)
-    got = P.run_layer(w, x, torch.bfloat16)
-    P.check_slices(w, x, got, _all_slices(w), grad_dtype=torch.bfloat16)
+    got = P.run_layer(w, x, grad_dtype)
+    stats = P.check_slices(w, x, got, _all_slices(w), grad_dtype=grad_dtype)
+    print(w.name, stats)
 
 
 def _special(T, a_fn, r_fn):
@@ -157,12 +159,44 @@ def test_lognorm_tiles_and_special_values(T):
 
 
 def test_repeatable():
+    """Two calls on the same inputs: O, lse, dK and dV are bit-identical (each
+    is produced by one CTA in a fixed order); dQ is the sum of fp32 reduce-adds
+    from several CTAs, whose order is not fixed, so it repeats to within the
+    rounding of that sum."""
     w = I.custom(1, 3, 700, [1])
     x = I.make_inputs(w, 2)
     a = P.run_layer(w, x)
     b = P.run_layer(w, x)
     for k in a:
-        assert torch.equal(a[k], b[k]), k
+        if k == "dq":
+            scale = max(1.0, a[k].abs().max().item())
+            assert (a[k] - b[k]).abs().max().item() <= 1e-5 * scale, k
+        else:
+            assert torch.equal(a[k], b[k]), k
+
+
+def test_dq_repeats_across_many_calls():
+    """dQ boxes are written by the last of their contributions: eight calls on a
+    layer with many contributions per box (T = 3000, 24 key blocks) and several
+    items per CTA give the same dQ up to the order of the fp32 reduce-adds, and
+    every call matches the oracle on a sampled slice."""
+    w = I.custom(4, 6, 3000, [2, 5])
+    x = I.make_inputs(w, 66)
+    g = P.to_gpu(x)
+    o, lse = saf.mixed_attn_fwd(g["q"], g["k"], g["v"], g["alpha"], g["rho"], x["mask"])
+    ref = None
+    for _ in range(8):
+        dq, dk, dv = saf.mixed_attn_bwd(g["q"], g["k"], g["v"], o, g["do"], lse, g["alpha"], g["rho"], x["mask"],
+                                        grad_dtype=torch.float32)
+        torch.cuda.synchronize()
+        if ref is None:
+            ref = (dq.clone(), dk.clone(), dv.clone())
+            got = {"o": o.cpu(), "lse": lse.cpu(), "dq": dq.cpu(), "dk": dk.cpu(), "dv": dv.cpu()}
+            P.check_slices(w, x, got, [(3, 0), (1, 5)])
+            continue
+        scale = max(1.0, ref[0].abs().max().item())
+        assert (dq - ref[0]).abs().max().item() <= 1e-5 * scale
+        assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
 
 
 def _full_size(name, grad_dtype=torch.float32, per_kind=2):
@@ -193,13 +227,34 @@ def test_full_size_bf16_grads_sampled():
 
 @pytest.mark.parametrize("name", I.PREFILL_SWEEP)
 def test_prefill_sweep_sampled(name):
-    _full_size(name, per_kind=1)
+    _full_size(name, per_kind=2)
 
 
 def test_factored_range_guard_falls_back(path):
     """a spanning far more than fp32's range: the factored form is refused for
     that head, which then runs the per-element exp path; results unchanged."""
     w, x = _special(777, lambda T: torch.randn(T) * 40.0, lambda T: -0.05 * torch.arange(T, dtype=torch.float32))
+    got = P.run_layer(w, x)
+    P.check_slices(w, x, got, _all_slices(w))
+
+
+def test_rows_far_below_the_pattern_maxima(path):
+    """Rows whose log Z sits far below max a + max r: a sink a[0] = 25 that
+    rows past 200 cannot see (r = -1000 beyond distance 200) and every other
+    key near -50, so max a + max r - log Z(i) is about 70 for those rows,
+    above the factored form's limit of 50 while max a - min a stays under 80:
+    the log Z limit alone sends the head to the per-element path.  Every
+    slice against the oracle."""
+    def a_fn(T):
+        a = torch.randn(T) * 0.5 - 50.0
+        a[0] = 25.0
+        return a
+
+    def r_fn(T):
+        r = torch.zeros(T)
+        r[200:] = -1000.0
+        return r
+    w, x = _special(900, a_fn, r_fn)
     got = P.run_layer(w, x)
     P.check_slices(w, x, got, _all_slices(w))
 
@@ -239,7 +294,7 @@ def test_grouped_kv_layer(B, H, Hkv, T, replaced, grad_dtype):
     assert tuple(dk.shape) == (B, Hkv, T, 64) and tuple(dv.shape) == (B, Hkv, T, 64)
     o_ref, lse_ref = oracle.fwd_gqa(x["q"], k, v, x["alpha"], x["rho"], x["mask"])
     dq_ref, dk_ref, dv_ref = oracle.bwd_gqa(x["q"], k, v, x["do"], x["alpha"], x["rho"], x["mask"])
-    P.compare("O", o.cpu(), o_ref, stored_bf16=True)
+    P.compare("O", o.cpu(), o_ref, stored_bf16=True, gradient=False)
     lse_fin = np.isfinite(lse_ref)
     assert np.abs(lse.cpu().double().numpy()[lse_fin] - lse_ref[lse_fin]).max() <= P.TOL_LSE
     bf = grad_dtype == torch.bfloat16
