@@ -188,9 +188,7 @@ saf_status saf_mixed_attn_bwd_gqa(const void* q, const void* k, const void* v, c
 
     cudaStream_t s = (cudaStream_t)stream;
     char* ws = static_cast<char*>(workspace);
-    // log Z: the caller's, or computed into the workspace
     float* lzw = reinterpret_cast<float*>(ws + L.logz);
-    const float* lz = logz ? logz : lzw;
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
     const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v);
@@ -198,6 +196,7 @@ saf_status saf_mixed_attn_bwd_gqa(const void* q, const void* k, const void* v, c
     const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
     if (force_mma_path()) {
         if (H_kv != H) return SAF_ERR_UNSUPPORTED;  // the warp-level path has no shared K/V
+        const float* lz = logz ? logz : lzw;
         if (hl.n > 0 && !logz && launch_lognorm(a, r, hl, T, lzw, s) != cudaSuccess) return SAF_ERR_CUDA;
         float* dvec = reinterpret_cast<float*>(ws + L.dvec);
         if (launch_bwd_dot(ob, dob, dvec, hl, B, H, T, s) != cudaSuccess) return SAF_ERR_CUDA;
@@ -208,10 +207,12 @@ saf_status saf_mixed_attn_bwd_gqa(const void* q, const void* k, const void* v, c
     float* nlse2p = reinterpret_cast<float*>(ws + L.nlse2p);
     float* dvecp = reinterpret_cast<float*>(ws + L.dvecp);
     float* dqacc = reinterpret_cast<float*>(ws + L.dqacc);
-    // one launch: the row terms, the zeroed dQ accumulator and counters, and
-    // the replaced heads' patterns
-    if (launch_bwd_pre(ob, dob, lse, B * H, T, nlse2p, dvecp, dqacc, a, r, logz, logz ? nullptr : lzw, hl, rw,
-                       s) != cudaSuccess)
+    // log Z: the caller's, or batch 0's lse rows of the replaced heads (the
+    // forward wrote log Z there, laid out [H, T] like logz)
+    const float* lz = logz ? logz : lse;
+    // one launch: the row terms, the zeroed dQ accumulator, and the replaced
+    // heads' factored arrays
+    if (launch_bwd_pre(ob, dob, lse, B * H, T, nlse2p, dvecp, dqacc, a, r, lz, nullptr, hl, rw, s) != cudaSuccess)
         return SAF_ERR_CUDA;
     // shared K/V: per-query-head fp32 dK, dV into the workspace, then summed per group
     const bool grouped = H_kv != H;

@@ -63,6 +63,32 @@ def test_noalloc_backward_full_size_layer():
         _close(got, ref)
 
 
+@pytest.mark.gpu
+def test_noalloc_call_allocates_no_device_memory():
+    """The property the entry point exists for: with the outputs passed in, a
+    call (after a first one, which looks up the scratch array's address and
+    loads the kernels) changes neither the device's free memory nor torch's
+    allocated bytes."""
+    w = I.custom(2, 4, 700, [1, 3])
+    x, g, o, lse = _layer(w, 23)
+    outs = [torch.empty(w.B, w.H, w.T, 64, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+
+    def call():
+        saf.mixed_attn_bwd_noalloc(g["q"], g["k"], g["v"], o, g["do"], lse, g["alpha"], g["rho"], x["mask"],
+                                   grad_dtype=torch.bfloat16, dq=outs[0], dk=outs[1], dv=outs[2])
+
+    call()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"device free memory moved by {free0 - free1} bytes"
+    assert torch.cuda.memory_allocated() == alloc0
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
     """Checked on the host before any CUDA call, so it also runs without a GPU."""
     lib = saf.load()
