@@ -145,8 +145,8 @@ saf_status saf_mixed_attn_fwd_gqa(const void* q, const void* k, const void* v, v
     const ReplacedWs rw = replaced_ws(ws, L, T);
     if (hl.n > 0 && launch_pattern(a, r, logz, logz ? nullptr : lzw, hl, T, &rw, s) != cudaSuccess)
         return SAF_ERR_CUDA;
-    cudaError_t e =
-        launch_fwd_tc(qb, kb, vb, ob, lse, a, r, lz, hl, rw, B, H, H_kv, T, reinterpret_cast<unsigned int*>(ws), s);
+    cudaError_t e = launch_fwd_tc(qb, kb, vb, ob, lse, a, r, lz, hl, rw, B, H, H_kv, T,
+                                  reinterpret_cast<unsigned int*>(ws), hl.n > 0, s);
     if (e == cudaErrorNotSupported) return SAF_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return SAF_ERR_CUDA;
     return SAF_OK;

@@ -174,10 +174,12 @@ cudaError_t launch_pattern(const float* a, const float* r, const float* logz_in,
 // leave fp32 range, flag 1, take per-element exps of a + r - log Z); returns
 // cudaErrorNotSupported when the tensor maps cannot be built.
 // k, v hold Hkv heads; query head h reads K/V head h / (H / Hkv).
+// after_pattern: the launch right before it on the stream is this call's
+// pattern preparation, which the kernel then overlaps (programmatic launch).
 cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
                           const HeadList& hl, const ReplacedWs& w, int B, int H, int Hkv, int T, unsigned int* err,
-                          cudaStream_t stream);
+                          bool after_pattern, cudaStream_t stream);
 // Backward preprocessing for the tensor-core backward, one launch: padded
 // -lse*log2(e) and rowsum(dO o O), a zeroed dQ accumulator, and (hl.n > 0)
 // the replaced heads' pattern preparation (what launch_pattern does: log Z

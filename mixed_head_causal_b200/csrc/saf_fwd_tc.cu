@@ -63,8 +63,7 @@ constexpr uint32_t SM_V = SM_K + NSK * TILE_BYTES;
 // reads the same atom)
 constexpr uint32_t SM_ONES = SM_V + NSV * TILE_BYTES;
 constexpr uint32_t SM_BAR = SM_ONES + 2048;
-constexpr uint32_t SM_DFL = SM_BAR + 256;  // per replaced slot: 1 = per-element path
-constexpr uint32_t SM_TOTAL = SM_DFL + 256;
+constexpr uint32_t SM_TOTAL = SM_BAR + 256;
 
 struct FwdTcParams {
     __nv_bfloat16* o;
@@ -178,6 +177,15 @@ __device__ __noinline__ void direct_p_row(const float* ah, const float* rh, cons
     }
 }
 
+// Whether replaced slot s takes the per-element path: any of its tiles' range
+// flags (a warp-wide OR).  Out of line: it runs once per replaced item and
+// keeps its registers out of the row loop's allocation.
+__device__ __noinline__ bool head_direct(const ReplacedWs& w, int s) {
+    int any = 0;
+    for (int t = threadIdx.x & 31; t < w.ntiles; t += 32) any |= w.tflag[(size_t)s * w.ntiles + t];
+    return __any_sync(0xffffffffu, any != 0);
+}
+
 __global__ void __launch_bounds__(NTHREADS, 2)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const FwdTcParams p) {
@@ -239,8 +247,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         for (int u = 0; u < 4; ++u) st_shared_v4(sbase + SM_ONES + (u * 32 + lane) * 16, one2, one2, one2, one2);
         fence_proxy_async_smem();
     }
-    uint8_t* dfl = smem + SM_DFL;
-    if (warp == 0) slot_flags(p.w, p.nslots, dfl);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -259,12 +265,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // (query block I visits I + 1 key blocks)
     struct Item {
         int bh, bhkv, I, h, slot;  // query slice, its K/V slice, query block, head, replaced slot
-        bool rep, direct;
+        bool rep;
     };
-    // the published item word carries the head's per-element flag in bit 30
-    // (set by the producer from the per-slot flags)
-    auto decode = [&](int word) {
-        const int item = word & 0x3fffffff;
+    auto decode = [&](int item) {
         Item it;
         int rank;
         grouped_order((unsigned)item, p.BH, p.nqb, it.bh, rank);
@@ -273,7 +276,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         it.bhkv = (it.bh / p.H) * p.Hkv + it.h / (p.H / p.Hkv);
         it.slot = p.slot_of_head[it.h];
         it.rep = it.slot >= 0;
-        it.direct = it.rep && ((word >> 30) & 1) != 0;  // per-element exps instead of the factored form
         return it;
     };
 
@@ -287,11 +289,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             bool ok = true;
             for (int n = 0; ok; ++n) {
                 const int w = (int)atomicAdd(p.err + kCtrFwdNext, 1u);
-                int item = w < total ? w : -1;
-                if (item >= 0) {
-                    const Item pre = decode(item);
-                    if (pre.rep && dfl[pre.slot]) item |= 1 << 30;
-                }
+                const int item = w < total ? w : -1;
                 if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                 *reinterpret_cast<volatile int*>(item_slot + (n & 1)) = item;
                 mbar_arrive(bar_itf + 8 * (n & 1));
@@ -422,6 +420,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t tO = tmem + lane_off + TO_COL;
         const uint32_t tP = tmem + lane_off + TP_COL;
         int go = 0, gr = 0;  // ordinary and replaced blocks so far
+        // Replaced heads read what the pattern preparation writes (the factored
+        // arrays, their range flags, log Z); with a programmatic launch this
+        // kernel may start before that grid ends, so the row warps wait for it
+        // at their first replaced item.  A head's per-element flag (any of its
+        // tiles' range flags) is found then and cached per warp (slots < 32).
+        bool waited = false;
         bool ok = true;
         for (int n = 0; ok; ++n) {
             int item;
@@ -429,14 +433,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (!ok) { report(p.err, 0x305); break; }
             if (item < 0) break;
             int I, slot, h;
-            bool rep, direct;
+            bool rep, direct = false;
             {
                 const Item it = decode(item);
                 I = it.I;
                 slot = it.slot;
                 h = it.h;
                 rep = it.rep;
-                direct = it.direct;
+            }
+            if (rep) {
+                if (!waited) {
+                    griddep_wait();
+                    waited = true;
+                }
+                direct = head_direct(p.w, slot);  // per-element exps instead of the factored form
             }
             const int nkb = I + 1;
             const int i = I * BM + row;
@@ -640,7 +650,7 @@ bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out) {
 cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                           __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
                           const HeadList& hl, const ReplacedWs& w, int B, int H, int Hkv, int T, unsigned int* err,
-                          cudaStream_t stream) {
+                          bool after_pattern, cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     const int BH = B * H;
     if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, B * Hkv, T, &mk) ||
@@ -674,8 +684,21 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     const int items = BH * p.nqb;
     const int grid = std::min(items, 2 * sm_count());
     launch_begin(KID_FWD_TC, stream);
-    fwd_tc_kernel<<<dim3((unsigned)grid), NTHREADS, smem, stream>>>(mq, mk, mv, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    // after the pattern preparation of this call (after_pattern), the kernel
+    // may start while that grid runs: its ordinary items do not depend on it
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_pattern ? 1 : 0;
+    cudaError_t le = cudaLaunchKernelEx(&cfg, fwd_tc_kernel, mq, mk, mv, p);
     launch_end(KID_FWD_TC, stream);
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 

@@ -269,6 +269,9 @@ __device__ void pattern_tile(const PatternJob& J, int slot, int t, float* dyn, P
 __global__ void __launch_bounds__(kPpThreads) pattern_kernel(const PatternJob J) {
     extern __shared__ float pp_smem[];
     __shared__ PatternShared sh;
+    // the forward kernel that follows waits for this grid only where it reads
+    // what this grid writes: it may start now
+    tc::griddep_launch_dependents();
     pattern_tile(J, blockIdx.y, J.ntiles - 1 - blockIdx.x, pp_smem, sh);
 }
 
