@@ -99,17 +99,20 @@ __device__ __forceinline__ uint32_t packed_kcol(int k) { return k < 4 ? 8 * k : 
 
 // P^T for queries [32c, 32c + 32) of key row jl: exp2(S^T * scale - lse2),
 // packed as 16 bf16 pairs over TMEM columns packed_col(c) of the S^T region.
-// nlse2 holds -lse2 per query (read as pairs); the scale-and-shift runs on
-// paired fp32 FMAs.  MASK: zero where the query precedes the key on the
-// diagonal tile, or where the key lies past T.
+// Shared memory at nlse2 holds -lse2 per query (read as pairs, 16 bytes at a
+// time, while the TMEM load is in flight); the scale-and-shift runs on paired
+// fp32 FMAs.  MASK: zero where the query precedes the key on the diagonal
+// tile, or where the key lies past T.
 template <bool MASK>
-__device__ __forceinline__ void p_chunk(uint32_t tS, int c, const float* nlse2, float scale, int jl, bool diag,
+__device__ __forceinline__ void p_chunk(uint32_t tS, int c, uint32_t nlse2, float scale, int jl, bool diag,
                                         bool key_ok, uint32_t (&pw)[16]) {
     uint32_t v[32];
     tmem_ld32(tS + 32 * c, v);
+    uint64_t nl[16];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) ld_shared_2x64(nlse2 + 128 * c + 16 * q, nl[2 * q], nl[2 * q + 1]);
     tmem_wait_ld();
     const uint64_t sc2 = f32x2(scale, scale);
-    const uint64_t* nl = reinterpret_cast<const uint64_t*>(nlse2 + 32 * c);
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
         const int ql = 32 * c + e;
@@ -502,8 +505,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int jl = quarter * 32 + lane;  // key within the block = TMEM lane
         const uint32_t lo = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + lo + C_S, tDP = tmem + lo + C_DP;
-        const float* vec1 = reinterpret_cast<const float*>(smem + SM_VEC1);
-        const float* vec2 = reinterpret_cast<const float*>(smem + SM_VEC2);
+        const uint32_t vec1 = sb + SM_VEC1, vec2 = sb + SM_VEC2;  // shared addresses
         int s = 0, u = 0, go = 0, gr = 0;  // ring stage and pass; ordinary, replaced tiles so far
         bool ok = true;
         for (int n = 0; ok; ++n) {
@@ -521,9 +523,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const int I = it.J + t;
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_qf + 8 * s, u & 1, kWaitLimit));
                 if (!ok) { report(p.err, 0x1301); break; }
-                const float* v1 = vec1 + 128 * s;
+                const uint32_t v1 = vec1 + 512 * s;
                 if (!it.rep) {
-                    const float* v2 = vec2 + 128 * s;
+                    const uint32_t v2 = vec2 + 512 * s;
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s, go & 1, kWaitLimit));
                     if (!ok) { report(p.err, 0x1302); break; }
                     tc_fence_after();
@@ -557,8 +559,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         const int c = 2 * half + cc;
                         uint32_t v[32], dsw[16];
                         tmem_ld32(tDP + 32 * c, v);
+                        uint64_t d2[16];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) ld_shared_2x64(v2 + 128 * c + 16 * q, d2[2 * q], d2[2 * q + 1]);
                         tmem_wait_ld();
-                        const uint64_t* d2 = reinterpret_cast<const uint64_t*>(v2 + 32 * c);
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
                             // (dP - D) paired, times P (bf16, widened), one rounding
@@ -603,14 +607,19 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                             const int c = 2 * half + cc;
                             uint32_t hw[16], lw[16];
 #pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
+                            for (int e = 0; e < 32; e += 4) {
                                 const int ql = 32 * c + e;
-                                const float w0 = __ldg(ef + ql) * v1[ql];
-                                const float w1 = __ldg(ef + ql + 1) * v1[ql + 1];
-                                const uint32_t hb = pack_bf16x2(w0, w1);
-                                const float2 hf = unpack_bf16x2(hb);
-                                hw[e / 2] = hb;
-                                lw[e / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                                const float4 r4 = ld_shared_f4(v1 + 4 * ql);
+                                const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+                                for (int u = 0; u < 4; u += 2) {
+                                    const float w0 = __ldg(ef + ql + u) * rr[u];
+                                    const float w1 = __ldg(ef + ql + u + 1) * rr[u + 1];
+                                    const uint32_t hb = pack_bf16x2(w0, w1);
+                                    const float2 hf = unpack_bf16x2(hb);
+                                    hw[(e + u) / 2] = hb;
+                                    lw[(e + u) / 2] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+                                }
                             }
                             tmem_st16(tW + 16 * c, hw);
                             tmem_st16(tW + 64 + 16 * c, lw);

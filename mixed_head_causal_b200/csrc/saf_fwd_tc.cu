@@ -91,21 +91,13 @@ __device__ __forceinline__ void load_s_row(uint32_t tS, uint32_t (&v)[128]) {
     tmem_wait_ld();
 }
 
-// Row max of one 128-key block of raw scores.  MASK: the diagonal block,
-// where keys past the row (or past T) do not count.  Three-input max, four
+// Row max of one 128-key block of raw scores.  Three-input max, four
 // independent chains.
-template <bool MASK>
-__device__ __forceinline__ float row_max(const uint32_t (&v)[128], int kbase, int i, int T) {
+__device__ __forceinline__ float row_max(const uint32_t (&v)[128]) {
     float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
-    for (int e = 0; e < 128; e += 2) {
-        float s0 = __uint_as_float(v[e]), s1 = __uint_as_float(v[e + 1]);
-        if (MASK) {
-            if (kbase + e > i || kbase + e >= T) s0 = kNegInf;
-            if (kbase + e + 1 > i || kbase + e + 1 >= T) s1 = kNegInf;
-        }
-        mx[(e >> 1) & 3] = max3(mx[(e >> 1) & 3], s0, s1);
-    }
+    for (int e = 0; e < 128; e += 2)
+        mx[(e >> 1) & 3] = max3(mx[(e >> 1) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
     return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
@@ -113,24 +105,111 @@ __device__ __forceinline__ float row_max(const uint32_t (&v)[128], int kbase, in
 // returns the sum of the (unrounded) probabilities.  The scale-and-shift and
 // the running sums use the paired fp32 instructions (same rounding as the
 // scalar ones).
-template <bool MASK>
-__device__ __forceinline__ float exp_row(const uint32_t (&v)[128], int kbase, int i, int T, float scale, float m,
-                                         uint32_t (&pw)[64]) {
+__device__ __forceinline__ float exp_row(const uint32_t (&v)[128], float scale, float m, uint32_t (&pw)[64]) {
     const uint64_t sc2 = f32x2(scale, scale), nm2 = f32x2(-m, -m);
     uint64_t l2[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int e = 0; e < 128; e += 2) {
         const float2 x = split_f32x2(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nm2));
-        float p0 = ex2(x.x), p1 = ex2(x.y);
-        if (MASK) {
-            if (kbase + e > i || kbase + e >= T) p0 = 0.f;
-            if (kbase + e + 1 > i || kbase + e + 1 >= T) p1 = 0.f;
-        }
+        const float p0 = ex2(x.x), p1 = ex2(x.y);
         l2[(e >> 1) & 3] = add_f32x2(l2[(e >> 1) & 3], f32x2(p0, p1));
         pw[e >> 1] = pack_bf16x2(p0, p1);
     }
     const float2 a = split_f32x2(add_f32x2(add_f32x2(l2[0], l2[1]), add_f32x2(l2[2], l2[3])));
     return a.x + a.y;
+}
+
+// Rescales this warp's 32 O rows by f (a whole-warp TMEM round trip, taken
+// when any row of the warp needs it).
+__device__ __forceinline__ void rescale_o(uint32_t tO, float f) {
+    if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+            tmem_st32(tO + 32 * c, ov);
+        }
+    }
+}
+
+// The running max m moves only when a block's max mx exceeds it by more than
+// 8 (log2 units), so P stays below 2^8 and O is rarely rescaled; returns the
+// factor f for l and O (1 when m stays).
+__device__ __forceinline__ float update_max(float mx, float& m, float& l) {
+    float f = 1.f;
+    if (m == kNegInf) {
+        m = mx;
+    } else if (mx > m + 8.f) {
+        f = ex2(m - mx);
+        l *= f;
+        m = mx;
+    }
+    return f;
+}
+
+// The diagonal block of an item (query block I, key block I; key e and row r
+// counted from the same start, BN = BM) keeps key e of row r when e <= r.  It
+// runs once per item, so its code is short and out of line (loops over
+// 32-key chunks, S read from TMEM in each pass) where the other blocks' is
+// unrolled: a cold unrolled copy, fetched once per item, costs several times
+// its arithmetic.  Rows of lane quarter q see every key of chunks c < q, part
+// of chunk q and none past it.  No key of a stored row lies past T
+// (key <= row < T); rows past T see zero-filled keys.  S stays in TMEM until
+// P is handed over (the next S, the next item's first, is issued after this
+// block's P.V).  Waits for P.V_{j-1} (parity o_par) unless j = 0, rescales O,
+// writes P (zeros past the row) to the P columns; m and l in ml (x, y) are
+// updated.  False when the wait gave up.
+__device__ __noinline__ bool diag_block(uint32_t tS, uint32_t tO, uint32_t tP, int quarter, int row, float scale,
+                                        bool first, uint32_t bar_o, uint32_t o_par, float2& ml) {
+    float m = ml.x, l = ml.y;
+    float mx2[2] = {kNegInf, kNegInf};
+#pragma unroll 1
+    for (int c = 0; c <= quarter; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + 32 * c, v);
+        tmem_wait_ld();
+        const int lim = row - 32 * c;
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+            mx2[(e >> 1) & 1] = max3(mx2[(e >> 1) & 1], e > lim ? kNegInf : __uint_as_float(v[e]),
+                                     e + 1 > lim ? kNegInf : __uint_as_float(v[e + 1]));
+    }
+    const float f = update_max(fmaxf(mx2[0], mx2[1]) * scale, m, l);
+    if (!first) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o, o_par, kWaitLimit))) return false;
+        tc_fence_after();
+    }
+    rescale_o(tO, f);
+    const uint64_t sc2 = f32x2(scale, scale), nm2 = f32x2(-m, -m);
+    uint64_t l2[2] = {0, 0};
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t pw[16];
+        if (c <= quarter) {
+            uint32_t v[32];
+            tmem_ld32(tS + 32 * c, v);
+            tmem_wait_ld();
+            const int lim = row - 32 * c;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+                const float2 x =
+                    split_f32x2(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nm2));
+                const float p0 = e > lim ? 0.f : ex2(x.x), p1 = e + 1 > lim ? 0.f : ex2(x.y);
+                l2[(e >> 1) & 1] = add_f32x2(l2[(e >> 1) & 1], f32x2(p0, p1));
+                pw[e >> 1] = pack_bf16x2(p0, p1);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pw[e] = 0u;
+        }
+        tmem_st16(tP + 16 * c, pw);
+    }
+    const float2 a = split_f32x2(add_f32x2(l2[0], l2[1]));
+    ml = make_float2(m, l + (a.x + a.y));
+    return true;
 }
 
 // W(i, j) = E[i-j] c_j for 64 keys (q0 = 0 or 8 selects the half): bf16 pair
@@ -456,51 +535,36 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_s, (go + j) & 1, kWaitLimit));
                     if (!ok) { report(p.err, 0x301); break; }
                     tc_fence_after();
-                    uint32_t v[128];
-                    load_s_row(tS, v);
-                    tc_fence_before();
-                    mbar_arrive_warp(bar_sf);  // the MMA warp may now overwrite S
-                    const bool diag = (j == I);
-                    const int kbase = j * BN;
-                    // row max of the block (the scale is positive); every row of a
-                    // visited block has a visible key, so mx is finite.  The running
-                    // max m moves only when the block's max exceeds it by more than
-                    // 8 (log2 units), so P stays below 2^8 and O is rarely rescaled.
-                    const float mx =
-                        (diag ? row_max<true>(v, kbase, i, T) : row_max<false>(v, kbase, i, T)) * p.scale_log2;
-                    float f = 1.f;
-                    if (m == kNegInf) {
-                        m = mx;
-                    } else if (mx > m + 8.f) {
-                        f = ex2(m - mx);
-                        l *= f;
-                        m = mx;
-                    }
-                    uint32_t pw[64];  // P as bf16 pairs
-                    l += diag ? exp_row<true>(v, kbase, i, T, p.scale_log2, m, pw)
-                              : exp_row<false>(v, kbase, i, T, p.scale_log2, m, pw);
-                    // P_j replaces P_{j-1} in TMEM once P.V_{j-1} has read it (the
-                    // previous item's last P.V was waited for by its epilogue); the
-                    // O rows are rescaled (by the whole warp, when any row needs
-                    // it) once that P.V has landed in O
-                    if (j > 0) {
-                        ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (go + j - 1) & 1, kWaitLimit));
+                    if (j == I) {
+                        float2 ml = make_float2(m, l);
+                        ok = diag_block(tS, tO, tP, quarter, row, p.scale_log2, j == 0, bar_o, (go + j - 1) & 1, ml);
                         if (!ok) { report(p.err, 0x302); break; }
-                        tc_fence_after();
-                    }
-                    if (__any_sync(0xffffffffu, f != 1.f)) {
-#pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            uint32_t ov[32];
-                            tmem_ld32(tO + 32 * c, ov);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-                            tmem_st32(tO + 32 * c, ov);
+                        m = ml.x;
+                        l = ml.y;
+                        tc_fence_before();
+                        mbar_arrive_warp(bar_sf);
+                    } else {
+                        uint32_t v[128];
+                        load_s_row(tS, v);
+                        tc_fence_before();
+                        mbar_arrive_warp(bar_sf);  // the MMA warp may now overwrite S
+                        // row max of the block (the scale is positive); every row of
+                        // a visited block has a visible key, so it is finite
+                        const float f = update_max(row_max(v) * p.scale_log2, m, l);
+                        uint32_t pw[64];  // P as bf16 pairs
+                        l += exp_row(v, p.scale_log2, m, pw);
+                        // P_j replaces P_{j-1} in TMEM once P.V_{j-1} has read it (the
+                        // previous item's last P.V was waited for by its epilogue); the
+                        // O rows are rescaled once that P.V has landed in O
+                        if (j > 0) {
+                            ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (go + j - 1) & 1, kWaitLimit));
+                            if (!ok) { report(p.err, 0x302); break; }
+                            tc_fence_after();
                         }
+                        rescale_o(tO, f);
+                        tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
+                        tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
                     }
-                    tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
-                    tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
                 } else {
                     // W(i,j) = E[i-j] c_j, bf16 pairs, into buffer g & 1 (g counts
                     // replaced blocks), last read by the P.V of block g - 2 (one

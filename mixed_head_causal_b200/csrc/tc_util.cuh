@@ -246,6 +246,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Packed fp32 pairs (sm_100 two-wide FFMA/FADD) and the three-input max.
+// 16 bytes of shared memory as two fp32 pairs, or as four floats (explicit
+// shared-space loads: a pointer rounded up to an alignment boundary through
+// an integer loses its address space, and generic loads cost more).
+__device__ __forceinline__ void ld_shared_2x64(uint32_t addr, uint64_t& a, uint64_t& b) {
+    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];\n" : "=l"(a), "=l"(b) : "r"(addr));
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
     uint64_t r;
     asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(lo), "f"(hi));
