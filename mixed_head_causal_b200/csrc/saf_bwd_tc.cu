@@ -77,6 +77,7 @@ struct BwdTcParams {
     unsigned int* err;
     int16_t slot_of_head[kMaxHeads];
     int H, Hkv, BH, T, Tp, nqb, grad_fp32;  // Hkv: K/V heads (H / Hkv query heads share one)
+    int tma_grads;  // bf16 dK, dV written by TMA stores of 32-row boxes (else per-thread row stores)
     int nslots;  // replaced heads
     float scale, scale_log2;
 };
@@ -179,7 +180,8 @@ __device__ __noinline__ void direct_pt_half(const BwdTcParams& p, int h, int T, 
 __global__ void __launch_bounds__(NTHREADS, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-              const __grid_constant__ CUtensorMap tmDQ, const BwdTcParams p) {
+              const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+              const __grid_constant__ CUtensorMap tmDV, const BwdTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_addr(smem);
@@ -554,6 +556,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, go & 1, kWaitLimit));
                     if (!ok) { report(p.err, 0x1303); break; }
                     tc_fence_after();
+                    if (t == 0 && p.tma_grads) {  // this warp's last dK/dV box has been read
+                        if (lane == 0) bulk_wait_read0();
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int c = 2 * half + cc;
@@ -664,10 +670,34 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             tc_fence_before();
             mbar_arrive_warp(bar_acr);
-            // per-thread row stores (fire and forget: the warps move on to the next
-            // item at once, which measured faster than staging for coalescing)
-            if (j < T) store_row(half == 0 ? p.dv : p.dk, p.grad_fp32, (size_t)it.bh * T + j, vals);
+            if (p.tma_grads) {
+                // bf16: the warp's 32 rows as one TMA box, staged in the warp's own
+                // 4 KB of the dS^T area (row `lane`, 16-byte chunks in the 128-byte
+                // swizzle of the store map), where this warp alone writes its dS^T
+                // rows.  The area is idle here: the item's last dQ MMA, its last
+                // reader, completed before bar_acc.  The warp moves on once the
+                // store is issued; 32 per-thread row stores instead block its next
+                // shared-memory and barrier operations for thousands of cycles.
+                const uint32_t box = sb + SM_DS + half * 16384 + quarter * 4096;
+                if (lane == 0) bulk_wait_read0();  // the previous box has been read
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    st_shared_v4(box + lane * 128 + ((k ^ (lane & 7)) << 4), pack_bf16x2(vals[8 * k], vals[8 * k + 1]),
+                                 pack_bf16x2(vals[8 * k + 2], vals[8 * k + 3]),
+                                 pack_bf16x2(vals[8 * k + 4], vals[8 * k + 5]),
+                                 pack_bf16x2(vals[8 * k + 6], vals[8 * k + 7]));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(half == 0 ? &tmDV : &tmDK, box, 0, it.J * BN + quarter * 32, it.bh);
+                    bulk_commit();
+                }
+            } else if (j < T) {
+                store_row(half == 0 ? p.dv : p.dk, p.grad_fp32, (size_t)it.bh * T + j, vals);
+            }
         }
+        if (lane == 0) bulk_wait0();  // the dK/dV stores complete before the CTA ends
     } else {
         // ------------------------------------------------ dQ tiles -> global accumulator
         // Each warp moves its own 32 query rows: TMEM -> two 4 KB swizzled boxes
@@ -842,11 +872,15 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
                           const ReplacedWs& w, int B, int H, int Hkv, int T, void* dk, void* dv, int grad_fp32,
                           unsigned int* err, cudaStream_t stream) {
     const int BH = B * H;
-    CUtensorMap mq, mk, mv, mdo, mdq;
+    CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
     if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, B * Hkv, T, &mk) ||
         !make_tmap_bhtd(v, B * Hkv, T, &mv) ||
         !make_tmap_bhtd(dout, BH, T, &mdo) || !make_tmap_bhtd_f32(dqacc, BH, T, &mdq))
         return cudaErrorNotSupported;
+    // bf16 dK, dV [BH, T, 64] by 32-row TMA stores when their maps encode (a
+    // base the encoder rejects, e.g. not 16-byte aligned, takes the row stores)
+    const bool tma_grads = !grad_fp32 && make_tmap_bhtd(dk, BH, T, &mdk, 32) && make_tmap_bhtd(dv, BH, T, &mdv, 32);
+    if (!tma_grads) mdk = mdv = mq;  // not read
     BwdTcParams p;
     p.nlse2p = nlse2p;
     p.dvecp = dvecp;
@@ -870,6 +904,7 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     p.nqb = (T + BM - 1) / BM;
     if ((int64_t)BH * p.nqb >= (int64_t)1 << 30) return cudaErrorNotSupported;  // item words hold 30 bits
     p.grad_fp32 = grad_fp32;
+    p.tma_grads = tma_grads ? 1 : 0;
     p.scale = 0.125f;
     p.scale_log2 = kLog2e * 0.125f;
     const int smem = SM_TOTAL + 1024;
@@ -879,7 +914,7 @@ cudaError_t launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     const int items = BH * p.nqb;
     const int grid = items < sm_count() ? items : sm_count();
     launch_begin(KID_BWD_TC, stream);
-    bwd_tc_kernel<<<dim3((unsigned)grid), NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
+    bwd_tc_kernel<<<dim3((unsigned)grid), NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
     launch_end(KID_BWD_TC, stream);
     return cudaGetLastError();
 }

@@ -218,7 +218,7 @@ cudaError_t launch_pattern_grad(const __nv_bfloat16* v, const __nv_bfloat16* dou
 cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream);
 cudaError_t launch_group_sum(const float* src, void* dst, int B, int H, int Hkv, int T, int grad_fp32,
                              cudaStream_t stream);
-bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out);
+bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out, int box_rows = 128);
 bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out);
 // Warp-level (mma.sync) forward and backward of every head, the reference
 // path selected by SAF_FORCE_MMA.

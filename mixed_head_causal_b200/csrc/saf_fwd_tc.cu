@@ -698,12 +698,12 @@ int sm_count() {
 
 // [BH, T, 64] bf16 viewed as a 3-D tensor (d, t, bh); 128 x 64 boxes with the
 // 128-byte swizzle; rows past T read as zeros.
-bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out) {
+bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)BH};
     cuuint64_t strides[2] = {64 * 2, (cuuint64_t)T * 64 * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

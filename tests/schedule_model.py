@@ -54,6 +54,7 @@ class Machine:
         self.inflight = set()  # resources a TMA copy is writing
         self.pipe = []         # issued MMAs / commits not yet executed
         self.tma = []          # (barrier, units, resources) copies in flight
+        self.stores = []       # (barrier, resource, version, who) stores in flight
         self.slot = [None, None]
 
     def bar(self, name, count=1):
@@ -97,6 +98,17 @@ class Machine:
                 self.write(res, version, who)
         else:
             self.bars[op[1]].arrive()
+
+    def store(self, bar, res, want, who):
+        """A bulk store out of shared memory: reads `res` (which must still hold
+        `want`) whenever it runs, then arrives on `bar` (the issuer's wait for
+        its stores to have read their source)."""
+        self.stores.append((bar, res, want, who))
+
+    def step_store(self, i):
+        bar, res, want, who = self.stores.pop(i)
+        self.read(res, want, who)
+        self.bars[bar].arrive()
 
     def step_tma(self, i):
         bar, units, resources = self.tma.pop(i)
@@ -152,17 +164,20 @@ def simulate(m, roles, rng, max_steps=200000):
         if m.pipe:
             ready.append(("pipe", None))
         ready += [("tma", i) for i in range(len(m.tma))]
+        ready += [("store", i) for i in range(len(m.stores))]
         if not ready:
             if all(w is None for w in waiting.values()):
                 return
             stuck = {k: v[1:] for k, v in waiting.items() if v is not None}
             raise ModelError(f"deadlock: {stuck}")
-        weights = [speed[arg] if kind == "role" else speed[kind] for kind, arg in ready]
+        weights = [speed[arg] if kind == "role" else speed["tma" if kind == "store" else kind] for kind, arg in ready]
         kind, arg = rng.choices(ready, weights)[0]
         if kind == "pipe":
             m.step_pipe()
         elif kind == "tma":
             m.step_tma(arg)
+        elif kind == "store":
+            m.step_store(arg)
         else:
             waiting[arg] = next(roles[arg], None)
     raise ModelError("no progress")

@@ -24,6 +24,10 @@ import pytest
 from tests.schedule_model import Machine, ModelError, W, mutate, publish, simulate, take
 
 NQS = 3  # Q/dO ring depth
+# dK, dV are declared complete (bar_acc) after the item's last dQ MMA, the
+# last reader of the dS^T area that the row warps then stage dK/dV rows in
+# (the alternative, right after the last dK MMA, is the planted mistake below)
+ACC_AFTER_DQ = True
 ROWS = 8  # key-row warps: each owns one slice (lane quarter x column half) of S^T, dP^T and dS^T
 DQW = 4   # dQ warps: each owns one lane quarter of the dQ tiles
 
@@ -107,10 +111,14 @@ def mma_issuer(m):
                 yield W("ds", go, go & 1)
                 acc_in = [("C_DK", ("dK", n, t - 1))] if t > 0 else []
                 m.mma(all_of("C_DP", ROWS, ("dS", go)) + [(f"Q{st}", ("Q", g))] + acc_in, [("C_DK", ("dK", n, t))], "dK")
+                if not more and not ACC_AFTER_DQ:
+                    m.commit("acc")
                 b = go & 1
                 yield W(f"dqe{b}", (go >> 1) - 1, ((go >> 1) & 1) ^ 1)
                 m.mma(all_of("DS", ROWS, ("dS", go)) + [(f"K{kb}", ("K", nk))], all_of(f"C_DQ{b}", DQW, ("dQ", go)), "dQ")
                 m.commit(f"dqf{b}")
+                if not more and ACC_AFTER_DQ:
+                    m.commit("acc")
                 if more:
                     m.mma([("V", ("V", nk)), (f"DO{s1}", ("DO", g + 1))], all_of("C_DP", ROWS, ("dP", go + 1)), "dP")
                     m.commit("dp")
@@ -118,7 +126,6 @@ def mma_issuer(m):
                         m.commit("ve")
                 m.commit(f"qe{st}")
                 go += 1
-            m.commit("acc")
             m.commit(f"ke{kb}")
             nk += 1
         else:
@@ -144,6 +151,7 @@ def key_rows(m, w):
     go = gr = 0
     G = 0
     n = 0
+    ns = 0  # dK/dV boxes this warp has stored from its slice of the dS^T area
     while True:
         it = yield from take(m, n)
         if it is None:
@@ -162,6 +170,8 @@ def key_rows(m, w):
                 yield W("dp", go, go & 1)
                 m.read(f"C_DP.{w}", ("dP", go), "rows dS")
                 m.read(f"VEC2_{s}", ("VEC", g), "rows dS")
+                if t == 0 and ns > 0:  # the last box has been read out of DS.w
+                    yield W(f"sr{w}", ns - 1, (ns - 1) & 1)
                 m.write(f"C_DP.{w}", ("dS", go), "rows dS")
                 m.write(f"DS.{w}", ("dS", go), "rows dS")
                 m.bars["ds"].arrive()
@@ -180,6 +190,13 @@ def key_rows(m, w):
         if not rep:
             m.read("C_DK", ("dK", n, ntiles - 1), "rows epilogue")
         m.bars["acr"].arrive()
+        # the warp's dK or dV rows staged in its slice of the dS^T area, then
+        # stored out by one bulk store (after the previous one has read it)
+        if ns > 0:
+            yield W(f"sr{w}", ns - 1, (ns - 1) & 1)
+        m.write(f"DS.{w}", ("stage", n), "rows stage")
+        m.store(f"sr{w}", f"DS.{w}", ("stage", n), "dK/dV store")
+        ns += 1
         n += 1
 
 
@@ -218,6 +235,8 @@ def run(items, seed):
         m.bar(name)
     for name in ("p", "ds", "acr"):
         m.bar(name, ROWS)
+    for w in range(ROWS):
+        m.bar(f"sr{w}")
     roles = {"producer": producer(m, items), "mma": mma_issuer(m)}
     roles.update({f"rows{w}": key_rows(m, w) for w in range(ROWS)})
     roles.update({f"dq{w}": dq_warp(m, w) for w in range(DQW)})
@@ -276,11 +295,23 @@ def _caught(seed):
     ("mma_issuer", 'yield W(f"dqe{b}", (go >> 1) - 1, ((go >> 1) & 1) ^ 1)', 'pass'),
     # the rows read dP^T before its MMA has run
     ("key_rows", 'yield W("dp", go, go & 1)', 'pass'),
-], ids=["no_ke", "no_qe", "no_ve", "no_wb", "no_dqe", "no_dp_wait"])
+    # dS^T written over a dK/dV box its store has not read yet
+    ("key_rows", "if t == 0 and ns > 0:", "if False:"),
+    # a box staged over the previous box before its store has read it
+    ("key_rows", "if ns > 0:\n", "if False:\n"),
+], ids=["no_ke", "no_qe", "no_ve", "no_wb", "no_dqe", "no_dp_wait", "no_store_read_ds", "no_store_read_stage"])
 def test_model_catches_planted_mistakes(monkeypatch, fn_name, old, new):
     """Each planted mistake in the protocol is caught on some schedule."""
     import tests.test_bwd_schedule_model as mod
     mutate(monkeypatch, mod, fn_name, old, new)
+    assert _caught(5)
+
+
+def test_acc_before_last_dq_is_caught(monkeypatch):
+    """dK, dV declared complete right after the item's last dK MMA: the rows
+    stage their dK/dV rows over dS^T that the last dQ MMA has not read yet."""
+    import tests.test_bwd_schedule_model as mod
+    monkeypatch.setattr(mod, "ACC_AFTER_DQ", False)
     assert _caught(5)
 
 
