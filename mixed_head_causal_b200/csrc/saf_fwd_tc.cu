@@ -63,7 +63,12 @@ constexpr uint32_t SM_V = SM_K + NSK * TILE_BYTES;
 // reads the same atom)
 constexpr uint32_t SM_ONES = SM_V + NSV * TILE_BYTES;
 constexpr uint32_t SM_BAR = SM_ONES + 2048;
-constexpr uint32_t SM_TOTAL = SM_BAR + 256;
+// replaced heads: what block g's W is built from, in stage g & 1: the 256 E
+// pairs [128 (I - j), + 256) of the padded array (1 KB), then the 64 c pairs
+// of the key block (256 B)
+constexpr uint32_t WST_E = 1024, WST_BYTES = 1280;
+constexpr uint32_t SM_WST = SM_BAR + 256;
+constexpr uint32_t SM_TOTAL = SM_WST + 2 * WST_BYTES;
 
 struct FwdTcParams {
     __nv_bfloat16* o;
@@ -213,16 +218,17 @@ __device__ __noinline__ bool diag_block(uint32_t tS, uint32_t tO, uint32_t tP, i
 }
 
 // W(i, j) = E[i-j] c_j for 64 keys (q0 = 0 or 8 selects the half): bf16 pair
-// products of the padded E pairs (walking down from row i) and the c pairs.
-__device__ __forceinline__ void build_w_half(const uint32_t* ep, const uint4* cp, int q0, uint32_t (&pw)[32]) {
+// products of the E pairs (walking down from row i; shared address e_row)
+// and the c pairs (shared address c0), both staged in shared memory.
+__device__ __forceinline__ void build_w_half(uint32_t e_row, uint32_t c0, int q0, uint32_t (&pw)[32]) {
 #pragma unroll
     for (int q4 = 0; q4 < 8; ++q4) {
-        const uint4 c4 = __ldg(cp + q0 + q4);
+        const uint4 c4 = ld_shared_u4(c0 + 16 * (q0 + q4));
         const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int mm = 4 * (q0 + q4) + u;  // key pair (2mm, 2mm+1)
-            const uint32_t e2 = __ldg(ep - 2 * mm);
+            const uint32_t e2 = ld_shared_u32(e_row - 8 * mm);
             __nv_bfloat162 prod = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&e2),
                                           *reinterpret_cast<const __nv_bfloat162*>(&cw[u]));
             pw[4 * q4 + u] = *reinterpret_cast<uint32_t*>(&prod);
@@ -285,9 +291,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_o = bar_p + 8;             // P.V done (ordinary head)
     const uint32_t bar_ob = bar_o + 8;            // [2] P.V of W buffer b done (replaced head)
     const uint32_t bar_pb = bar_ob + 16;          // [2] W buffer b written (replaced head, 4 warp arrivals)
+    const uint32_t bar_wf = bar_pb + 16;          // [2] W inputs of stage b landed (replaced head)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 232);
     int* item_slot = reinterpret_cast<int*>(smem + SM_BAR + 240);  // [2]
-    static_assert(16 * 4 + 16 * NSK + 16 * NSV + 32 + 32 <= 232, "barrier area");
+    static_assert(16 * 4 + 16 * NSK + 16 * NSV + 32 + 48 <= 232, "barrier area");
 
     const int T = p.T;
     const int total = p.BH * p.nqb;  // work items: one query block of one (b, h) slice
@@ -301,6 +308,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_init(bar_qe + 8 * b, 1);
             mbar_init(bar_ob + 8 * b, 1);
             mbar_init(bar_pb + 8 * b, 4);
+            mbar_init(bar_wf + 8 * b, 1);
         }
         for (int s = 0; s < NSK; ++s) {
             mbar_init(bar_kf + 8 * s, 1);
@@ -364,8 +372,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            int gk = 0, gv = 0, nq = 0;  // K blocks, V blocks, ordinary items so far
-            bool ok = true;
+            int gk = 0, gv = 0, gr = 0, nq = 0;  // K, V, replaced blocks; ordinary items so far
+            bool ok = true, waited = false;
             for (int n = 0; ok; ++n) {
                 const int w = (int)atomicAdd(p.err + kCtrFwdNext, 1u);
                 const int item = w < total ? w : -1;
@@ -394,12 +402,30 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (!it.rep && !load_k(0)) { ok = false; break; }
                 for (int j = 0; j < nkb; ++j) {
                     if (!it.rep && j + 1 < nkb && !load_k(j + 1)) { ok = false; break; }
+                    if (it.rep) {
+                        // the W inputs of replaced block g into stage g & 1, once the
+                        // rows have built block g - 2's W from it; the arrays come
+                        // from the pattern preparation, which a programmatic launch
+                        // may still be running: wait for it once
+                        const int g = gr + j, b = g & 1;
+                        if (!waited) {
+                            griddep_wait();
+                            waited = true;
+                        }
+                        if (g >= 2 && !mbar_wait(bar_pb + 8 * b, ((g >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
+                        const uint32_t st = sbase + SM_WST + b * WST_BYTES;
+                        mbar_expect_tx(bar_wf + 8 * b, WST_BYTES);
+                        bulk_load(st, p.w.epair + (size_t)it.slot * p.w.Lp + (size_t)(it.I - j) * BN, WST_E, bar_wf + 8 * b);
+                        bulk_load(st + WST_E, p.w.cpair + (size_t)it.slot * (p.w.Tp / 2) + (size_t)j * 64,
+                                  WST_BYTES - WST_E, bar_wf + 8 * b);
+                    }
                     const int g = gv + j, s = g % NSV, u = g / NSV;
                     if (!mbar_wait(bar_ve + 8 * s, (u & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                     mbar_expect_tx(bar_vf + 8 * s, TILE_BYTES);
                     tma_load_3d(sbase + SM_V + s * TILE_BYTES, &tmV, bar_vf + 8 * s, 0, j * BN, it.bhkv);
                 }
-                if (!it.rep) gk += nkb;
+                if (it.rep) gr += nkb;
+                else gk += nkb;
                 gv += nkb;
             }
             if (!ok) report(p.err, 0x101);
@@ -575,14 +601,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                         mbar_wait(bar_ob + 8 * (g & 1), ((g >> 1) & 1) ^ 1, kWaitLimit));
                         if (!ok) { report(p.err, 0x303); break; }
                     }
+                    // its inputs, staged by the producer
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_wf + 8 * (g & 1), (g >> 1) & 1, kWaitLimit));
+                    if (!ok) { report(p.err, 0x306); break; }
                     tc_fence_after();
                     if (!direct) {
                         uint32_t pw0[32], pw1[32];
-                        const uint32_t* ep = p.w.epair + (size_t)slot * p.w.Lp + 128 + (I - j) * BN + row;
-                        const uint4* cp =
-                            reinterpret_cast<const uint4*>(p.w.cpair + (size_t)slot * (p.w.Tp / 2) + j * 64);
-                        build_w_half(ep, cp, 0, pw0);
-                        build_w_half(ep, cp, 8, pw1);
+                        // E pair 128 + (I - j) BN + row - 2mm of the padded array is entry
+                        // 128 + row - 2mm of the staged window
+                        const uint32_t st = sbase + SM_WST + (g & 1) * WST_BYTES;
+                        build_w_half(st + 4 * (128 + row), st + WST_E, 0, pw0);
+                        build_w_half(st + 4 * (128 + row), st + WST_E, 8, pw1);
                         tmem_st32(tS + 64 * (g & 1), pw0);
                         tmem_st32(tS + 64 * (g & 1) + 32, pw1);
                     } else {

@@ -27,7 +27,7 @@ def all_of(res, version):
 
 
 def producer(m, items):
-    gk = gv = nq = 0  # K blocks, V blocks, ordinary items so far
+    gk = gv = gr = nq = 0  # K, V, replaced blocks; ordinary items so far
     for n, it in enumerate(items + [None]):
         yield from publish(m, n, it)
         if it is None:
@@ -50,11 +50,20 @@ def producer(m, items):
         for j in range(nkb):
             if not rep and j + 1 < nkb:
                 yield from load_k(j + 1)
+            if rep:
+                # a replaced block's W inputs (E and c) into stage gw & 1, once
+                # the rows have built block gw - 2 from it
+                gw = gr + j
+                if gw >= 2:
+                    yield W(f"pb{gw & 1}", (gw >> 1) - 1, ((gw >> 1) & 1) ^ 1)
+                m.copy(f"wf{gw & 1}", [(f"WST{gw & 1}", ("WIN", gw))], "producer")
             g = gv + j
             s, u = g % NSV, g // NSV
             yield W(f"ve{s}", u - 1, (u & 1) ^ 1)
             m.copy(f"vf{s}", [(f"V{s}", ("V", g))], "producer")
-        if not rep:
+        if rep:
+            gr += nkb
+        else:
             gk += nkb
         gv += nkb
 
@@ -121,20 +130,31 @@ def query_rows(m, w):
         rep, nkb = it
         for j in range(nkb):
             if not rep:
+                last = j == nkb - 1
                 yield W("s", go + j, (go + j) & 1)
                 m.read(f"S_lo.{w}", ("S", go + j), "rows")
                 m.read(f"S_hi.{w}", ("S", go + j), "rows")
-                m.bars["sf"].arrive()
+                if not last:
+                    m.bars["sf"].arrive()
                 if j > 0:
                     yield W("o", go + j - 1, (go + j - 1) & 1)
                     m.read(f"O.{w}", ("O", n, j - 1), "rows rescale")
                     m.write(f"O.{w}", ("O", n, j - 1), "rows rescale")
+                if last:
+                    # the diagonal block reads S a second time (its exp pass)
+                    # and releases it only then
+                    m.read(f"S_lo.{w}", ("S", go + j), "rows diagonal")
+                    m.read(f"S_hi.{w}", ("S", go + j), "rows diagonal")
                 m.write(f"P.{w}", ("P", go + j), "rows")
+                if last:
+                    m.bars["sf"].arrive()
                 m.bars["p"].arrive()
             else:
                 g = gr + j
                 if g >= 2:
                     yield W(f"ob{g & 1}", (g >> 1) - 1, ((g >> 1) & 1) ^ 1)
+                yield W(f"wf{g & 1}", g >> 1, (g >> 1) & 1)
+                m.read(f"WST{g & 1}", ("WIN", g), "rows W")
                 m.write(f"{'S_lo' if g % 2 == 0 else 'S_hi'}.{w}", ("W", g), "rows W")
                 m.bars[f"pb{g & 1}"].arrive()
         gl = (gr if rep else go) + nkb - 1  # the item's last P.V
@@ -155,7 +175,7 @@ def run(items, seed):
     for b in range(2):
         m.bar(f"itf{b}")
         m.bar(f"ite{b}", 1 + ROWS)  # the MMA warp and each row warp acknowledge an item
-        for name in ("qf", "qe", "ob"):
+        for name in ("qf", "qe", "ob", "wf"):
             m.bar(f"{name}{b}")
         m.bar(f"pb{b}", ROWS)
     for s in range(NSK):
@@ -222,7 +242,11 @@ def _caught(seed):
     ("producer", 'yield W(f"ke{s}", u - 1, (u & 1) ^ 1)', 'yield from ()'),
     # the next-but-one item's Q loaded over a Q still in use
     ("producer", 'yield W(f"qe{b}", (nq >> 1) - 1, ((nq >> 1) & 1) ^ 1)', 'pass'),
-], ids=["no_sf", "no_o", "no_ob", "no_ke", "no_qe"])
+    # a replaced block's W inputs staged over those the rows still build from
+    ("producer", "if gw >= 2:\n", "if False:\n"),
+    # the rows build W before its inputs have landed
+    ("query_rows", 'yield W(f"wf{g & 1}", g >> 1, (g >> 1) & 1)', 'pass'),
+], ids=["no_sf", "no_o", "no_ob", "no_ke", "no_qe", "no_pb_stage", "no_wf"])
 def test_model_catches_planted_mistakes(monkeypatch, fn_name, old, new):
     """Each planted mistake in the protocol is caught on some schedule."""
     import tests.test_fwd_schedule_model as mod
