@@ -218,7 +218,9 @@ cudaError_t launch_pattern_grad(const __nv_bfloat16* v, const __nv_bfloat16* dou
 cudaError_t launch_dq_convert(const float* dqacc, void* dq, int64_t rows, int grad_fp32, cudaStream_t stream);
 cudaError_t launch_group_sum(const float* src, void* dst, int B, int H, int Hkv, int T, int grad_fp32,
                              cudaStream_t stream);
-bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out, int box_rows = 128);
+// bf16 [BH, T, 64] as a 3-D tensor map (d, t, bh); boxes of box_rows x
+// box_cols (128 or 32 columns, with the 128- or 64-byte swizzle).
+bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out, int box_rows = 128, int box_cols = 64);
 bool make_tmap_bhtd_f32(const void* base, int BH, int T, CUtensorMap* out);
 // Warp-level (mma.sync) forward and backward of every head, the reference
 // path selected by SAF_FORCE_MMA.

@@ -68,7 +68,10 @@ constexpr uint32_t SM_BAR = SM_ONES + 2048;
 // of the key block (256 B)
 constexpr uint32_t WST_E = 1024, WST_BYTES = 1280;
 constexpr uint32_t SM_WST = SM_BAR + 256;
-constexpr uint32_t SM_TOTAL = SM_WST + 2 * WST_BYTES;
+// O staging: per row warp a 2 KB box (its 32 rows x 32 columns of bf16, the
+// 64-byte swizzle of the store map), stored to global by TMA twice per item
+constexpr uint32_t SM_OST = (SM_WST + 2 * WST_BYTES + 1023) & ~1023u;
+constexpr uint32_t SM_TOTAL = SM_OST + 4 * 2048;
 
 struct FwdTcParams {
     __nv_bfloat16* o;
@@ -81,6 +84,7 @@ struct FwdTcParams {
     int16_t slot_of_head[kMaxHeads];
     int H, Hkv, BH, T, nqb;  // query heads, K/V heads (H / Hkv query heads share one)
     int nslots;  // replaced heads
+    int tma_o;   // O written by TMA stores of 32 x 32 boxes (else per-thread row stores)
     float scale_log2;
 };
 
@@ -273,7 +277,8 @@ __device__ __noinline__ bool head_direct(const ReplacedWs& w, int s) {
 
 __global__ void __launch_bounds__(NTHREADS, 2)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const FwdTcParams p) {
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const FwdTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
@@ -649,6 +654,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     scale = (i < T && sum > 0.f) ? 1.f / sum : 0.f;
                 }
                 __nv_bfloat16* orow = p.o + ((size_t)bh * T + (i < T ? i : 0)) * kHeadDim;
+                // The warp's 32 rows go out as two 32-column TMA boxes through its
+                // 2 KB staging area (row `lane` at lane * 64, 16-byte chunks in the
+                // 64-byte swizzle); the warp moves on once a store is issued, where
+                // 32 per-thread row stores would block its next barrier waits.
+                // Rows past T are clipped by the store.
+                const uint32_t ost = sbase + SM_OST + quarter * 2048 + lane * 64;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t v[32];
@@ -659,7 +670,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     for (int e = 0; e < 16; ++e)
                         packed[e] =
                             pack_bf16x2(__uint_as_float(v[2 * e]) * scale, __uint_as_float(v[2 * e + 1]) * scale);
-                    if (i < T) {
+                    if (p.tma_o) {
+                        if (lane == 0) bulk_wait_read0();  // the previous box has been read
+                        __syncwarp();
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            st_shared_v4(ost + ((k ^ ((lane >> 1) & 3)) << 4), packed[4 * k], packed[4 * k + 1],
+                                         packed[4 * k + 2], packed[4 * k + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&tmO, sbase + SM_OST + quarter * 2048, 32 * c, I * BM + quarter * 32, bh);
+                            bulk_commit();
+                        }
+                    } else if (i < T) {
                         uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
@@ -674,6 +698,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (rep) gr += nkb;
             else go += nkb;
         }
+        if (lane == 0) bulk_wait0();  // the O stores complete before the CTA ends
     }
     tc_fence_before();
     __syncthreads();
@@ -727,16 +752,17 @@ int sm_count() {
 
 // [BH, T, 64] bf16 viewed as a 3-D tensor (d, t, bh); 128 x 64 boxes with the
 // 128-byte swizzle; rows past T read as zeros.
-bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out, int box_rows) {
+bool make_tmap_bhtd(const void* base, int BH, int T, CUtensorMap* out, int box_rows, int box_cols) {
     EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
+    if (!fn || (box_cols != 64 && box_cols != 32)) return false;
     cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)BH};
     cuuint64_t strides[2] = {64 * 2, (cuuint64_t)T * 64 * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -744,12 +770,16 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
                           __nv_bfloat16* o, float* lse, const float* a, const float* r, const float* logz,
                           const HeadList& hl, const ReplacedWs& w, int B, int H, int Hkv, int T, unsigned int* err,
                           bool after_pattern, cudaStream_t stream) {
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     const int BH = B * H;
     if (!make_tmap_bhtd(q, BH, T, &mq) || !make_tmap_bhtd(k, B * Hkv, T, &mk) ||
         !make_tmap_bhtd(v, B * Hkv, T, &mv))
         return cudaErrorNotSupported;
     FwdTcParams p;
+    // O by 32 x 32 TMA stores when its map encodes (a base the encoder
+    // rejects, e.g. not 16-byte aligned, takes the row stores)
+    p.tma_o = make_tmap_bhtd(o, BH, T, &mo, 32, 32) ? 1 : 0;
+    if (!p.tma_o) mo = mq;  // not read
     p.o = o;
     p.lse = lse;
     p.a = a;
@@ -789,7 +819,7 @@ cudaError_t launch_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_pattern ? 1 : 0;
-    cudaError_t le = cudaLaunchKernelEx(&cfg, fwd_tc_kernel, mq, mk, mv, p);
+    cudaError_t le = cudaLaunchKernelEx(&cfg, fwd_tc_kernel, mq, mk, mv, mo, p);
     launch_end(KID_FWD_TC, stream);
     if (le != cudaSuccess) return le;
     return cudaGetLastError();

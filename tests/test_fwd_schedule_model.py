@@ -123,6 +123,7 @@ def mma_issuer(m):
 def query_rows(m, w):
     go = gr = 0
     n = 0
+    ns = 0  # O boxes this warp has stored from its staging area
     while True:
         it = yield from take(m, n)
         if it is None:
@@ -163,6 +164,14 @@ def query_rows(m, w):
         else:
             yield W("o", gl, gl & 1)
         m.read(f"O.{w}", ("O", n, nkb - 1), "rows epilogue")
+        # two 32-column boxes through the warp's staging area, each written
+        # once the previous box's store has read it
+        for c in range(2):
+            if ns > 0:
+                yield W(f"sr{w}", ns - 1, (ns - 1) & 1)
+            m.write(f"OST.{w}", ("O box", n, c), "rows stage")
+            m.store(f"sr{w}", f"OST.{w}", ("O box", n, c), "O store")
+            ns += 1
         if rep:
             gr += nkb
         else:
@@ -188,6 +197,8 @@ def run(items, seed):
         m.bar(name)
     for name in ("sf", "p"):
         m.bar(name, ROWS)
+    for w in range(ROWS):
+        m.bar(f"sr{w}")
     roles = {"producer": producer(m, items), "mma": mma_issuer(m)}
     roles.update({f"rows{w}": query_rows(m, w) for w in range(ROWS)})
     simulate(m, roles, random.Random(seed))
@@ -246,7 +257,9 @@ def _caught(seed):
     ("producer", "if gw >= 2:\n", "if False:\n"),
     # the rows build W before its inputs have landed
     ("query_rows", 'yield W(f"wf{g & 1}", g >> 1, (g >> 1) & 1)', 'pass'),
-], ids=["no_sf", "no_o", "no_ob", "no_ke", "no_qe", "no_pb_stage", "no_wf"])
+    # an O box staged over the previous one before its store has read it
+    ("query_rows", "if ns > 0:\n", "if False:\n"),
+], ids=["no_sf", "no_o", "no_ob", "no_ke", "no_qe", "no_pb_stage", "no_wf", "no_store_read"])
 def test_model_catches_planted_mistakes(monkeypatch, fn_name, old, new):
     """Each planted mistake in the protocol is caught on some schedule."""
     import tests.test_fwd_schedule_model as mod
