@@ -224,9 +224,9 @@ def run_oracle_sample(w, slices, seed=0, threads=None):
 
 
 def cpu_baseline(w):
-    # four groups of the head-kind mix: 16 slices, about ten seconds of CPU
-    # work at the 124M shape on the machine's host cores
-    slices = oracle_sample(w, groups=4)
+    # sixteen groups of the head-kind mix: 64 slices, about eight seconds on
+    # 16 host cores at the 124M shape (half a minute on 4)
+    slices = oracle_sample(w, groups=16)
     dt, frac, cores = run_oracle_sample(w, slices)
     return {"value": w.tokens * frac / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{len(slices)} of {w.B * w.H} (batch, head) slices of {w.name} (same head-kind mix), "
