@@ -98,35 +98,45 @@ __device__ __forceinline__ uint32_t packed_col(int c) { return c < 2 ? 16 * c : 
 // A-operand column of MMA k-step k (16 queries) in that packing.
 __device__ __forceinline__ uint32_t packed_kcol(int k) { return k < 4 ? 8 * k : 64 + 8 * (k - 4); }
 
-// P^T for queries [32c, 32c + 32) of key row jl: exp2(S^T * scale - lse2),
-// packed as 16 bf16 pairs over TMEM columns packed_col(c) of the S^T region.
-// Shared memory at nlse2 holds -lse2 per query (read as pairs, 16 bytes at a
-// time, while the TMEM load is in flight); the scale-and-shift runs on paired
-// fp32 FMAs.  MASK: zero where the query precedes the key on the diagonal
-// tile, or where the key lies past T.
+// P^T for this warp's 64 queries [64 half, 64 half + 64) of key row jl:
+// exp2(S^T * scale - lse2), as bf16 pairs over the S^T columns already read
+// (the 32-query chunk c goes to packed_col(c)).  Shared memory at nlse2 holds
+// -lse2 per query (read as pairs, 16 bytes at a time); the scale-and-shift
+// runs on paired fp32 FMAs.  Four 16-query steps whose TMEM loads are double
+// buffered: the load of step k + 1 is in flight while step k is computed.
+// MASK: zero where the query precedes the key on the diagonal tile, or where
+// the key lies past T.
 template <bool MASK>
-__device__ __forceinline__ void p_chunk(uint32_t tS, int c, uint32_t nlse2, float scale, int jl, bool diag,
-                                        bool key_ok, uint32_t (&pw)[16]) {
-    uint32_t v[32];
-    tmem_ld32(tS + 32 * c, v);
-    uint64_t nl[16];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) ld_shared_2x64(nlse2 + 128 * c + 16 * q, nl[2 * q], nl[2 * q + 1]);
-    tmem_wait_ld();
+__device__ __forceinline__ void p_half(uint32_t tS, int half, uint32_t nlse2, float scale, int jl, bool diag,
+                                       bool key_ok, uint32_t (&pw)[2][16]) {
     const uint64_t sc2 = f32x2(scale, scale);
+    uint32_t va[16], vb[16];
+    tmem_ld16(tS + 64 * half, va);
+    tmem_wait_ld();
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        const int ql = 32 * c + e;
-        const float2 x =
-            split_f32x2(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nl[e / 2]));
-        float p0 = ex2(x.x), p1 = ex2(x.y);
-        if (MASK) {
-            if (!key_ok || (diag && ql < jl)) p0 = 0.f;
-            if (!key_ok || (diag && ql + 1 < jl)) p1 = 0.f;
+    for (int k = 0; k < 4; ++k) {
+        uint32_t(&cur)[16] = (k & 1) ? vb : va;
+        uint32_t(&nxt)[16] = (k & 1) ? va : vb;
+        if (k < 3) tmem_ld16(tS + 64 * half + 16 * (k + 1), nxt);
+        const int q0 = 64 * half + 16 * k;  // first query of the step
+        uint64_t nl[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ld_shared_2x64(nlse2 + 4 * q0 + 16 * q, nl[2 * q], nl[2 * q + 1]);
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+            const int ql = q0 + e;
+            const float2 x =
+                split_f32x2(fma_f32x2(f32x2(__uint_as_float(cur[e]), __uint_as_float(cur[e + 1])), sc2, nl[e / 2]));
+            float p0 = ex2(x.x), p1 = ex2(x.y);
+            if (MASK) {
+                if (!key_ok || (diag && ql < jl)) p0 = 0.f;
+                if (!key_ok || (diag && ql + 1 < jl)) p1 = 0.f;
+            }
+            pw[k >> 1][8 * (k & 1) + e / 2] = pack_bf16x2(p0, p1);
         }
-        pw[e / 2] = pack_bf16x2(p0, p1);
+        if (k & 1) tmem_st16(tS + packed_col(2 * half + (k >> 1)), pw[k >> 1]);
+        if (k < 3) tmem_wait_ld();
     }
-    tmem_st16(tS + packed_col(c), pw);
 }
 
 // Stores one 64-wide row of an fp32 accumulator (already scaled) as bf16 or fp32.
@@ -538,15 +548,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     // P^T stays in registers for dS^T: the S^T columns are reused by
                     // the next tile's S^T as soon as dV has read them.
                     uint32_t pw[2][16];
-                    if (t == 0 || it.ragged) {
-#pragma unroll
-                        for (int cc = 0; cc < 2; ++cc)
-                            p_chunk<true>(tS, 2 * half + cc, v1, p.scale_log2, jl, t == 0, j < T, pw[cc]);
-                    } else {
-#pragma unroll
-                        for (int cc = 0; cc < 2; ++cc)
-                            p_chunk<false>(tS, 2 * half + cc, v1, p.scale_log2, jl, false, true, pw[cc]);
-                    }
+                    if (t == 0 || it.ragged)
+                        p_half<true>(tS, half, v1, p.scale_log2, jl, t == 0, j < T, pw);
+                    else
+                        p_half<false>(tS, half, v1, p.scale_log2, jl, false, true, pw);
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(bar_p);
@@ -560,23 +565,34 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         if (lane == 0) bulk_wait_read0();
                         __syncwarp();
                     }
+                    // 16 queries per step, the TMEM load of the next step in flight
+                    uint32_t va[16], vb[16];
+                    tmem_ld16(tDP + 64 * half, va);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int c = 2 * half + cc;
-                        uint32_t v[32], dsw[16];
-                        tmem_ld32(tDP + 32 * c, v);
-                        uint64_t d2[16];
+                        uint32_t dsw[16];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) ld_shared_2x64(v2 + 128 * c + 16 * q, d2[2 * q], d2[2 * q + 1]);
-                        tmem_wait_ld();
+                        for (int k2 = 0; k2 < 2; ++k2) {
+                            const int k = 2 * cc + k2;
+                            uint32_t(&cur)[16] = (k & 1) ? vb : va;
+                            uint32_t(&nxt)[16] = (k & 1) ? va : vb;
+                            if (k < 3) tmem_ld16(tDP + 64 * half + 16 * (k + 1), nxt);
+                            uint64_t d2[8];
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            // (dP - D) paired, times P (bf16, widened), one rounding
-                            const float2 pf = unpack_bf16x2(pw[cc][e / 2]);
-                            const uint64_t g =
-                                sub_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), d2[e / 2]);
-                            const float2 ds = split_f32x2(mul_f32x2(f32x2(pf.x, pf.y), g));
-                            dsw[e / 2] = pack_bf16x2(ds.x, ds.y);
+                            for (int q = 0; q < 4; ++q)
+                                ld_shared_2x64(v2 + 4 * (64 * half + 16 * k) + 16 * q, d2[2 * q], d2[2 * q + 1]);
+#pragma unroll
+                            for (int e = 0; e < 16; e += 2) {
+                                // (dP - D) paired, times P (bf16, widened), one rounding
+                                const float2 pf = unpack_bf16x2(pw[cc][8 * k2 + e / 2]);
+                                const uint64_t g =
+                                    sub_f32x2(f32x2(__uint_as_float(cur[e]), __uint_as_float(cur[e + 1])), d2[e / 2]);
+                                const float2 ds = split_f32x2(mul_f32x2(f32x2(pf.x, pf.y), g));
+                                dsw[8 * k2 + e / 2] = pack_bf16x2(ds.x, ds.y);
+                            }
+                            if (k < 3) tmem_wait_ld();
                         }
                         tmem_st16(tDP + packed_col(c), dsw);
                         // queries [64 half, 64 half + 64) form the MN atom `half`
