@@ -62,7 +62,8 @@ constexpr uint32_t SM_DQ = SM_DS + 2 * TILE;
 constexpr uint32_t SM_VEC1 = SM_DQ + 2 * TILE;        // NQS x 512 B: -lse2 (ordinary) / r (replaced)
 constexpr uint32_t SM_VEC2 = SM_VEC1 + 512 * NQS;  // NQS x 512 B: D
 constexpr uint32_t SM_BAR = SM_VEC2 + 512 * NQS;
-constexpr uint32_t SM_DFL = SM_BAR + 256;  // per replaced slot: 1 = per-element path
+// (SM_BAR + 256: the two work-item slots, 16 bytes each)
+constexpr uint32_t SM_DFL = SM_BAR + 512;  // per replaced slot: 1 = per-element path
 constexpr uint32_t SM_TOTAL = SM_DFL + 256;
 
 struct BwdTcParams {
@@ -214,7 +215,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_wb = bar_acr + 8;    // [2] replaced head: W buffer b consumed
     const uint32_t bar_pb = bar_wb + 16;    // [2] replaced head: W buffer b written (256 arrivals)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 240);
-    int* item_slot = reinterpret_cast<int*>(smem + SM_BAR + 248);  // [2]
+    // [2] work item n & 1, decoded by the producer: {word (-1: none left), bh, J, h}
+    const uint32_t item_slot = sb + SM_BAR + 256;
     static_assert(80 + 16 * NQS + 112 <= 240, "barrier area");
 
     const int T = p.T;
@@ -259,13 +261,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     // Work item n of this CTA (-1: none left), published by the producer
     // through a 2-slot ring; every consumer warp acknowledges it.
-    auto take_item = [&](int n, int& item) -> bool {
-        if (!mbar_wait(bar_itf + 8 * (n & 1), (n >> 1) & 1, kWaitLimit)) return false;
-        item = *reinterpret_cast<volatile int*>(item_slot + (n & 1));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_ite + 8 * (n & 1));
-        return true;
-    };
     // (b, h) slice and key block of an item, grouped longest-first order (key
     // block J walks nqb - J query blocks; a group's Q/dO tiles and dQ
     // accumulator rows stay in L2)
@@ -290,6 +285,26 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         it.ragged = (it.J + 1) * BN > T;  // the key block runs past T
         return it;
     };
+    // Work item n of this CTA (-1: none left), published by the producer,
+    // already decoded, through a 2-slot ring; every consumer warp acknowledges
+    // it.
+    auto take_item = [&](int n, int& item, Item& it) -> bool {
+        if (!mbar_wait(bar_itf + 8 * (n & 1), (n >> 1) & 1, kWaitLimit)) return false;
+        const uint4 w = ld_shared_u4(item_slot + 16 * (n & 1));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ite + 8 * (n & 1));
+        item = (int)w.x;
+        it.bh = (int)w.y;
+        it.J = (int)w.z;
+        it.h = (int)w.w;
+        it.bhkv = -1;  // the producer's alone
+        it.slot = item >= 0 ? p.slot_of_head[it.h] : -1;
+        it.rep = it.slot >= 0;
+        it.direct = it.rep && ((item >> 30) & 1) != 0;
+        it.ntiles = p.nqb - it.J;
+        it.ragged = (it.J + 1) * BN > T;
+        return true;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -303,15 +318,18 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (int n = 0; ok; ++n) {
                 const int w = (int)atomicAdd(p.err + kCtrBwdNext, 1u);
                 int item = w < total ? w : -1;
+                Item it{};
                 if (item >= 0) {
-                    const Item pre = decode(item);
-                    if (pre.rep && dfl[pre.slot]) item |= 1 << 30;
+                    it = decode(item);
+                    if (it.rep && dfl[it.slot]) {
+                        item |= 1 << 30;
+                        it.direct = true;
+                    }
                 }
                 if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
-                *reinterpret_cast<volatile int*>(item_slot + (n & 1)) = item;
+                st_shared_v4(item_slot + 16 * (n & 1), (uint32_t)item, (uint32_t)it.bh, (uint32_t)it.J, (uint32_t)it.h);
                 mbar_arrive(bar_itf + 8 * (n & 1));
                 if (item < 0) break;
-                const Item it = decode(item);
                 if (!it.rep) {
                     // K of the key block into stage nk & 1, once the MMAs of the
                     // ordinary item two before (the stage's last user) are done;
@@ -372,13 +390,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         for (int n = 0; ok; ++n) {
             int item;
-            ok = __all_sync(0xffffffffu, take_item(n, item));
+            Item it;
+            ok = __all_sync(0xffffffffu, take_item(n, item, it));
             if (!ok) {
                 if (lane == 0) report(p.err, 0x1208);
                 break;
             }
             if (item < 0) break;
-            const Item it = decode(item);
             int okl = 1;
             if (lane == 0) {
                 if (!it.rep) {
@@ -522,13 +540,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         for (int n = 0; ok; ++n) {
             int item;
-            ok = __all_sync(0xffffffffu, take_item(n, item));
+            Item it;
+            ok = __all_sync(0xffffffffu, take_item(n, item, it));
             if (!ok) {
                 report(p.err, 0x1306);
                 break;
             }
             if (item < 0) break;
-            const Item it = decode(item);
             const int j = it.J * BN + jl;
             const float aj = (it.direct && j < T) ? p.a[(size_t)it.h * T + j] : kNegInf;
             for (int t = 0; t < it.ntiles; ++t) {
@@ -727,13 +745,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         for (int n = 0; ok; ++n) {
             int item;
-            ok = __all_sync(0xffffffffu, take_item(n, item));
+            Item it;
+            ok = __all_sync(0xffffffffu, take_item(n, item, it));
             if (!ok) {
                 report(p.err, 0x1402);
                 break;
             }
             if (item < 0) break;
-            const Item it = decode(item);
             if (it.rep) continue;  // a replaced head adds nothing to dQ
             for (int t = 0; t < it.ntiles; ++t, ++go) {
                 const int I = it.J + t, b = go & 1;

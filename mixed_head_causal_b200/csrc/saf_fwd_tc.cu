@@ -67,7 +67,7 @@ constexpr uint32_t SM_BAR = SM_ONES + 2048;
 // pairs [128 (I - j), + 256) of the padded array (1 KB), then the 64 c pairs
 // of the key block (256 B)
 constexpr uint32_t WST_E = 1024, WST_BYTES = 1280;
-constexpr uint32_t SM_WST = SM_BAR + 256;
+constexpr uint32_t SM_WST = SM_BAR + 512;  // (SM_BAR + 256: the two work-item slots, 16 bytes each)
 // O staging: per row warp a 2 KB box (its 32 rows x 32 columns of bf16, the
 // 64-byte swizzle of the store map), stored to global by TMA twice per item
 constexpr uint32_t SM_OST = (SM_WST + 2 * WST_BYTES + 1023) & ~1023u;
@@ -298,7 +298,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t bar_pb = bar_ob + 16;          // [2] W buffer b written (replaced head, 4 warp arrivals)
     const uint32_t bar_wf = bar_pb + 16;          // [2] W inputs of stage b landed (replaced head)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SM_BAR + 232);
-    int* item_slot = reinterpret_cast<int*>(smem + SM_BAR + 240);  // [2]
+    // [2] work item n & 1, decoded by the producer: {item (-1: none left), bh, I, h}
+    const uint32_t item_slot = sbase + SM_BAR + 256;
     static_assert(16 * 4 + 16 * NSK + 16 * NSV + 32 + 48 <= 232, "barrier area");
 
     const int T = p.T;
@@ -344,15 +345,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    // Work item n of this CTA (-1: none left), published by the producer
-    // through a 2-slot ring; every consumer warp acknowledges it.
-    auto take_item = [&](int n, int& item) -> bool {
-        if (!mbar_wait(bar_itf + 8 * (n & 1), (n >> 1) & 1, kWaitLimit)) return false;
-        item = *reinterpret_cast<volatile int*>(item_slot + (n & 1));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_ite + 8 * (n & 1));
-        return true;
-    };
     // (b, h) slice and query block of an item, grouped longest-first order
     // (query block I visits I + 1 key blocks)
     struct Item {
@@ -370,6 +362,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         it.rep = it.slot >= 0;
         return it;
     };
+    // Work item n of this CTA (-1: none left), published by the producer,
+    // already decoded, through a 2-slot ring; every consumer warp acknowledges
+    // it.
+    auto take_item = [&](int n, int& item, Item& it) -> bool {
+        if (!mbar_wait(bar_itf + 8 * (n & 1), (n >> 1) & 1, kWaitLimit)) return false;
+        const uint4 w = ld_shared_u4(item_slot + 16 * (n & 1));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ite + 8 * (n & 1));
+        item = (int)w.x;
+        it.bh = (int)w.y;
+        it.I = (int)w.z;
+        it.h = (int)w.w;
+        it.bhkv = -1;  // the producer's alone
+        it.slot = item >= 0 ? p.slot_of_head[it.h] : -1;
+        it.rep = it.slot >= 0;
+        return true;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -382,11 +391,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (int n = 0; ok; ++n) {
                 const int w = (int)atomicAdd(p.err + kCtrFwdNext, 1u);
                 const int item = w < total ? w : -1;
+                const Item it = item >= 0 ? decode(item) : Item{0, 0, 0, 0, -1, false};
                 if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
-                *reinterpret_cast<volatile int*>(item_slot + (n & 1)) = item;
+                st_shared_v4(item_slot + 16 * (n & 1), (uint32_t)item, (uint32_t)it.bh, (uint32_t)it.I, (uint32_t)it.h);
                 mbar_arrive(bar_itf + 8 * (n & 1));
                 if (item < 0) break;
-                const Item it = decode(item);
                 const int nkb = it.I + 1;
                 if (!it.rep) {
                     const int b = nq & 1;
@@ -450,10 +459,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool ok = true;
         for (int n = 0; ok; ++n) {
             int item;
-            ok = __all_sync(0xffffffffu, take_item(n, item));
+            Item it;
+            ok = __all_sync(0xffffffffu, take_item(n, item, it));
             if (!ok) { if (lane == 0) report(p.err, 0x205); break; }
             if (item < 0) break;
-            const Item it = decode(item);
             const int nkb = it.I + 1;
             if (lane == 0) {
                 const int b = nq & 1;
@@ -538,19 +547,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bool waited = false;
         bool ok = true;
         for (int n = 0; ok; ++n) {
-            int item;
-            ok = __all_sync(0xffffffffu, take_item(n, item));
-            if (!ok) { report(p.err, 0x305); break; }
-            if (item < 0) break;
-            int I, slot, h;
+            int item, I, slot, h, bh;
             bool rep, direct = false;
             {
-                const Item it = decode(item);
+                Item it;
+                ok = __all_sync(0xffffffffu, take_item(n, item, it));
                 I = it.I;
                 slot = it.slot;
                 h = it.h;
+                bh = it.bh;
                 rep = it.rep;
             }
+            if (!ok) { report(p.err, 0x305); break; }
+            if (item < 0) break;
             if (rep) {
                 if (!waited) {
                     griddep_wait();
@@ -637,7 +646,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (!ok) report(p.err, 0x304);
             }
             tc_fence_after();
-            const int bh = decode(item).bh;
             if (ok) {
                 float scale = 0.f, lse_v = kNegInf;
                 if (i < T) {
