@@ -130,8 +130,10 @@ def test_lognorm_entry_point_and_explicit_logz():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     d1 = saf.mixed_attn_bwd(g["q"], g["k"], g["v"], o1, g["do"], l1, g["alpha"], g["rho"], x["mask"])
     d2 = saf.mixed_attn_bwd(g["q"], g["k"], g["v"], o1, g["do"], l1, g["alpha"], g["rho"], x["mask"], logz=lz)
-    for a, b in zip(d1, d2):
-        assert torch.equal(a, b)
+    # dK, dV bit-exact; dQ up to the order of its fp32 reduce-adds across CTAs
+    assert torch.equal(d1[1], d2[1]) and torch.equal(d1[2], d2[2])
+    scale = max(1.0, d1[0].abs().max().item())
+    assert (d1[0].float() - d2[0].float()).abs().max().item() <= 1e-5 * scale
 
 
 @pytest.mark.parametrize("T", [1, 31, 32, 257, 545, 4101])
