@@ -543,7 +543,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // arrays, their range flags, log Z); with a programmatic launch this
         // kernel may start before that grid ends, so the row warps wait for it
         // at their first replaced item.  A head's per-element flag (any of its
-        // tiles' range flags) is found then and cached per warp (slots < 32).
+        // tiles' range flags) is read at each of its items.
         bool waited = false;
         bool ok = true;
         for (int n = 0; ok; ++n) {
