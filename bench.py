@@ -141,6 +141,19 @@ class ClockSampler:
                 "samples": len(loaded), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
 
 
+# The sources a tensor-core kernel is built from: its own file and the two
+# headers every kernel file includes.
+KERNEL_SOURCES = {"fwd_tc": "saf_fwd_tc.cu", "bwd_tc": "saf_bwd_tc.cu"}
+
+
+def kernel_source_hash(kernel):
+    csrc = os.path.join(ROOT, "mixed_head_causal_b200", "csrc")
+    own = KERNEL_SOURCES.get(kernel)
+    if own is None:
+        return None
+    return source_hash([os.path.join(csrc, f) for f in (own, "saf_common.cuh", "tc_util.cuh")])
+
+
 def source_hash(paths):
     h = hashlib.sha256()
     for p in sorted(paths):
@@ -491,8 +504,7 @@ def our_arm(args, world, rank, local):
     if os.path.exists(tpath):
         with open(tpath) as f:
             tj = json.load(f)
-        csrc = os.path.join(ROOT, "mixed_head_causal_b200", "csrc")
-        cur = source_hash([os.path.join(csrc, f) for f in os.listdir(csrc)])
+        cur = kernel_source_hash(dom)
         ent = tj.get(dom)
         if ent and ent.get("source_hash") == cur and ent.get("workload") == w.name:
             traffic = ent.get("bytes_per_launch")
