@@ -110,22 +110,21 @@ __device__ __forceinline__ float row_max(const uint32_t (&v)[128]) {
     return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// P = exp2(s * scale - m) for the 128 keys of the block as 64 bf16 pairs;
-// returns the sum of the (unrounded) probabilities.  The scale-and-shift and
-// the running sums use the paired fp32 instructions (same rounding as the
-// scalar ones).
-__device__ __forceinline__ float exp_row(const uint32_t (&v)[128], float scale, float m, uint32_t (&pw)[64]) {
-    const uint64_t sc2 = f32x2(scale, scale), nm2 = f32x2(-m, -m);
-    uint64_t l2[4] = {0, 0, 0, 0};
+// P = exp2(s * scale - m) for keys [64 Q, 64 Q + 64) of the block (Q = 0 or
+// 1) as 32 bf16 pairs; the (unrounded) probabilities are added to the paired
+// sums l2.  The scale-and-shift (sc2 = scale, nm2 = -m, paired) and the sums
+// use the paired fp32 instructions (same rounding as the scalar ones).
+template <int Q>
+__device__ __forceinline__ void exp_half(const uint32_t (&v)[128], uint64_t sc2, uint64_t nm2, uint64_t (&l2)[4],
+                                         uint32_t (&pw)[32]) {
 #pragma unroll
-    for (int e = 0; e < 128; e += 2) {
-        const float2 x = split_f32x2(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2, nm2));
+    for (int e = 0; e < 64; e += 2) {
+        const float2 x = split_f32x2(
+            fma_f32x2(f32x2(__uint_as_float(v[64 * Q + e]), __uint_as_float(v[64 * Q + e + 1])), sc2, nm2));
         const float p0 = ex2(x.x), p1 = ex2(x.y);
         l2[(e >> 1) & 3] = add_f32x2(l2[(e >> 1) & 3], f32x2(p0, p1));
         pw[e >> 1] = pack_bf16x2(p0, p1);
     }
-    const float2 a = split_f32x2(add_f32x2(add_f32x2(l2[0], l2[1]), add_f32x2(l2[2], l2[3])));
-    return a.x + a.y;
 }
 
 // Rescales this warp's 32 O rows by f (a whole-warp TMEM round trip, taken
@@ -591,19 +590,31 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         // row max of the block (the scale is positive); every row of
                         // a visited block has a visible key, so it is finite
                         const float f = update_max(row_max(v) * p.scale_log2, m, l);
-                        uint32_t pw[64];  // P as bf16 pairs
-                        l += exp_row(v, p.scale_log2, m, pw);
                         // P_j replaces P_{j-1} in TMEM once P.V_{j-1} has read it (the
-                        // previous item's last P.V was waited for by its epilogue); the
-                        // O rows are rescaled once that P.V has landed in O
+                        // previous item's last P.V was waited for by its epilogue), which
+                        // is done by now as a rule.  P then goes to TMEM 64 keys at a time,
+                        // so only half of it is held in registers; the O rows are rescaled
+                        // after (that P.V has landed in O; P.V_j waits for this warp)
                         if (j > 0) {
                             ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (go + j - 1) & 1, kWaitLimit));
                             if (!ok) { report(p.err, 0x302); break; }
                             tc_fence_after();
                         }
+                        const uint64_t sc2 = f32x2(p.scale_log2, p.scale_log2), nm2 = f32x2(-m, -m);
+                        uint64_t l2[4] = {0, 0, 0, 0};
+                        {
+                            uint32_t pw[32];  // P as bf16 pairs, keys 0..63
+                            exp_half<0>(v, sc2, nm2, l2, pw);
+                            tmem_st32(tP, pw);
+                        }
+                        {
+                            uint32_t pw[32];  // keys 64..127
+                            exp_half<1>(v, sc2, nm2, l2, pw);
+                            tmem_st32(tP + 32, pw);
+                        }
+                        const float2 ls = split_f32x2(add_f32x2(add_f32x2(l2[0], l2[1]), add_f32x2(l2[2], l2[3])));
+                        l += ls.x + ls.y;
                         rescale_o(tO, f);
-                        tmem_st32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
-                        tmem_st32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
                     }
                 } else {
                     // W(i,j) = E[i-j] c_j, bf16 pairs, into buffer g & 1 (g counts
