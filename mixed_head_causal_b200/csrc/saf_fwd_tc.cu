@@ -110,17 +110,17 @@ __device__ __forceinline__ float row_max(const uint32_t (&v)[128]) {
     return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// P = exp2(s * scale - m) for keys [64 Q, 64 Q + 64) of the block (Q = 0 or
-// 1) as 32 bf16 pairs; the (unrounded) probabilities are added to the paired
+// P = exp2(s * scale - m) for keys [32 Q, 32 Q + 32) of the block (Q = 0..3)
+// as 16 bf16 pairs; the (unrounded) probabilities are added to the paired
 // sums l2.  The scale-and-shift (sc2 = scale, nm2 = -m, paired) and the sums
 // use the paired fp32 instructions (same rounding as the scalar ones).
 template <int Q>
-__device__ __forceinline__ void exp_half(const uint32_t (&v)[128], uint64_t sc2, uint64_t nm2, uint64_t (&l2)[4],
-                                         uint32_t (&pw)[32]) {
+__device__ __forceinline__ void exp_quarter(const uint32_t (&v)[128], uint64_t sc2, uint64_t nm2, uint64_t (&l2)[4],
+                                            uint32_t (&pw)[16]) {
 #pragma unroll
-    for (int e = 0; e < 64; e += 2) {
+    for (int e = 0; e < 32; e += 2) {
         const float2 x = split_f32x2(
-            fma_f32x2(f32x2(__uint_as_float(v[64 * Q + e]), __uint_as_float(v[64 * Q + e + 1])), sc2, nm2));
+            fma_f32x2(f32x2(__uint_as_float(v[32 * Q + e]), __uint_as_float(v[32 * Q + e + 1])), sc2, nm2));
         const float p0 = ex2(x.x), p1 = ex2(x.y);
         l2[(e >> 1) & 3] = add_f32x2(l2[(e >> 1) & 3], f32x2(p0, p1));
         pw[e >> 1] = pack_bf16x2(p0, p1);
@@ -592,8 +592,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         const float f = update_max(row_max(v) * p.scale_log2, m, l);
                         // P_j replaces P_{j-1} in TMEM once P.V_{j-1} has read it (the
                         // previous item's last P.V was waited for by its epilogue), which
-                        // is done by now as a rule.  P then goes to TMEM 64 keys at a time,
-                        // so only half of it is held in registers; the O rows are rescaled
+                        // is done by now as a rule.  P then goes to TMEM 32 keys at a time,
+                        // so only a quarter of it is held in registers; the O rows are rescaled
                         // after (that P.V has landed in O; P.V_j waits for this warp)
                         if (j > 0) {
                             ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (go + j - 1) & 1, kWaitLimit));
@@ -603,14 +603,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         const uint64_t sc2 = f32x2(p.scale_log2, p.scale_log2), nm2 = f32x2(-m, -m);
                         uint64_t l2[4] = {0, 0, 0, 0};
                         {
-                            uint32_t pw[32];  // P as bf16 pairs, keys 0..63
-                            exp_half<0>(v, sc2, nm2, l2, pw);
-                            tmem_st32(tP, pw);
+                            uint32_t pw[16];  // P as bf16 pairs, keys 0..31
+                            exp_quarter<0>(v, sc2, nm2, l2, pw);
+                            tmem_st16(tP, pw);
                         }
                         {
-                            uint32_t pw[32];  // keys 64..127
-                            exp_half<1>(v, sc2, nm2, l2, pw);
-                            tmem_st32(tP + 32, pw);
+                            uint32_t pw[16];
+                            exp_quarter<1>(v, sc2, nm2, l2, pw);
+                            tmem_st16(tP + 16, pw);
+                        }
+                        {
+                            uint32_t pw[16];
+                            exp_quarter<2>(v, sc2, nm2, l2, pw);
+                            tmem_st16(tP + 32, pw);
+                        }
+                        {
+                            uint32_t pw[16];
+                            exp_quarter<3>(v, sc2, nm2, l2, pw);
+                            tmem_st16(tP + 48, pw);
                         }
                         const float2 ls = split_f32x2(add_f32x2(add_f32x2(l2[0], l2[1]), add_f32x2(l2[2], l2[3])));
                         l += ls.x + ls.y;
