@@ -54,7 +54,9 @@ class Machine:
         self.inflight = set()  # resources a TMA copy is writing
         self.pipe = []         # issued MMAs / commits not yet executed
         self.tma = []          # (barrier, units, resources) copies in flight
-        self.stores = []       # (barrier, resource, version, who) stores in flight
+        self.stores = []       # (issuer key, resource, version, who, number) stores in flight
+        self.store_seq = {}    # issuer key -> stores made
+        self.store_done = {}   # issuer key -> numbers of the stores that have read their source
         self.slot = [None, None]
 
     def bar(self, name, count=1):
@@ -101,14 +103,20 @@ class Machine:
 
     def store(self, bar, res, want, who):
         """A bulk store out of shared memory: reads `res` (which must still hold
-        `want`) whenever it runs, then arrives on `bar` (the issuer's wait for
-        its stores to have read their source)."""
-        self.stores.append((bar, res, want, who))
+        `want`) whenever it runs, in any order with the issuer's other stores;
+        `bar` names the issuer's stores for its bulk-group waits (WC)."""
+        seq = self.store_seq.get(bar, 0)
+        self.store_seq[bar] = seq + 1
+        self.stores.append((bar, res, want, who, seq))
 
     def step_store(self, i):
-        bar, res, want, who = self.stores.pop(i)
+        bar, res, want, who, seq = self.stores.pop(i)
         self.read(res, want, who)
-        self.bars[bar].arrive()
+        self.store_done.setdefault(bar, set()).add(seq)
+
+    def stores_done_below(self, bar, upto):
+        done = self.store_done.get(bar, set())
+        return all(q in done for q in range(upto))
 
     def step_tma(self, i):
         bar, units, resources = self.tma.pop(i)
@@ -119,6 +127,14 @@ class Machine:
 
 def W(name, k, parity):
     return ("wait", name, k, parity)
+
+
+def WC(name, upto):
+    """A bulk-group wait: until every store the issuer made through `name`
+    before its store number `upto` (counted from 0) has read its source, the
+    later ones may still be pending (cp.async.bulk.wait_group.read N leaves
+    the N most recent groups pending).  No phase parity is involved."""
+    return ("count", name, upto, None)
 
 
 def take(m, n):
@@ -149,7 +165,11 @@ def simulate(m, roles, rng, max_steps=200000):
         for name, w in waiting.items():
             if w is None:
                 continue
-            _, bname, k, parity = w
+            kind, bname, k, parity = w
+            if kind == "count":
+                if m.stores_done_below(bname, k):
+                    ready.append(("role", name))
+                continue
             bar = m.bars[bname]
             if (name, bname, k) not in checked:
                 checked.add((name, bname, k))

@@ -21,7 +21,7 @@ import random
 
 import pytest
 
-from tests.schedule_model import Machine, ModelError, W, mutate, publish, simulate, take
+from tests.schedule_model import Machine, ModelError, W, WC, mutate, publish, simulate, take
 
 NQS = 3  # Q/dO ring depth
 # dK, dV are declared complete (bar_acc) after the item's last dQ MMA, the
@@ -171,7 +171,7 @@ def key_rows(m, w):
                 m.read(f"C_DP.{w}", ("dP", go), "rows dS")
                 m.read(f"VEC2_{s}", ("VEC", g), "rows dS")
                 if t == 0 and ns > 0:  # the last box has been read out of DS.w
-                    yield W(f"sr{w}", ns - 1, (ns - 1) & 1)
+                    yield WC(f"sr{w}", ns)
                 m.write(f"C_DP.{w}", ("dS", go), "rows dS")
                 m.write(f"DS.{w}", ("dS", go), "rows dS")
                 m.bars["ds"].arrive()
@@ -193,7 +193,7 @@ def key_rows(m, w):
         # the warp's dK or dV rows staged in its slice of the dS^T area, then
         # stored out by one bulk store (after the previous one has read it)
         if ns > 0:
-            yield W(f"sr{w}", ns - 1, (ns - 1) & 1)
+            yield WC(f"sr{w}", ns)
         m.write(f"DS.{w}", ("stage", n), "rows stage")
         m.store(f"sr{w}", f"DS.{w}", ("stage", n), "dK/dV store")
         ns += 1
@@ -235,8 +235,6 @@ def run(items, seed):
         m.bar(name)
     for name in ("p", "ds", "acr"):
         m.bar(name, ROWS)
-    for w in range(ROWS):
-        m.bar(f"sr{w}")
     roles = {"producer": producer(m, items), "mma": mma_issuer(m)}
     roles.update({f"rows{w}": key_rows(m, w) for w in range(ROWS)})
     roles.update({f"dq{w}": dq_warp(m, w) for w in range(DQW)})

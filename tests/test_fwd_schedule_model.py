@@ -15,7 +15,7 @@ import random
 
 import pytest
 
-from tests.schedule_model import Machine, ModelError, W, mutate, publish, simulate, take
+from tests.schedule_model import Machine, ModelError, W, WC, mutate, publish, simulate, take
 
 NSK = NSV = 2  # K, V ring stages
 ROWS = 4       # query-row warps: each owns one lane quarter of S, P and O
@@ -165,10 +165,10 @@ def query_rows(m, w):
             yield W("o", gl, gl & 1)
         m.read(f"O.{w}", ("O", n, nkb - 1), "rows epilogue")
         # two 32-column boxes through the warp's staging area, each written
-        # once the previous box's store has read it
+        # once every earlier store has read it (a bulk-group wait for all)
         for c in range(2):
             if ns > 0:
-                yield W(f"sr{w}", ns - 1, (ns - 1) & 1)
+                yield WC(f"sr{w}", ns)
             m.write(f"OST.{w}", ("O box", n, c), "rows stage")
             m.store(f"sr{w}", f"OST.{w}", ("O box", n, c), "O store")
             ns += 1
@@ -197,8 +197,6 @@ def run(items, seed):
         m.bar(name)
     for name in ("sf", "p"):
         m.bar(name, ROWS)
-    for w in range(ROWS):
-        m.bar(f"sr{w}")
     roles = {"producer": producer(m, items), "mma": mma_issuer(m)}
     roles.update({f"rows{w}": query_rows(m, w) for w in range(ROWS)})
     simulate(m, roles, random.Random(seed))
