@@ -321,6 +321,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 Item it{};
                 if (item >= 0) {
                     it = decode(item);
+                    if (!SAF_CHECKED_OK(p.err,
+                                        it.bh >= 0 && it.bh < p.BH && it.J >= 0 && it.J < p.nqb && it.h >= 0 &&
+                                            it.h < p.H && it.slot < p.nslots && it.bhkv >= 0 &&
+                                            it.bhkv < (p.BH / p.H) * p.Hkv,
+                                        0x9201u)) {
+                        ok = false;
+                        break;
+                    }
                     if (it.rep && dfl[it.slot]) {
                         item |= 1 << 30;
                         it.direct = true;
@@ -350,6 +358,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         mbar_expect_tx(bq, 2 * TILE + 1024);
                         tma_load_3d(sb + SM_Q + s * TILE, &tmQ, bq, 0, I * BM, it.bh);
                         tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, it.bh);
+                        if (!SAF_CHECKED_OK(p.err, I < p.nqb && (size_t)I * BM + BM <= (size_t)p.Tp, 0x9202u)) {
+                            ok = false;
+                            break;
+                        }
                         bulk_load(sb + SM_VEC1 + 512 * s, p.nlse2p + (size_t)it.bh * p.Tp + I * BM, 512, bq);
                         bulk_load(sb + SM_VEC2 + 512 * s, p.dvecp + (size_t)it.bh * p.Tp + I * BM, 512, bq);
                         if (t == 0) {
@@ -361,6 +373,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     } else {
                         mbar_expect_tx(bq, TILE + 512);
                         tma_load_3d(sb + SM_DO + s * TILE, &tmDO, bq, 0, I * BM, it.bh);
+                        if (!SAF_CHECKED_OK(p.err, it.slot >= 0 && I < p.nqb && (size_t)I * BM + BM <= (size_t)p.w.Tp,
+                                            0x9203u)) {
+                            ok = false;
+                            break;
+                        }
                         bulk_load(sb + SM_VEC1 + 512 * s, p.w.rsc + (size_t)it.slot * p.w.Tp + I * BM, 512, bq);
                     }
                     if (++s == NQS) {
@@ -642,6 +659,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     tc_fence_after();
                     if (!it.direct) {
                         const float* ef = p.w.ef + (size_t)it.slot * p.w.Lp + 128 + (I - it.J) * BM - jl;
+                        // the 64 entries this thread reads lie inside the slot's padded array
+                        const int e_lo = 128 + (I - it.J) * BM - jl + 64 * half;
+                        const bool win_ok = SAF_CHECKED_OK(p.err, e_lo >= 0 && e_lo + 64 <= p.w.Lp, 0x9204u);
 #pragma unroll
                         for (int cc = 0; cc < 2; ++cc) {
                             const int c = 2 * half + cc;
@@ -653,8 +673,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                                 const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
                                 for (int u = 0; u < 4; u += 2) {
-                                    const float w0 = __ldg(ef + ql + u) * rr[u];
-                                    const float w1 = __ldg(ef + ql + u + 1) * rr[u + 1];
+                                    const float w0 = win_ok ? __ldg(ef + ql + u) * rr[u] : 0.f;
+                                    const float w1 = win_ok ? __ldg(ef + ql + u + 1) * rr[u + 1] : 0.f;
                                     const uint32_t hb = pack_bf16x2(w0, w1);
                                     const float2 hf = unpack_bf16x2(hb);
                                     hw[(e + u) / 2] = hb;

@@ -145,6 +145,25 @@ struct WsHeader {
 // (the last one resets both to zero for the next launch).
 constexpr int kCtrFwdNext = 2, kCtrFwdDone = 3, kCtrBwdNext = 4, kCtrBwdDone = 5;
 
+// Index checks of the checked build (compiled with -DSAF_CHECKED, built as
+// libsaf_checked.so for tests): SAF_CHECKED_OK(err, cond, code) is `cond`
+// there and records a failed check in the workspace error word (bit 0, and
+// `code` in word 1 if none was recorded yet), so that the caller skips the
+// access it guards and the host reads SAF_ERR_TIMEOUT-class status from
+// saf_device_status; in the regular build it is `true` and compiles away.
+#ifdef SAF_CHECKED
+__device__ __forceinline__ bool saf_checked_ok(unsigned int* err, bool cond, unsigned int code) {
+    if (!cond) {
+        atomicOr(err, 1u);
+        atomicCAS(err + 1, 0u, code);
+    }
+    return cond;
+}
+#define SAF_CHECKED_OK(err, cond, code) saf_checked_ok((err), (cond), (code))
+#else
+#define SAF_CHECKED_OK(err, cond, code) true
+#endif
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

@@ -391,6 +391,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const int w = (int)atomicAdd(p.err + kCtrFwdNext, 1u);
                 const int item = w < total ? w : -1;
                 const Item it = item >= 0 ? decode(item) : Item{0, 0, 0, 0, -1, false};
+                if (item >= 0 && !SAF_CHECKED_OK(p.err,
+                                                 it.bh >= 0 && it.bh < p.BH && it.I >= 0 && it.I < p.nqb && it.h >= 0 &&
+                                                     it.h < p.H && it.slot < p.nslots,
+                                                 0x9101u)) {
+                    ok = false;
+                    break;
+                }
                 if (!mbar_wait(bar_ite + 8 * (n & 1), ((n >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                 st_shared_v4(item_slot + 16 * (n & 1), (uint32_t)item, (uint32_t)it.bh, (uint32_t)it.I, (uint32_t)it.h);
                 mbar_arrive(bar_itf + 8 * (n & 1));
@@ -427,6 +434,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         }
                         if (g >= 2 && !mbar_wait(bar_pb + 8 * b, ((g >> 1) & 1) ^ 1, kWaitLimit)) { ok = false; break; }
                         const uint32_t st = sbase + SM_WST + b * WST_BYTES;
+                        if (!SAF_CHECKED_OK(p.err,
+                                            (size_t)(it.I - j) * BN + 256 <= (size_t)p.w.Lp &&
+                                                (size_t)j * 64 + 64 <= (size_t)p.w.Tp / 2,
+                                            0x9102u)) {
+                            ok = false;
+                            break;
+                        }
                         mbar_expect_tx(bar_wf + 8 * b, WST_BYTES);
                         bulk_load(st, p.w.epair + (size_t)it.slot * p.w.Lp + (size_t)(it.I - j) * BN, WST_E, bar_wf + 8 * b);
                         bulk_load(st + WST_E, p.w.cpair + (size_t)it.slot * (p.w.Tp / 2) + (size_t)j * 64,
