@@ -64,7 +64,7 @@ __device__ __forceinline__ void slot_flags(const ReplacedWs& w, int nslots, uint
 // longest).  Slices are taken kHeadGroup at a time, so the tiles they share
 // stay in L2, and inside a group the CTAs run longest first across all its
 // slices, so the last CTAs to start are the shortest and the tail is small.
-constexpr int kHeadGroup = 16;
+constexpr int kHeadGroup = 32;
 __host__ __device__ __forceinline__ void grouped_order(unsigned b, int BH, int nblk, int& bh, int& rank) {
     const unsigned per_group = (unsigned)kHeadGroup * (unsigned)nblk;
     const int g = (int)(b / per_group);

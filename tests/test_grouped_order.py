@@ -1,7 +1,7 @@
 """The work-item order shared by both persistent kernels (`grouped_order` in
 csrc/saf_common.cuh), compiled for the host from the same header and checked
 exhaustively: every item maps to a distinct (slice, block rank), all of them
-are covered, slices come in groups of 16 in order, and inside a group the
+are covered, slices come in groups of 32 in order, and inside a group the
 ranks never decrease (rank 0 is the longest block: the forward visits
 nqb - rank key blocks for its query block, the backward nqb - rank query
 blocks for its key block)."""
@@ -19,7 +19,7 @@ extern "C" void order_all(int BH, int nblk, int* bh, int* rank) {
     for (unsigned b = 0; b < (unsigned)(BH * nblk); ++b) saf::grouped_order(b, BH, nblk, bh[b], rank[b]);
 }
 """
-GROUP = 16
+GROUP = 32
 
 
 @pytest.fixture(scope="module")
