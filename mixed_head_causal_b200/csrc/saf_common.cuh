@@ -61,18 +61,22 @@ __device__ __forceinline__ void slot_flags(const ReplacedWs& w, int nslots, uint
 
 // CTA order of the tensor-core kernels.  A CTA does one block-row of one
 // (batch, head) slice; its work shrinks with its causal rank (rank 0 = the
-// longest).  Slices are taken kHeadGroup at a time, so the tiles they share
-// stay in L2, and inside a group the CTAs run longest first across all its
-// slices, so the last CTAs to start are the shortest and the tail is small.
-constexpr int kHeadGroup = 32;
+// longest).  Slices are taken a group at a time, so the tiles they share stay
+// in L2, and inside a group the CTAs run longest first across all its slices,
+// so the last CTAs to start are the shortest and the tail is small.  A group
+// holds about kGroupItems items: kGroupItems / nblk slices, at least one (32
+// slices of 1 MB of K and V at T = 4096, 16 of 2 MB at T = 8192).
+constexpr int kGroupItems = 1024;
+__host__ __device__ __forceinline__ int head_group(int nblk) { return nblk >= kGroupItems ? 1 : kGroupItems / nblk; }
 __host__ __device__ __forceinline__ void grouped_order(unsigned b, int BH, int nblk, int& bh, int& rank) {
-    const unsigned per_group = (unsigned)kHeadGroup * (unsigned)nblk;
+    const int group = head_group(nblk);
+    const unsigned per_group = (unsigned)group * (unsigned)nblk;
     const int g = (int)(b / per_group);
     const int r = (int)(b - (unsigned)g * per_group);
-    const int left = BH - g * kHeadGroup;  // slices in this group (the last one may be partial)
-    const int heads = left < kHeadGroup ? left : kHeadGroup;
+    const int left = BH - g * group;  // slices in this group (the last one may be partial)
+    const int heads = left < group ? left : group;
     rank = r / heads;
-    bh = g * kHeadGroup + (r - rank * heads);
+    bh = g * group + (r - rank * heads);
 }
 
 // ---------------------------------------------------------------- workspace

@@ -1,8 +1,8 @@
 """The work-item order shared by both persistent kernels (`grouped_order` in
 csrc/saf_common.cuh), compiled for the host from the same header and checked
 exhaustively: every item maps to a distinct (slice, block rank), all of them
-are covered, slices come in groups of 32 in order, and inside a group the
-ranks never decrease (rank 0 is the longest block: the forward visits
+are covered, slices come in groups of 1024 // nblk (at least one) in order,
+and inside a group the ranks never decrease (rank 0 is the longest block: the forward visits
 nqb - rank key blocks for its query block, the backward nqb - rank query
 blocks for its key block)."""
 import ctypes
@@ -19,7 +19,11 @@ extern "C" void order_all(int BH, int nblk, int* bh, int* rank) {
     for (unsigned b = 0; b < (unsigned)(BH * nblk); ++b) saf::grouped_order(b, BH, nblk, bh[b], rank[b]);
 }
 """
-GROUP = 32
+GROUP_ITEMS = 1024
+
+
+def group(nblk):
+    return max(1, GROUP_ITEMS // nblk)
 
 
 @pytest.fixture(scope="module")
@@ -42,13 +46,14 @@ def order(lib, BH, nblk):
 
 
 @pytest.mark.parametrize("BH", [1, 2, 15, 16, 17, 31, 32, 33, 96, 100, 384])
-@pytest.mark.parametrize("nblk", [1, 2, 3, 8, 32, 64])
+@pytest.mark.parametrize("nblk", [1, 2, 3, 8, 32, 64, 100, 128, 1024, 1500])
 def test_grouped_order_is_a_longest_first_bijection(order_lib, BH, nblk):
     bh, rank = order(order_lib, BH, nblk)
     pairs = list(zip(bh, rank))
     assert sorted(pairs) == [(h, r) for h in range(BH) for r in range(nblk)]
+    G = group(nblk)
     for b, (h, r) in enumerate(pairs):
-        g = b // (GROUP * nblk)
-        assert g * GROUP <= h < min(BH, (g + 1) * GROUP)  # its group, in order
-        if b > 0 and (b - 1) // (GROUP * nblk) == g:
+        g = b // (G * nblk)
+        assert g * G <= h < min(BH, (g + 1) * G)  # its group, in order
+        if b > 0 and (b - 1) // (G * nblk) == g:
             assert r >= rank[b - 1]  # longest first inside the group
