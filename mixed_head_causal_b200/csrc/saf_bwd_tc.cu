@@ -11,7 +11,7 @@
 //   warp 0      TMA producer: work items; K (two stages), V per item; Q, dO
 //               and the per-query vectors of each query block through an
 //               NQS-stage ring that runs on across items
-//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warp 1      TMEM owner and MMA issuer (one elected lane)
 //   warps 2..9  key rows, two warps per row quarter (query columns 0..63 and
 //               64..127 of each tile): P^T, dS^T, and the dK/dV epilogue
 //   warps 10..13 one query row per thread: dQ tile TMEM -> smem -> reduce-add
@@ -415,117 +415,139 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             if (item < 0) break;
             int okl = 1;
-            if (lane == 0) {
-                if (!it.rep) {
-                    // Ordinary heads run one tile ahead: S^T of tile t+1 is issued
-                    // right after dV_t (the last reader of the P^T columns it
-                    // overwrites) and dP^T of tile t+1 right after dQ_t, so the tensor
-                    // cores work on the next tile while the row threads finish this
-                    // one; an item's first S^T and dP^T go in while the row threads
-                    // still read out the previous item's dK, dV.  The tensor pipe
-                    // executes one thread's MMAs in order, which orders those reuses.
-                    const int kb = nk & 1;
-                    const uint64_t dK = dK0 + (uint64_t)kb * kStage;
-                    auto issue_s = [&](uint64_t dQn) {
+            // The whole warp runs the schedule (its waits give one answer for
+            // all lanes) and one elected lane issues each group of MMAs and their
+            // commits (always the same lane, so a commit covers all its MMAs).
+            if (!it.rep) {
+                // Ordinary heads run one tile ahead: S^T of tile t+1 is issued
+                // right after dV_t (the last reader of the P^T columns it
+                // overwrites) and dP^T of tile t+1 right after dQ_t, so the tensor
+                // cores work on the next tile while the row threads finish this
+                // one; an item's first S^T and dP^T go in while the row threads
+                // still read out the previous item's dK, dV.  The tensor pipe
+                // executes one thread's MMAs in order, which orders those reuses.
+                const int kb = nk & 1;
+                const uint64_t dK = dK0 + (uint64_t)kb * kStage;
+                auto issue_s = [&](uint64_t dQn) {
+                    if (elect_one()) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k) mma_ss(tmem + C_S, dK + 2 * k, dQn + 2 * k, idSS, k > 0);
                         mma_commit(bar_s);
-                    };
-                    // dP^T of the item's last tile is V's last reader: V's buffer is
-                    // released with it
-                    auto issue_dp = [&](uint64_t dDOn, bool last) {
+                    }
+                    __syncwarp();
+                };
+                // dP^T of the item's last tile is V's last reader: V's buffer is
+                // released with it
+                auto issue_dp = [&](uint64_t dDOn, bool last) {
+                    if (elect_one()) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k) mma_ss(tmem + C_DP, dVd + 2 * k, dDOn + 2 * k, idSS, k > 0);
                         mma_commit(bar_dp);
                         if (last) mma_commit(bar_ve);
-                    };
-                    if (!mbar_wait(bar_kf + 8 * kb, (nk >> 1) & 1, kWaitLimit) ||
-                        !mbar_wait(bar_qf + 8 * s, ph, kWaitLimit)) {
-                        report(p.err, 0x1201);
+                    }
+                    __syncwarp();
+                };
+                if (!mbar_wait_warp(bar_kf + 8 * kb, (nk >> 1) & 1, kWaitLimit) ||
+                    !mbar_wait_warp(bar_qf + 8 * s, ph, kWaitLimit)) {
+                    report(p.err, 0x1201);
+                    okl = 0;
+                } else {
+                    tc_fence_after();
+                    issue_s(dQ0 + (uint64_t)s * kStage);
+                    if (!mbar_wait_warp(bar_vf, nk & 1, kWaitLimit)) {
+                        report(p.err, 0x120a);
                         okl = 0;
                     } else {
                         tc_fence_after();
-                        issue_s(dQ0 + (uint64_t)s * kStage);
-                        if (!mbar_wait(bar_vf, nk & 1, kWaitLimit)) {
-                            report(p.err, 0x120a);
-                            okl = 0;
-                        } else {
-                            tc_fence_after();
-                            issue_dp(dDO0 + (uint64_t)s * kStage, it.ntiles == 1);
-                        }
+                        issue_dp(dDO0 + (uint64_t)s * kStage, it.ntiles == 1);
                     }
-                    for (int t = 0; okl && t < it.ntiles; ++t) {
-                        const bool wrap = (s + 1 == NQS);
-                        const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;  // tile t + 1
-                        const uint64_t dQs = dQ0 + (uint64_t)s * kStage, dDOs = dDO0 + (uint64_t)s * kStage;
-                        const uint32_t acc = t > 0 ? 1u : 0u;
-                        if (!mbar_wait(bar_p, go & 1, kWaitLimit)) { report(p.err, 0x1203); okl = 0; break; }
-                        // dV, dK start over: the previous item's must have been read out
-                        // (already implied: the row warps read them out before writing
-                        // this P^T; the wait is a cheap safeguard)
-                        if (t == 0 && n > 0 && !mbar_wait(bar_acr, (n - 1) & 1, kWaitLimit)) {
-                            report(p.err, 0x1209);
-                            okl = 0;
-                            break;
-                        }
-                        tc_fence_after();
+                }
+                for (int t = 0; okl && t < it.ntiles; ++t) {
+                    const bool wrap = (s + 1 == NQS);
+                    const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;  // tile t + 1
+                    const uint64_t dQs = dQ0 + (uint64_t)s * kStage, dDOs = dDO0 + (uint64_t)s * kStage;
+                    const uint32_t acc = t > 0 ? 1u : 0u;
+                    if (!mbar_wait_warp(bar_p, go & 1, kWaitLimit)) { report(p.err, 0x1203); okl = 0; break; }
+                    // dV, dK start over: the previous item's must have been read out
+                    // (already implied: the row warps read them out before writing
+                    // this P^T; the wait is a cheap safeguard)
+                    if (t == 0 && n > 0 && !mbar_wait_warp(bar_acr, (n - 1) & 1, kWaitLimit)) {
+                        report(p.err, 0x1209);
+                        okl = 0;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (elect_one()) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             mma_ts(tmem + C_DV, tmem + C_S + packed_kcol(k), dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
-                        const bool more = t + 1 < it.ntiles;
-                        if (more) {
-                            if (!mbar_wait(bar_qf + 8 * s1, ph1, kWaitLimit)) { report(p.err, 0x1207); okl = 0; break; }
-                            tc_fence_after();
-                            issue_s(dQ0 + (uint64_t)s1 * kStage);
-                        }
-                        if (!mbar_wait(bar_ds, go & 1, kWaitLimit)) { report(p.err, 0x1204); okl = 0; break; }
+                    }
+                    __syncwarp();
+                    const bool more = t + 1 < it.ntiles;
+                    if (more) {
+                        if (!mbar_wait_warp(bar_qf + 8 * s1, ph1, kWaitLimit)) { report(p.err, 0x1207); okl = 0; break; }
                         tc_fence_after();
+                        issue_s(dQ0 + (uint64_t)s1 * kStage);
+                    }
+                    if (!mbar_wait_warp(bar_ds, go & 1, kWaitLimit)) { report(p.err, 0x1204); okl = 0; break; }
+                    tc_fence_after();
+                    if (elect_one()) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             mma_ts(tmem + C_DK, tmem + C_DP + packed_kcol(k), dQs + 128 * k, idTS, k > 0 ? 1u : acc);
-                        const int b = go & 1;
-                        if (!mbar_wait(bar_dqe + 8 * b, ((go >> 1) & 1) ^ 1, kWaitLimit)) {
-                            report(p.err, 0x1205);
-                            okl = 0;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t cdq = b ? C_DQ1 : C_DQ0;
+                    }
+                    __syncwarp();
+                    const int b = go & 1;
+                    if (!mbar_wait_warp(bar_dqe + 8 * b, ((go >> 1) & 1) ^ 1, kWaitLimit)) {
+                        report(p.err, 0x1205);
+                        okl = 0;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t cdq = b ? C_DQ1 : C_DQ0;
+                    if (elect_one()) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k) mma_ss(tmem + cdq, dDS + 128 * k, dK + 128 * k, idDQ, k > 0);
                         mma_commit(bar_dqf + 8 * b);
-                        if (more) issue_dp(dDO0 + (uint64_t)s1 * kStage, t + 2 == it.ntiles);
-                        mma_commit(bar_qe + 8 * s);
-                        s = s1;
-                        ph = ph1;
-                        ++go;
                     }
-                    if (okl) {
+                    __syncwarp();
+                    if (more) issue_dp(dDO0 + (uint64_t)s1 * kStage, t + 2 == it.ntiles);
+                    if (elect_one()) mma_commit(bar_qe + 8 * s);
+                    __syncwarp();
+                    s = s1;
+                    ph = ph1;
+                    ++go;
+                }
+                if (okl) {
+                    if (elect_one()) {
                         mma_commit(bar_acc);
                         mma_commit(bar_ke + 8 * kb);
                     }
-                    ++nk;
-                } else {
-                    for (int t = 0; okl && t < it.ntiles; ++t) {
-                        const bool wrap = (s + 1 == NQS);
-                        const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;
-                        const uint64_t dDOs = dDO0 + (uint64_t)s * kStage;
-                        const uint32_t acc = t > 0 ? 1u : 0u;
-                        if (!mbar_wait(bar_qf + 8 * s, ph, kWaitLimit)) { report(p.err, 0x1202); okl = 0; break; }
-                        if (!mbar_wait(bar_pb + 8 * (gr & 1), (gr >> 1) & 1, kWaitLimit)) {
-                            report(p.err, 0x1206);
-                            okl = 0;
-                            break;
-                        }
-                        if (t == 0 && n > 0 && !mbar_wait(bar_acr, (n - 1) & 1, kWaitLimit)) {
-                            report(p.err, 0x1209);
-                            okl = 0;
-                            break;
-                        }
-                        tc_fence_after();
-                        // W of this tile sits in buffer gr & 1 (the S^T or the dP^T
-                        // columns, both unused by a replaced head): hi, then lo
-                        const uint32_t wcol = C_S + 128 * (gr & 1);
+                    __syncwarp();
+                }
+                ++nk;
+            } else {
+                for (int t = 0; okl && t < it.ntiles; ++t) {
+                    const bool wrap = (s + 1 == NQS);
+                    const int s1 = wrap ? 0 : s + 1, ph1 = wrap ? ph ^ 1 : ph;
+                    const uint64_t dDOs = dDO0 + (uint64_t)s * kStage;
+                    const uint32_t acc = t > 0 ? 1u : 0u;
+                    if (!mbar_wait_warp(bar_qf + 8 * s, ph, kWaitLimit)) { report(p.err, 0x1202); okl = 0; break; }
+                    if (!mbar_wait_warp(bar_pb + 8 * (gr & 1), (gr >> 1) & 1, kWaitLimit)) {
+                        report(p.err, 0x1206);
+                        okl = 0;
+                        break;
+                    }
+                    if (t == 0 && n > 0 && !mbar_wait_warp(bar_acr, (n - 1) & 1, kWaitLimit)) {
+                        report(p.err, 0x1209);
+                        okl = 0;
+                        break;
+                    }
+                    tc_fence_after();
+                    // W of this tile sits in buffer gr & 1 (the S^T or the dP^T
+                    // columns, both unused by a replaced head): hi, then lo
+                    const uint32_t wcol = C_S + 128 * (gr & 1);
+                    if (elect_one()) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             mma_ts(tmem + C_DV, tmem + wcol + 8 * k, dDOs + 128 * k, idTS, k > 0 ? 1u : acc);
@@ -534,14 +556,18 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                             mma_ts(tmem + C_DV, tmem + wcol + 64 + 8 * k, dDOs + 128 * k, idTS, 1u);
                         mma_commit(bar_wb + 8 * (gr & 1));
                         mma_commit(bar_qe + 8 * s);
-                        s = s1;
-                        ph = ph1;
-                        ++gr;
                     }
-                    if (okl) mma_commit(bar_acc);
+                    __syncwarp();
+                    s = s1;
+                    ph = ph1;
+                    ++gr;
+                }
+                if (okl) {
+                    if (elect_one()) mma_commit(bar_acc);
+                    __syncwarp();
                 }
             }
-            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            ok = okl != 0;  // the same in every lane
         }
     } else if (warp < 10) {
         // ------------------------------------------------ key rows

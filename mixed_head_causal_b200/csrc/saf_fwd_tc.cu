@@ -6,7 +6,7 @@
 //   warp 0      TMA producer: Q once, then K and V tiles of 128 keys through
 //               separate rings (2 K stages, 2 V stages), K one block ahead of
 //               V (K is skipped for replaced heads)
-//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warp 1      TMEM owner and MMA issuer (one elected lane)
 //   warps 2..5  one query row per thread: softmax / pattern builder, epilogue
 //
 // Ordinary head, per key block j (FlashAttention-style online softmax, the
@@ -477,40 +477,46 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (!ok) { if (lane == 0) report(p.err, 0x205); break; }
             if (item < 0) break;
             const int nkb = it.I + 1;
-            if (lane == 0) {
+            // The whole warp runs the schedule (its waits give one answer for
+            // all lanes) and one elected lane issues each group of MMAs and their
+            // commits (always the same lane, so a commit covers all its MMAs).
+            {
                 const int b = nq & 1;
                 const uint64_t dq = dQ0 + (uint64_t)b * kStage;
                 // S_j = Q K_j^T into the S columns; frees K stage j when done,
                 // and the Q buffer after the item's last block
                 auto issue_s = [&](int j) -> bool {
                     const int g = gk + j, s = g % NSK, u = g / NSK;
-                    if (!mbar_wait(bar_kf + 8 * s, u & 1, kWaitLimit)) return false;
+                    if (!mbar_wait_warp(bar_kf + 8 * s, u & 1, kWaitLimit)) return false;
                     tc_fence_after();
                     const uint64_t dk = dK0 + (uint64_t)s * kStage;
+                    if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
-                        mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
-                    mma_commit(bar_s);
-                    mma_commit(bar_ke + 8 * s);
-                    if (j == nkb - 1) mma_commit(bar_qe + 8 * b);
+                        for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
+                            mma_ss(tmem + TS_COL, dq + 2 * k, dk + 2 * k, idS, k > 0 ? 1u : 0u);
+                        mma_commit(bar_s);
+                        mma_commit(bar_ke + 8 * s);
+                        if (j == nkb - 1) mma_commit(bar_qe + 8 * b);
+                    }
+                    __syncwarp();
                     return true;
                 };
-                if (!it.rep) ok = mbar_wait(bar_qf + 8 * b, (nq >> 1) & 1, kWaitLimit) && issue_s(0);
+                if (!it.rep) ok = mbar_wait_warp(bar_qf + 8 * b, (nq >> 1) & 1, kWaitLimit) && issue_s(0);
                 if (!ok) report(p.err, 0x201);
                 for (int j = 0; ok && j < nkb; ++j) {
                     if (!it.rep && j + 1 < nkb) {
                         // S_{j+1} once the rows have copied S_j out of TMEM
-                        if (!mbar_wait(bar_sf, (go + j) & 1, kWaitLimit) || !issue_s(j + 1)) {
+                        if (!mbar_wait_warp(bar_sf, (go + j) & 1, kWaitLimit) || !issue_s(j + 1)) {
                             report(p.err, 0x202);
                             ok = false;
                             break;
                         }
                     }
                     const int g = gv + j, s = g % NSV, u = g / NSV;
-                    if (!mbar_wait(bar_vf + 8 * s, u & 1, kWaitLimit)) { report(p.err, 0x203); ok = false; break; }
+                    if (!mbar_wait_warp(bar_vf + 8 * s, u & 1, kWaitLimit)) { report(p.err, 0x203); ok = false; break; }
                     const int wb = (gr + j) & 1;
-                    if (!(it.rep ? mbar_wait(bar_pb + 8 * wb, ((gr + j) >> 1) & 1, kWaitLimit)
-                                 : mbar_wait(bar_p, (go + j) & 1, kWaitLimit))) {
+                    if (!(it.rep ? mbar_wait_warp(bar_pb + 8 * wb, ((gr + j) >> 1) & 1, kWaitLimit)
+                                 : mbar_wait_warp(bar_p, (go + j) & 1, kWaitLimit))) {
                         report(p.err, 0x204);
                         ok = false;
                         break;
@@ -520,20 +526,22 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     // a replaced head's W alternates between two buffers in the S
                     // columns (unused there), so building W_{j+1} overlaps this MMA
                     const uint32_t acol = it.rep ? 64 * wb : TP_COL;
+                    if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
-                        mma_ts(tmem + TO_COL, tmem + acol + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
-                    if (it.rep) {
+                        for (int k = 0; k < 8; ++k)  // K = 128 keys in steps of 16 (16 rows x 128 B)
+                            mma_ts(tmem + TO_COL, tmem + acol + 8 * k, dv + 128 * k, idO, (j > 0 || k > 0) ? 1u : 0u);
+                        if (it.rep) {
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)  // row sums of the same W
-                            mma_ts(tmem + TSUM_COL, tmem + acol + 8 * k, dOnes + 2 * (k & 3), idSum,
-                                   (j > 0 || k > 0) ? 1u : 0u);
+                            for (int k = 0; k < 8; ++k)  // row sums of the same W
+                                mma_ts(tmem + TSUM_COL, tmem + acol + 8 * k, dOnes + 2 * (k & 3), idSum,
+                                       (j > 0 || k > 0) ? 1u : 0u);
+                        }
+                        mma_commit(it.rep ? bar_ob + 8 * wb : bar_o);
+                        mma_commit(bar_ve + 8 * s);
                     }
-                    mma_commit(it.rep ? bar_ob + 8 * wb : bar_o);
-                    mma_commit(bar_ve + 8 * s);
+                    __syncwarp();
                 }
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
             if (it.rep) {
                 gr += nkb;
             } else {

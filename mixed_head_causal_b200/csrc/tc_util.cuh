@@ -56,6 +56,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
         if (clock64() - t0 > limit_cycles) return false;
     }
 }
+// mbar_wait by a whole warp with one answer for all its lanes.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, long long limit_cycles) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_cycles));
+}
+
+// True in one lane of a converged warp (the lowest, so the same lane each
+// time the whole warp runs it).  Single-thread tcgen05 issue goes under this
+// test rather than `lane == 0`: measured on B200, M = 128 MMAs with N <= 128
+// issued under `lane == 0` take about 60 cycles each whatever their size,
+// under elect.sync they run at the tensor pipe's rate (32 cycles at N = 64).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
 
 // ------------------------------------------------------------------ TMA
 // 3-D tiled load [x, y, z] -> shared memory, completion on an mbarrier.
