@@ -182,7 +182,7 @@ SAF_API saf_status saf_mixed_attn_bwd_gqa(const void *q, const void *k, const vo
  * need only per-row scratch, not the tensor-core (tcgen05) backward, whose
  * fp32 dQ accumulator of B*H*T*64 floats no fixed array of modest size can
  * hold.  Measured on one B200 at B=8, H=12, T=4096 (3 heads replaced, bf16
- * gradients): 2.81 ms against 0.72 ms for saf_mixed_attn_bwd.  Its
+ * gradients): 2.81 ms against 0.60 ms for saf_mixed_attn_bwd.  Its
  * scratch (the per-row terms rowsum(dO o O), and the replaced heads' log Z
  * when logz is NULL) lives in one 8 MiB array of device memory inside the
  * library, one per GPU, held from load until process exit.  Limit:
