@@ -376,6 +376,8 @@ def rates(w, t, pk):
     res["tokens_per_s"] = w.tokens / (t["step_ms"] * 1e-3)
     res["tflops"] = fl["total"] / (t["step_ms"] * 1e-3) / 1e12
     res["frac_of_peak"] = res["tflops"] / pk["bf16_tflops"]
+    if w.backward:  # the ordinary backward's four products, no recompute of Q K^T
+        res["tflops_strict"] = I.flops(w, strict=True)["total"] / (t["step_ms"] * 1e-3) / 1e12
     res["fwd_tflops"] = fl["fwd"] / (t["fwd_ms"] * 1e-3) / 1e12
     if w.backward:
         res["bwd_tflops"] = fl["bwd"] / (t["bwd_ms"] * 1e-3) / 1e12
@@ -478,6 +480,8 @@ def our_arm(args, world, rank, local):
     value = tokens / (ms_step * 1e-3)
     fl = I.flops(w)
     tflops = fl["total"] * world / (ms_step * 1e-3) / 1e12
+    # the same time against the strict count (ordinary backward without the recompute of Q K^T)
+    tflops_strict = I.flops(w, strict=True)["total"] * world / (ms_step * 1e-3) / 1e12
 
     # ---- per-kernel timing (separate pass, same steps, events around each launch)
     prof_steps = min(args.steps, 20)
@@ -601,6 +605,7 @@ def our_arm(args, world, rank, local):
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "tflops": tflops, "tflops_frac_of_peak": tflops / pk["bf16_tflops"],
+            "tflops_strict": tflops_strict, "tflops_strict_frac_of_peak": tflops_strict / pk["bf16_tflops"],
             "config": arm_config(w, world, args.grad_dtype),
             "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
             "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,

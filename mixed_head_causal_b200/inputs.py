@@ -158,11 +158,12 @@ def make_inputs(w: Workload, seed: int = 0, tensors: Iterable[str] = ("q", "k", 
     return out
 
 
-def flops(w: Workload, backward: Optional[bool] = None) -> Dict[str, float]:
+def flops(w: Workload, backward: Optional[bool] = None, strict: bool = False) -> Dict[str, float]:
     """Algorithmic flop counts, causal T^2/2 convention.
 
     Ordinary head: forward 2*d*T^2 (QK^T and PV), backward 5*d*T^2 (five
-    T x T x d contractions counting the recompute of QK^T).  Replaced head:
+    T x T x d contractions counting the recompute of QK^T; `strict` counts
+    the method's own four, 4*d*T^2, without the recompute).  Replaced head:
     forward d*T^2 (PV only), backward d*T^2 (P^T dO only).
     """
     if backward is None:
@@ -171,5 +172,5 @@ def flops(w: Workload, backward: Optional[bool] = None) -> Dict[str, float]:
     n_o = w.H - n_r
     unit = float(w.d) * w.T * w.T * w.B
     fwd = unit * (2 * n_o + 1 * n_r)
-    bwd = unit * (5 * n_o + 1 * n_r) if backward else 0.0
+    bwd = unit * ((4 if strict else 5) * n_o + 1 * n_r) if backward else 0.0
     return {"fwd": fwd, "bwd": bwd, "total": fwd + bwd}

@@ -44,3 +44,9 @@ def test_flops_convention():
     w = I.WORKLOADS["124m_b8_t4096_r25"]
     f = I.flops(w)
     assert abs(f["total"] - 8 * (9 * 7 + 3 * 2) * 64 * 4096 ** 2) < 1
+    # the strict count drops the backward's recompute of Q K^T: ordinary 6 units, replaced 2
+    s = I.flops(w, strict=True)
+    assert abs(s["total"] - 8 * (9 * 6 + 3 * 2) * 64 * 4096 ** 2) < 1
+    assert s["fwd"] == f["fwd"]
+    fo = I.flops(I.WORKLOADS["prefill_124m_b64_t4096"], strict=True)
+    assert fo["bwd"] == 0.0 and fo["total"] == I.flops(I.WORKLOADS["prefill_124m_b64_t4096"])["total"]
