@@ -56,31 +56,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
         if (clock64() - t0 > limit_cycles) return false;
     }
 }
-// mbar_try_wait with a suspend-time hint: the thread may sleep (up to `ns`)
-// until the phase completes instead of polling.
-__device__ __forceinline__ bool mbar_try_wait_s(uint32_t bar, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.b32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_s(uint32_t bar, uint32_t parity, long long limit_cycles) {
-    if (mbar_try_wait_s(bar, parity, 0x989680u)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try_wait_s(bar, parity, 0x989680u)) return true;
-        if (clock64() - t0 > limit_cycles) return false;
-    }
-}
-__device__ __forceinline__ bool mbar_wait_warp_s(uint32_t bar, uint32_t parity, long long limit_cycles) {
-    return __all_sync(0xffffffffu, mbar_wait_s(bar, parity, limit_cycles));
-}
-
 // mbar_wait by a whole warp with one answer for all its lanes.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, long long limit_cycles) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_cycles));
