@@ -589,11 +589,12 @@ def our_arm(args, world, rank, local):
     # ---- the pass split of the headline shape, the other shapes and the
     # per-head cost (separate timings after the headline; milliseconds each)
     split = rates(w, time_passes(w, dev, x, 20, gd), pk)
-    extra, hc = None, None
+    extra, hc, sec = None, None, None
     if rank == 0 and not args.no_extra:
         extra = per_config(dev, pk)
         if w.backward and n_r:
             hc = head_cost_fit(w, dev)
+        sec = secondary(w, dev, x)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -609,7 +610,7 @@ def our_arm(args, world, rank, local):
             "config": arm_config(w, world, args.grad_dtype),
             "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
             "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
-            "passes": split, "per_config": extra, "head_cost": hc,
+            "passes": split, "per_config": extra, "head_cost": hc, "secondary": sec,
         }
         print(json.dumps(line), flush=True)
 
@@ -636,63 +637,50 @@ def _time(fn, steps):
     return e0.elapsed_time(e1) / steps
 
 
-def pattern_grad_cost(args, local):
-    """Trainable-pattern gradient of the workload's replaced heads: time per
-    call (log Z given), and the dP contraction's algorithmic TFLOP/s (one
-    causal T x T x d unit per replaced (b, h); the kernel runs it twice)
-    against the measured bf16 peak."""
+def pattern_grad_stats(w, x, reps):
+    """Trainable-pattern gradient of w's replaced heads on the inputs x (on
+    the device): ms per call (log Z given) and the dP contraction's
+    algorithmic TFLOP/s (one causal T x T x d unit per replaced (b, h); the
+    kernel runs it twice) against the bf16 peak."""
     from mixed_head_causal_b200 import saf
-    dev = torch.device("cuda", local)
-    w = I.WORKLOADS[args.workload]
-    x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
     mask = x["mask"]
-    n_r = int(mask.sum())
+    n_r = int(torch.as_tensor(mask).sum())
     lz = saf.replaced_lognorm(x["alpha"], x["rho"], mask)
-    da = torch.empty(w.H, w.T, dtype=torch.float32, device=dev)
+    da = torch.empty(w.H, w.T, dtype=torch.float32, device=x["v"].device)
     dr = torch.empty_like(da)
     ms = _time(lambda: saf.replaced_pattern_grad(x["v"], x["do"], x["alpha"], x["rho"], mask, logz=lz, da=da,
-                                                 dr=dr), args.steps)
-    flops = w.B * n_r * w.d * float(w.T) ** 2
+                                                 dr=dr), reps)
     pk = peaks()
-    tf = flops / (ms * 1e-3) / 1e12
-    print(json.dumps({"metric": "trainable-pattern gradient (dalpha, drho) ms per call", "value": ms, "unit": "ms",
-                      "higher_is_better": False,
-                      "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "n_replaced": n_r},
-                      "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                                   "frac": tf / pk["bf16_tflops"], "path": "warp-level mma.sync, two passes"}}),
-          flush=True)
+    tf = w.B * n_r * w.d * float(w.T) ** 2 / (ms * 1e-3) / 1e12
+    return {"ms": ms, "n_replaced": n_r,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / pk["bf16_tflops"], "path": "warp-level mma.sync, two passes"}}
 
 
-def calibration_cost(args, local):
-    """Calibration statistics over the workload's B sequences (every head
-    ordinary): ms per call and the score contraction's algorithmic TFLOP/s
+def calibration_stats(w, x, reps):
+    """Calibration statistics over w's B sequences of q, k (every head taken
+    as ordinary): ms per call and the score contraction's algorithmic TFLOP/s
     (one causal T x T x d unit per (sample, head); the kernel runs it twice)."""
     from mixed_head_causal_b200 import saf
-    dev = torch.device("cuda", local)
-    w = I.custom(I.WORKLOADS[args.workload].B, I.WORKLOADS[args.workload].H, I.WORKLOADS[args.workload].T, [])
-    x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
-    _, lse = saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], x["mask"])
-    a_hat = torch.empty(w.H, w.T, w.T, dtype=torch.float32, device=dev)
-    svar = torch.empty(w.H, dtype=torch.float32, device=dev)
-    ms = _time(lambda: saf.attn_calibration(x["q"], x["k"], lse, a_hat=a_hat, svar=svar), args.steps)
-    flops = w.B * w.H * w.d * float(w.T) ** 2
+    mask0 = torch.zeros(w.H, dtype=torch.bool)
+    _, lse0 = saf.mixed_attn_fwd(x["q"], x["k"], x["v"], x["alpha"], x["rho"], mask0)
+    a_hat = torch.empty(w.H, w.T, w.T, dtype=torch.float32, device=x["q"].device)
+    svar = torch.empty(w.H, dtype=torch.float32, device=x["q"].device)
+    ms = _time(lambda: saf.attn_calibration(x["q"], x["k"], lse0, a_hat=a_hat, svar=svar), reps)
     pk = peaks()
-    tf = flops / (ms * 1e-3) / 1e12
-    print(json.dumps({"metric": "calibration statistics (A_hat, s_var) ms per call", "value": ms, "unit": "ms",
-                      "higher_is_better": False,
-                      "config": {"workload": w.name, "N": w.B, "H": w.H, "T": w.T},
-                      "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                                   "frac": tf / pk["bf16_tflops"], "path": "warp-level mma.sync, two passes",
-                                   "a_hat_bytes": 4 * w.H * w.T * w.T}}), flush=True)
+    tf = w.B * w.H * w.d * float(w.T) ** 2 / (ms * 1e-3) / 1e12
+    del a_hat
+    return {"ms": ms, "N": w.B,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / pk["bf16_tflops"], "path": "warp-level mma.sync, two passes",
+                         "a_hat_bytes": 4 * w.H * w.T * w.T}}
 
 
-def fit_cost(args, local):
-    """Pattern fitting (400 Adam steps) of the workload's replaced heads, the
-    targets being their own patterns (dense [T, T] fp32, built on the GPU from
-    the pattern vectors by the forward with V = I in 128-row slabs)."""
+def fit_stats(w, dev):
+    """Pattern fitting (400 Adam steps) of w's replaced heads, the targets
+    being their own patterns (dense [T, T] fp32, built on the GPU from the
+    pattern vectors): ms per call and the final mean row KL of each head."""
     from mixed_head_causal_b200 import saf
-    dev = torch.device("cuda", local)
-    w = I.WORKLOADS[args.workload]
     a, r = I.make_pattern(w, 0)
     heads = I.replaced_heads(w)
     T = w.T
@@ -707,16 +695,62 @@ def fit_cost(args, local):
             logit = ah[j.expand(ii.shape[0], T)] + rh[(ii - j).clamp(min=0)] - lz[h][ii]
             targets[s_, i0:i0 + 512] = torch.where(j <= ii, torch.exp(logit), torch.zeros((), device=dev))
     torch.cuda.synchronize()
-    t0 = time.perf_counter()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     _, _, kl = saf.fit_pattern(targets, steps=400, lr=0.1)
     e1.record()
     torch.cuda.synchronize()
-    print(json.dumps({"metric": "pattern fitting, 400 Adam steps, ms per call", "value": e0.elapsed_time(e1),
+    del targets
+    return {"ms": e0.elapsed_time(e1), "heads": len(heads), "steps": 400, "kl": [float(v) for v in kl.cpu()]}
+
+
+def secondary(w, dev, x, reps=10):
+    """The entry points beside the layer (trainable-pattern gradient,
+    calibration statistics, pattern fitting) timed on the headline shape."""
+    out = {"workload": w.name}
+    if w.backward and int(torch.as_tensor(x["mask"]).sum()):
+        out["pattern_grad"] = pattern_grad_stats(w, x, reps)
+        out["fit"] = fit_stats(w, dev)
+    out["calibration"] = calibration_stats(w, x, reps)
+    torch.cuda.empty_cache()
+    return out
+
+
+def pattern_grad_cost(args, local):
+    """`--pattern-grad`: pattern_grad_stats on the workload's seeded inputs."""
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS[args.workload]
+    x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
+    st = pattern_grad_stats(w, x, args.steps)
+    print(json.dumps({"metric": "trainable-pattern gradient (dalpha, drho) ms per call", "value": st["ms"],
                       "unit": "ms", "higher_is_better": False,
-                      "config": {"workload": w.name, "heads": len(heads), "T": T},
-                      "kl": [float(x) for x in kl.cpu()], "wall_s": time.perf_counter() - t0}), flush=True)
+                      "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "n_replaced": st["n_replaced"]},
+                      "roofline": st["roofline"]}), flush=True)
+
+
+def calibration_cost(args, local):
+    """`--calibration`: calibration_stats over the workload's B sequences."""
+    dev = torch.device("cuda", local)
+    base = I.WORKLOADS[args.workload]
+    w = I.custom(base.B, base.H, base.T, [])
+    x = {k: (v.to(dev) if k != "mask" else v) for k, v in I.make_inputs(w, 0, threads=16).items()}
+    st = calibration_stats(w, x, args.steps)
+    print(json.dumps({"metric": "calibration statistics (A_hat, s_var) ms per call", "value": st["ms"],
+                      "unit": "ms", "higher_is_better": False,
+                      "config": {"workload": w.name, "N": w.B, "H": w.H, "T": w.T}, "roofline": st["roofline"]}),
+          flush=True)
+
+
+def fit_cost(args, local):
+    """`--fit`: fit_stats for the workload's replaced heads."""
+    dev = torch.device("cuda", local)
+    w = I.WORKLOADS[args.workload]
+    t0 = time.perf_counter()
+    st = fit_stats(w, dev)
+    print(json.dumps({"metric": "pattern fitting, 400 Adam steps, ms per call", "value": st["ms"],
+                      "unit": "ms", "higher_is_better": False,
+                      "config": {"workload": w.name, "heads": st["heads"], "T": w.T},
+                      "kl": st["kl"], "wall_s": time.perf_counter() - t0}), flush=True)
 
 
 def gqa_cost(args, local):
