@@ -1,11 +1,15 @@
 // Mixed-head causal attention forward on the 5th-generation tensor cores
 // (tcgen05, accumulators in TMEM, operands staged by TMA).
 //
-// One CTA computes one 128-row query block of one (batch, head) slice; both
-// head kinds share the grid, which is ordered longest rows first.  Warp roles:
-//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys through
-//               separate rings (2 K stages, 2 V stages), K one block ahead of
-//               V (K is skipped for replaced heads)
+// A work item is one 128-row query block of one (batch, head) slice; both
+// head kinds share the item stream.  The kernel is persistent: two CTAs per SM
+// pull items from a counter in the workspace header (reset by the last CTA),
+// in groups of slices with the longest rows first inside a group.  Warp roles:
+//   warp 0      TMA producer: work items (decoded, through a two-slot ring);
+//               Q per item (two buffers: this item and the next), then K and
+//               V tiles of 128 keys through separate rings (2 K stages, 2 V
+//               stages), K one block ahead of V (K is skipped for replaced
+//               heads, whose blocks' W inputs come through a two-stage ring)
 //   warp 1      TMEM owner and MMA issuer (one elected lane)
 //   warps 2..5  one query row per thread: softmax / pattern builder, epilogue
 //
