@@ -74,7 +74,7 @@ typedef enum saf_status {
 } saf_status;
 
 /* Human-readable name of a status code (static string; never NULL). */
-SAF_API const char *saf_status_string(int status);
+SAF_API const char *saf_status_string(saf_status status);
 
 /* Library version, as major*10000 + minor*100 + patch. */
 SAF_API int saf_version(void);

@@ -65,8 +65,8 @@ bool force_mma_path() {
 
 extern "C" {
 
-const char* saf_status_string(int status) {
-    switch (status) {
+const char* saf_status_string(saf_status status) {
+    switch ((int)status) {  // any int a C caller passes, known or not
         case SAF_OK: return "SAF_OK";
         case SAF_ERR_INVALID_ARG: return "SAF_ERR_INVALID_ARG";
         case SAF_ERR_UNSUPPORTED: return "SAF_ERR_UNSUPPORTED";
