@@ -686,7 +686,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     if (!it.direct) {
                         const float* ef = p.w.ef + (size_t)it.slot * p.w.Lp + 128 + (I - it.J) * BM - jl;
                         // the 64 entries this thread reads lie inside the slot's padded array
-                        const int e_lo = 128 + (I - it.J) * BM - jl + 64 * half;
+                        [[maybe_unused]] const int e_lo = 128 + (I - it.J) * BM - jl + 64 * half;
                         const bool win_ok = SAF_CHECKED_OK(p.err, e_lo >= 0 && e_lo + 64 <= p.w.Lp, 0x9204u);
 #pragma unroll
                         for (int cc = 0; cc < 2; ++cc) {
